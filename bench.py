@@ -1,0 +1,417 @@
+#!/usr/bin/env python
+"""LSTM forward (+ BPTT) throughput on B200 through the C-ABI library.
+
+One step is one pass of the whole hot path over one batch of synthetic input:
+the input projection, the persistent recurrence of every layer, and (for the
+training workload, the default) the BPTT recurrence, the weight-gradient and
+input-gradient GEMMs, plus a gradient all-reduce when N > 1.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c5]
+    python bench.py --impl reference ...   # the CPU oracle, timed on host cores
+
+Prints one JSON line (rank 0).  `value` is whole-job sequence tokens/s
+(batch x seq_len per step, summed over ranks) with inputs resident on the
+device; `e2e` is the same metric with the inputs copied from pinned host
+memory and the results read back every step.  L2 is flushed (a 256 MiB write)
+between timed steps, outside the timed events.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from layer_lstm_b200.workloads import DESCRIPTIONS, WORKLOADS, make_inputs, select_rows  # noqa: E402
+
+FFMA_LANES_PER_SM = 128
+SM_COUNT = 148
+SM_MAX_MHZ = 1965.0
+TF32_OVER_BF16 = 1.1 / 2.25   # nominal dense tf32 / bf16 ratio
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="c5")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
+                    bf16_tflops_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+# --------------------------------------------------------------- work model
+def kernel_work(wl, kind):
+    """Algorithmic work of all launches of `kind` in one step: (units, amount).
+
+    Recurrences and GEMMs count 2 flops per multiply-add of the matrix
+    products the method defines (elementwise gate math is not counted)."""
+    B, T, H, D, L, G = wl.B, wl.T, wl.H, wl.D, wl.L, 4 * wl.H
+    ins = [wl.in_size(k) for k in range(L)]
+    if kind == "fwd_rec":
+        return "flop", 2.0 * B * T * D * G * H * L
+    if kind == "bwd_rec":
+        return "flop", 2.0 * B * T * D * G * H * L
+    if kind == "proj_gemm":
+        return "flop", sum(2.0 * B * T * D * G * i for i in ins)
+    if kind == "dw_gemm":
+        return "flop", sum(2.0 * B * T * D * G * (i + H) for i in ins)
+    if kind == "dx_gemm":
+        return "flop", sum(2.0 * B * T * D * G * i for i in ins)
+    return None, 0.0
+
+
+# Bound and peak of each kernel kind as the library implements it.
+#   alu:    FP32 FMA on the CUDA cores, 148 SMs x 128 lanes x 2 flop x max SM clock
+#   tensor: tcgen05 tensor cores (peak from the measured cuBLAS bf16 figure)
+KIND_BOUND = {"fwd_rec": "alu", "bwd_rec": "alu", "proj_gemm": "alu", "dw_gemm": "alu",
+              "dx_gemm": "alu"}
+
+
+def alu_peak_tflops():
+    return SM_COUNT * FFMA_LANES_PER_SM * 2 * SM_MAX_MHZ * 1e6 / 1e12
+
+
+def traffic_for(kind, wl_name):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source (profiles/ncu_traffic.json records the source
+    hash); otherwise None."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kind)
+    if not e or e.get("workload") != wl_name:
+        return None
+    src = os.path.join(ROOT, e["source"])
+    if not os.path.exists(src):
+        return None
+    with open(src, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    if sha != e.get("source_sha"):
+        return None
+    return float(e["bytes_per_launch"])
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="lstm_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------ CPU oracle
+def cpu_oracle_rate(wl, rows_target=None, min_seconds=10.0):
+    """Times the oracle (as it stands) on a bounded sample of batch rows of the
+    workload; returns (tokens/s, cores, sample description, seconds)."""
+    import oracle
+    threads = oracle.num_threads()
+    inp = make_inputs(wl)
+    nrows = rows_target or min(wl.B, max(1, threads))
+    while True:
+        sub = select_rows(inp, list(range(nrows)))
+        t0 = time.perf_counter()
+        oracle.run_inputs(sub, backward=wl.train)
+        dt = time.perf_counter() - t0
+        if dt >= min_seconds or nrows >= wl.B or rows_target is not None:
+            break
+        nrows = min(wl.B, nrows * 2)
+    cores = min(threads, nrows)
+    kind = "forward + BPTT" if wl.train else "forward"
+    sample = f"{nrows} of {wl.B} batch rows, full T/L/H, {kind}, float64"
+    return nrows * wl.T / dt, cores, sample, dt
+
+
+# ------------------------------------------------------------------ arms
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def run_reference(args):
+    world, rank, _ = dist_setup(args)
+    if rank != 0:
+        return
+    wl = WORKLOADS[args.workload]
+    import oracle
+    threads = oracle.num_threads()
+    inp = make_inputs(wl)
+    nrows = min(wl.B, max(1, threads))
+    sub = select_rows(inp, list(range(nrows)))
+    for _ in range(args.warmup):
+        oracle.run_inputs(sub, backward=wl.train)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.run_inputs(sub, backward=wl.train)
+    dt = time.perf_counter() - t0
+    value = nrows * wl.T * args.steps / dt
+    sample = f"{nrows} of {wl.B} batch rows per step, full T/L/H, float64"
+    line = {
+        "impl": "reference", "metric": "sequence tokens/s", "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(wl, args.gpus),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": min(threads, nrows),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(wl, n):
+    return {"workload": f"{wl.name}: {DESCRIPTIONS[wl.name]}", "global_batch": wl.B * n,
+            "seq_len": wl.T, "layers": wl.L, "hidden": wl.H, "input": wl.I,
+            "bidirectional": wl.D == 2, "train": wl.train, "parallelism": f"dp{n}",
+            "l2": "flushed between timed steps (256 MiB write)"}
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from layer_lstm_b200 import binding
+    from layer_lstm_b200.runner import DeviceProblem
+
+    world, rank, local = dist_setup(args)
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    binding.load()
+    wl = WORKLOADS[args.workload]
+    inp = make_inputs(wl)
+    prob = DeviceProblem(inp, device=f"cuda:{local}")
+    grads = []
+    if wl.train:
+        grads = prob.dw_ih + prob.dw_hh + (prob.db_ih if wl.bias else [])
+        flat = torch.empty(sum(g.numel() for g in grads), device=prob.x.device, dtype=torch.float32)
+        off = 0
+        views = []
+        for g in grads:
+            v = flat[off:off + g.numel()].view_as(g)
+            off += g.numel()
+            views.append(v)
+        n_ih = len(prob.dw_ih)
+        prob.dw_ih = views[:n_ih]
+        prob.dw_hh = views[n_ih:2 * n_ih]
+        if wl.bias:
+            prob.db_ih = views[2 * n_ih:]
+            prob.db_hh = [torch.empty_like(v) for v in prob.db_ih]
+        grad_flat = flat
+    stream = torch.cuda.current_stream()
+
+    def step():
+        prob.step(stream)
+        if wl.train and world > 1:
+            dist.all_reduce(grad_flat)
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=prob.x.device)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = prob.status(stream)
+    if st != binding.LSTM_OK:
+        raise binding.LstmError(st, "warm-up")
+
+    # ------------------------------------------------ device-resident timing
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    binding.lstm_timing_reset()
+    binding.lstm_timing_enable(True)
+    for i in range(args.steps):
+        flush.zero_()
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    binding.lstm_timing_enable(False)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    st = prob.status(stream)
+    if st != binding.LSTM_OK:
+        raise binding.LstmError(st, "timed steps")
+    kern = binding.lstm_timing_read()
+    total_ms = sum(a.elapsed_time(b) for a, b in evs)
+    t = torch.tensor([total_ms], device=prob.x.device, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    tokens = wl.B * wl.T * world * args.steps
+    value = tokens / (total_ms / 1e3)
+
+    # ------------------------------------------------------ end to end (host)
+    e2e = None
+    if not args.no_e2e:
+        h_in = {"x": prob.x, "h0": prob.h0, "c0": prob.c0}
+        if wl.train:
+            h_in["grad_out"] = prob.grad_out
+        h_in = {k: v for k, v in h_in.items() if v is not None}
+        outs = [prob.out, prob.h_n, prob.c_n]
+        if wl.train:
+            outs += [prob.dx, prob.dh0, prob.dc0] + prob.dw_ih + prob.dw_hh + \
+                (prob.db_ih + prob.db_hh if wl.bias else [])
+        host_in = {k: v.detach().cpu().pin_memory() for k, v in h_in.items()}
+        host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+        h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+        d2h = sum(o.numel() * o.element_size() for o in outs)
+
+        def e2e_step():
+            for k, v in host_in.items():
+                h_in[k].copy_(v, non_blocking=True)
+            step()
+            for ho, o in zip(host_out, outs):
+                ho.copy_(o, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        if world > 1:
+            dist.barrier()
+        for i in range(args.steps):
+            flush.zero_()
+            ev2[i][0].record(stream)
+            e2e_step()
+            ev2[i][1].record(stream)
+        torch.cuda.synchronize()
+        e_ms = sum(a.elapsed_time(b) for a, b in ev2)
+        te = torch.tensor([e_ms], device=prob.x.device, dtype=torch.float64)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": tokens / (float(te.item()) / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    # ------------------------------------------------------------- roofline
+    peaks = load_peaks()
+    roof = None
+    dom = max(((k, v) for k, v in kern.items() if v[0] > 0 and KIND_BOUND.get(k)),
+              key=lambda kv: kv[1][1], default=None)
+    if dom is not None:
+        kind, (launches, kms) = dom
+        unit, work_step = kernel_work(wl, kind)
+        per_launch = work_step * args.steps / launches
+        avg_s = kms / launches / 1e3
+        bound = KIND_BOUND[kind]
+        if bound == "alu":
+            peak = alu_peak_tflops()
+            peak_note = "derived: 148 SMs x 128 FP32 lanes x 2 flop x 1965 MHz"
+        else:
+            peak = peaks["bf16_tflops_sustained"]
+            peak_note = f"{peaks['source']} bf16 sustained"
+        achieved = per_launch / avg_s / 1e12
+        traffic = traffic_for(kind, wl.name)
+        roof = {"bound": bound, "kernel": kind, "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                "peak_source": peak_note, "launches": launches,
+                "avg_launch_ms": kms / launches, "share_of_step": kms / total_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, cores, sample, secs = cpu_oracle_rate(wl)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": sample, "seconds": round(secs, 2)}
+
+    if rank == 0:
+        line = {
+            "metric": "sequence tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": wl.dtype, "data": "synthetic (seeded; identical batch on every rank)",
+            "config": workload_config(wl, world), "e2e": e2e,
+            "gpu_launches": int(sum(v[0] for v in kern.values())),
+            "kernels_ms": {k: round(v[1] / args.steps, 4) for k, v in kern.items() if v[0]},
+            "roofline": roof, "cpu_baseline": cpu, "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,178 @@
+/*
+ * lstm.h -- C ABI of the B200 (sm_100a) LSTM library liblstm_b200.so.
+ *
+ * Computes the multi-layer, optionally bidirectional 4-gate LSTM forward and
+ * its back-propagation-through-time backward on one GPU, asynchronously on a
+ * caller-supplied CUDA stream.  Sources of the definitions (web pages, cited
+ * by title and section):
+ *
+ *   [warp_nn]   "Long Short-Term Memory (LSTM)", warp_nn API page: equation
+ *               block (gates i, f, g, o; c' = f*c + i*g; h' = o*tanh(c')),
+ *               the "Learnable parameters" table (shapes, i|f|g|o row
+ *               stacking, _reverse parameters), __call__ parameters/returns
+ *               (x (B,T,I); h0/c0/h_n/c_n (D*L,B,H); out (B,T,D*H); zero
+ *               default state; ValueError conditions).
+ *   [trace]     "Complete Trace: nn.LSTM": Step 1 (batch_first handling,
+ *               zero hx default), Step 3 (lstm.input schema: input, hx,
+ *               params, has_biases, num_layers, dropout, train,
+ *               bidirectional, batch_first -> output, h_n, c_n), Step 5
+ *               (workspace / reserveSpace sizing, the backward split into a
+ *               data phase and a weight phase).
+ *   [mxnet]     "LSTM Forward Computation": Stack Multiple RNN Cells (layer
+ *               k+1 reads layer k's output sequence only), Loop Unroll (the
+ *               backward is reverse-mode differentiation of the unrolled
+ *               loop).
+ *   [pulsatrix] pulsatrix LSTMModule: backward() sums every weight and bias
+ *               gradient over all timesteps.
+ *
+ * Notation: L = num_layers, D = 1 + bidirectional, B = batch, T = seq_len,
+ * I = input_size, H = hidden_size, G = 4H, in_l = I for l = 0 else D*H.
+ *
+ * Memory and ownership.  Every data pointer is DEVICE memory owned by the
+ * caller; the library never allocates device memory and keeps no state between
+ * calls.  The pointer ARRAYS (w_ih, w_hh, b_ih, b_hh, dw_ih, ...) are HOST
+ * arrays of length L*D, indexed l*D + d (d = 0 forward, d = 1 reverse, the
+ * [warp_nn] _reverse parameters), each entry a device pointer.  Scratch comes
+ * from a caller-allocated workspace (size from lstm_workspace_size); training
+ * additionally needs a reserve (size from lstm_reserve_size) that the forward
+ * fills and the matching backward reads.  Calls that may overlap on the GPU
+ * need distinct workspaces.
+ *
+ * Layouts (row-major, contiguous):
+ *   x     (B, T, I) if batch_first else (T, B, I)
+ *   out   (B, T, D*H) / (T, B, D*H); forward direction in [0,H), reverse in
+ *         [H,2H) at the same time position ([warp_nn])
+ *   h0, c0, h_n, c_n, dh0, dc0, grad_hn, grad_cn: (L*D, B, H), index l*D+d
+ *   w_ih[l*D+d] (G, in_l); w_hh[l*D+d] (G, H); b_ih, b_hh: G values.  The G
+ *   rows are the four gate blocks in the order i, f, g, o.
+ *
+ * Types: lstm_desc.dtype selects the storage type of x, h0, weights, biases,
+ * out, h_n, grad_out, grad_hn, dx and dh0 (float32 or bf16).  Cell states
+ * (c0, c_n, grad_cn, dc0) are always float32, and so are the weight and bias
+ * gradients.  Arithmetic accumulates in float32.
+ *
+ * Errors: functions return an lstm_status.  Argument errors are detected on
+ * the host before anything is enqueued.  Kernel-side failures (a bounded wait
+ * that gave up) are written to a status word inside the workspace and read by
+ * lstm_query_status.
+ */
+#ifndef LSTM_B200_H
+#define LSTM_B200_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* cudaStream_t;
+
+typedef enum {
+    LSTM_OK = 0,
+    LSTM_ERR_INVALID_ARG = 1,  /* bad size, NULL required pointer, num_layers < 1
+                                  ([warp_nn] ValueError cases) */
+    LSTM_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement */
+    LSTM_ERR_WORKSPACE = 3,    /* workspace or reserve smaller than the query */
+    LSTM_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed */
+    LSTM_ERR_TIMEOUT = 5       /* a kernel's bounded inter-block wait gave up */
+} lstm_status;
+
+typedef enum { LSTM_F32 = 0, LSTM_BF16 = 1 } lstm_dtype;
+
+typedef struct {
+    int input_size;     /* I >= 1 */
+    int hidden_size;    /* H >= 1 */
+    int num_layers;     /* L >= 1 ([warp_nn]: ValueError if < 1) */
+    int bidirectional;  /* 0 or 1 */
+    int bias;           /* 0: b_ih/b_hh ignored and treated as zero, db not written */
+    int batch_first;    /* 1: x/out/grad_out/dx are (B,T,.); 0: (T,B,.) */
+    int batch;          /* B >= 0 */
+    int seq_len;        /* T >= 0; T == 0 gives h_n = h0, c_n = c0 */
+    lstm_dtype dtype;
+} lstm_desc;
+
+/* Workspace bytes needed by lstm_forward and lstm_backward for this
+ * description (one size serves both).  0 if the description is invalid. */
+size_t lstm_workspace_size(const lstm_desc* desc);
+
+/* Reserve bytes a training forward fills for the backward: per (layer,
+ * direction) the gate activations i, f, g, o and the cell state c of every
+ * step, and per layer its output sequence ([trace] Step 5, reserveSpace).
+ * 0 if the description is invalid. */
+size_t lstm_reserve_size(const lstm_desc* desc);
+
+/*
+ * Forward ([warp_nn] equation block, [mxnet] Stack Multiple RNN Cells).
+ *   x, w_ih, w_hh (and b_ih, b_hh when desc->bias): inputs, required.
+ *   h0, c0: initial states or NULL for zeros ([trace] Step 1; [warp_nn]).
+ *   out, h_n, c_n: outputs, required when B*T (resp. B) > 0.
+ *   workspace/ws_bytes: scratch, at least lstm_workspace_size bytes,
+ *     256-byte aligned.
+ *   reserve/rs_bytes: NULL for inference; otherwise at least
+ *     lstm_reserve_size bytes, filled for lstm_backward.
+ * Enqueued on `stream`; returns before the GPU finishes.
+ */
+lstm_status lstm_forward(const lstm_desc* desc, const void* x, const void* h0, const float* c0,
+                         const void* const* w_ih, const void* const* w_hh,
+                         const void* const* b_ih, const void* const* b_hh,
+                         void* out, void* h_n, float* c_n,
+                         void* workspace, size_t ws_bytes,
+                         void* reserve, size_t rs_bytes, cudaStream_t stream);
+
+/*
+ * Backward (BPTT, [mxnet] Loop Unroll; [pulsatrix] backward(); data then
+ * weight phase as in [trace] Step 5, cuDNN Backward).  Must follow an
+ * lstm_forward with a reserve, on the same x, h0, c0 and weights.
+ *   grad_out: gradient of the loss w.r.t. out (same layout), required.
+ *   grad_hn, grad_cn: gradients w.r.t. h_n, c_n or NULL for zeros.
+ *   dx (layout of x), dh0, dc0 (L*D, B, H): input-gradient outputs.
+ *   dw_ih, dw_hh, db_ih, db_hh: host arrays of L*D device pointers to float32
+ *     gradients, OVERWRITTEN (not accumulated); db arrays ignored if !bias.
+ *     db_ih and db_hh receive the same values (the biases enter as a sum).
+ * Only desc->dtype == LSTM_F32 is implemented; bf16 returns
+ * LSTM_ERR_UNSUPPORTED.
+ */
+lstm_status lstm_backward(const lstm_desc* desc, const void* x, const void* h0, const float* c0,
+                          const void* const* w_ih, const void* const* w_hh,
+                          const void* grad_out, const void* grad_hn, const float* grad_cn,
+                          const void* reserve, size_t rs_bytes,
+                          void* workspace, size_t ws_bytes,
+                          void* dx, void* dh0, float* dc0,
+                          float* const* dw_ih, float* const* dw_hh,
+                          float* const* db_ih, float* const* db_hh, cudaStream_t stream);
+
+/* Synchronises `stream` and returns the kernel-side status recorded in
+ * `workspace` by the last call that used it (LSTM_OK or LSTM_ERR_TIMEOUT), or
+ * LSTM_ERR_CUDA if the stream reports an error. */
+lstm_status lstm_query_status(void* workspace, cudaStream_t stream);
+
+/* Static string naming a status code. */
+const char* lstm_status_string(lstm_status status);
+
+/*
+ * Kernel timing (instrumentation; the pages define no counterpart).  While
+ * enabled, the library brackets every kernel it launches with a pair of CUDA
+ * events on the launching stream.  lstm_timing_read waits for the recorded
+ * events, adds their durations to per-kind totals and copies up to
+ * max_entries {name, launches, total_ms} records into `out` (a host array);
+ * it returns the number of records written (the number of kinds when out is
+ * NULL), or -1 if an event could not be read.  Kinds: pack, proj_gemm,
+ * fwd_rec, bwd_rec, dw_gemm, dx_gemm, db_reduce, seq_copy.  lstm_timing_reset
+ * zeroes the totals.  Process-wide and thread-safe; event recording adds a
+ * few microseconds per launch, so leave it off outside measurements.
+ */
+typedef struct {
+    const char* name;       /* static string */
+    long long launches;
+    double total_ms;
+} lstm_kernel_time;
+
+lstm_status lstm_timing_enable(int enable);
+int lstm_timing_read(lstm_kernel_time* out, int max_entries);
+void lstm_timing_reset(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LSTM_B200_H */

@@ -1,0 +1,565 @@
+// C-ABI entry points and host-side scheduler of the LSTM library.
+//
+// The forward follows the lstm.input contract of "Complete Trace: nn.LSTM"
+// (Step 3): input, hx, params, has_biases, num_layers, bidirectional,
+// batch_first -> output, h_n, c_n, with the shapes of the warp_nn
+// "Long Short-Term Memory (LSTM)" page.  Per layer: a time-batched input
+// projection Gx = X W_ih^T + b_ih + b_hh for both directions at once, then one
+// persistent recurrent launch in which the directions run concurrently.  The
+// backward runs the layers top-down: the persistent BPTT launch (data phase),
+// then time-batched GEMMs for dW_ih, dW_hh and the layer-input gradient
+// (weight phase), mirroring the data/weight split described under cuDNN
+// Backward on the same page.
+#include <stdlib.h>
+#include <string.h>
+
+#include <mutex>
+#include <vector>
+
+#include "../../include/lstm.h"
+#include "lstm_internal.h"
+
+namespace lstm {
+namespace {
+
+struct DevInfo {
+    int sms = 0;
+    size_t smem_optin = 0;
+    bool ok = false;
+};
+
+DevInfo device_info() {
+    static std::mutex mu;
+    static std::vector<DevInfo> cache;
+    int dev = 0;
+    DevInfo bad;
+    if (cudaGetDevice(&dev) != cudaSuccess) return bad;
+    std::lock_guard<std::mutex> lk(mu);
+    if ((int)cache.size() <= dev) cache.resize(dev + 1);
+    if (!cache[dev].ok) {
+        cudaDeviceProp prop;
+        if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return bad;
+        cache[dev].sms = prop.multiProcessorCount;
+        cache[dev].smem_optin = prop.sharedMemPerBlockOptin;
+        cache[dev].ok = true;
+    }
+    return cache[dev];
+}
+
+uint64_t timeout_ns() {
+    static uint64_t v = [] {
+        const char* e = getenv("LSTM_B200_WAIT_TIMEOUT_NS");
+        if (e && *e) return (uint64_t)strtoull(e, nullptr, 10);
+        return (uint64_t)2000000000ull;   // 2 s: far above any healthy step
+    }();
+    return v;
+}
+
+// ------------------------------------------------------------ kernel timing
+// When enabled, every kernel the library launches is bracketed by a pair of
+// CUDA events on its stream; lstm_timing_read() resolves them into per-kind
+// launch counts and summed device durations.
+enum Kind { K_PACK = 0, K_PROJ, K_FWD_REC, K_BWD_REC, K_DW, K_DX, K_DB, K_COPY, K_COUNT };
+const char* const kKindNames[K_COUNT] = {"pack", "proj_gemm", "fwd_rec", "bwd_rec",
+                                         "dw_gemm", "dx_gemm", "db_reduce", "seq_copy"};
+
+struct Timing {
+    std::mutex mu;
+    bool on = false;
+    struct Pending { int kind; cudaEvent_t a, b; };
+    std::vector<Pending> pending;
+    std::vector<cudaEvent_t> pool;
+    double total_ms[K_COUNT] = {};
+    long long launches[K_COUNT] = {};
+};
+
+Timing& timing() {
+    static Timing t;
+    return t;
+}
+
+cudaEvent_t take_event(Timing& tm) {
+    cudaEvent_t e = nullptr;
+    if (!tm.pool.empty()) {
+        e = tm.pool.back();
+        tm.pool.pop_back();
+    } else if (cudaEventCreate(&e) != cudaSuccess) {
+        e = nullptr;
+    }
+    return e;
+}
+
+template <typename F>
+cudaError_t timed(int kind, cudaStream_t s, F&& f) {
+    Timing& tm = timing();
+    if (!tm.on) return f();
+    std::lock_guard<std::mutex> lk(tm.mu);
+    cudaEvent_t a = take_event(tm), b = take_event(tm);
+    if (!a || !b) return cudaErrorMemoryAllocation;
+    cudaError_t e = cudaEventRecord(a, s);
+    if (e != cudaSuccess) return e;
+    e = f();
+    if (e != cudaSuccess) return e;
+    e = cudaEventRecord(b, s);
+    if (e != cudaSuccess) return e;
+    tm.pending.push_back({kind, a, b});
+    return cudaSuccess;
+}
+
+constexpr size_t kAlign = 256;
+inline size_t al(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+
+// Shapes and the planned kernel partitions for one description.  The plans
+// depend on the device (SM count, shared memory), so the layout is computed
+// for the current device.
+struct Layout {
+    int L, D, I, H, B, T, G;
+    DType dt;
+    size_t es;
+    RecPlan fwd, bwd;
+    bool bwd_ok;
+    // workspace offsets
+    size_t status, ctr_f, ctr_b, wih[32], bias[32], whh_f, whh_b, gx, seq[2], dG, dseq[2], xt,
+        dbpart, total;
+    // reserve offsets
+    size_t act[32], cst[32], hseq[32], rtotal;   // per layer: [D][T][B][G], [D][T][B][H], [T][B][D*H]
+};
+
+int in_size(const Layout& l, int layer) { return layer == 0 ? l.I : l.D * l.H; }
+
+bool valid_desc(const lstm_desc* d) {
+    if (!d) return false;
+    if (d->input_size < 1 || d->hidden_size < 1 || d->num_layers < 1) return false;
+    if (d->num_layers > 32) return false;
+    if (d->bidirectional != 0 && d->bidirectional != 1) return false;
+    if (d->batch < 0 || d->seq_len < 0) return false;
+    if (d->dtype != LSTM_F32 && d->dtype != LSTM_BF16) return false;
+    // sizes addressed with 32-bit loop counters inside kernels
+    const long long H = d->hidden_size, I = d->input_size;
+    if (H > (1 << 16) || I > (1 << 20)) return false;
+    return true;
+}
+
+bool make_layout(const lstm_desc* d, Layout& l) {
+    if (!valid_desc(d)) return false;
+    DevInfo dev = device_info();
+    if (!dev.ok) {
+        // No device: plan against a nominal B200 so sizes can still be queried.
+        dev.sms = 148;
+        dev.smem_optin = 232448;
+    }
+    l.L = d->num_layers;
+    l.D = d->bidirectional ? 2 : 1;
+    l.I = d->input_size;
+    l.H = d->hidden_size;
+    l.B = d->batch;
+    l.T = d->seq_len;
+    l.G = 4 * l.H;
+    l.dt = d->dtype == LSTM_F32 ? DType::F32 : DType::BF16;
+    l.es = dtype_size(l.dt);
+    const size_t smem_max = dev.smem_optin - 1024;
+    const int Bp = l.B > 0 ? l.B : 1;
+    l.fwd = plan_fwd_rec(l.H, Bp, l.D, l.dt, dev.sms, smem_max);
+    if (l.fwd.ctas == 0) return false;
+    l.bwd = plan_bwd_rec(l.H, Bp, l.D, dev.sms, smem_max);
+    l.bwd_ok = l.bwd.ctas > 0;
+    const size_t TB = (size_t)l.T * l.B;
+    size_t o = 0;
+    l.status = o; o += al(sizeof(int));
+    l.ctr_f = o; o += al(sizeof(unsigned) * (size_t)l.L * l.D * l.fwd.nbg);
+    l.ctr_b = o; o += al(sizeof(unsigned) * (size_t)l.L * l.D * (l.bwd_ok ? l.bwd.nbg : 1));
+    for (int k = 0; k < l.L; ++k) {
+        l.wih[k] = o; o += al((size_t)l.D * l.G * in_size(l, k) * l.es);
+        l.bias[k] = o; o += al((size_t)l.D * l.G * 4);
+    }
+    l.whh_f = o; o += al((size_t)l.D * l.fwd.nu * ((l.H + 3) & ~3) * 4 * l.fwd.U * l.es);
+    l.whh_b = o; o += al(l.bwd_ok ? (size_t)l.D * l.bwd.nu * l.G * l.bwd.U * 4 : 0);
+    l.gx = o; o += al(TB * l.D * l.G * 4);
+    l.seq[0] = o; o += al(TB * l.D * l.H * l.es);
+    l.seq[1] = o; o += al(TB * l.D * l.H * l.es);
+    const size_t maxin = (size_t)(l.I > l.D * l.H ? l.I : l.D * l.H);
+    if (l.dt == DType::F32) {
+        l.dG = o; o += al(TB * l.D * l.G * 4);
+        l.dseq[0] = o; o += al(TB * maxin * 4);
+        l.dseq[1] = o; o += al(TB * maxin * 4);
+        l.xt = o; o += al(TB * l.I * 4);
+        l.dbpart = o; o += al((size_t)l.D * (l.bwd_ok ? l.bwd.nbg : 1) * l.G * 4);
+    } else {
+        l.dG = l.dseq[0] = l.dseq[1] = l.xt = l.dbpart = 0;
+    }
+    l.total = o;
+    size_t r = 0;
+    for (int k = 0; k < l.L; ++k) {
+        l.act[k] = r; r += al((size_t)l.D * TB * l.G * 4);
+        l.cst[k] = r; r += al((size_t)l.D * TB * l.H * 4);
+        l.hseq[k] = r; r += al(TB * l.D * l.H * l.es);
+    }
+    l.rtotal = r;
+    return true;
+}
+
+inline char* P(void* base, size_t off) { return static_cast<char*>(base) + off; }
+
+#define LSTM_CUDA(call)                                  \
+    do {                                                 \
+        if ((call) != cudaSuccess) return LSTM_ERR_CUDA; \
+    } while (0)
+
+}  // namespace
+}  // namespace lstm
+
+using namespace lstm;
+
+extern "C" {
+
+size_t lstm_workspace_size(const lstm_desc* desc) {
+    Layout l;
+    if (!make_layout(desc, l)) return 0;
+    return l.total;
+}
+
+size_t lstm_reserve_size(const lstm_desc* desc) {
+    Layout l;
+    if (!make_layout(desc, l)) return 0;
+    return l.rtotal;
+}
+
+lstm_status lstm_timing_enable(int enable) {
+    Timing& tm = timing();
+    std::lock_guard<std::mutex> lk(tm.mu);
+    tm.on = enable != 0;
+    return LSTM_OK;
+}
+
+int lstm_timing_read(lstm_kernel_time* out, int max_entries) {
+    Timing& tm = timing();
+    std::lock_guard<std::mutex> lk(tm.mu);
+    for (const auto& p : tm.pending) {
+        float ms = 0.f;
+        if (cudaEventSynchronize(p.b) == cudaSuccess && cudaEventElapsedTime(&ms, p.a, p.b) == cudaSuccess) {
+            tm.total_ms[p.kind] += ms;
+            tm.launches[p.kind] += 1;
+        } else {
+            return -1;
+        }
+        tm.pool.push_back(p.a);
+        tm.pool.push_back(p.b);
+    }
+    tm.pending.clear();
+    int n = 0;
+    for (int k = 0; k < K_COUNT && n < max_entries; ++k, ++n) {
+        if (!out) break;
+        out[n].name = kKindNames[k];
+        out[n].launches = tm.launches[k];
+        out[n].total_ms = tm.total_ms[k];
+    }
+    return out ? n : (int)K_COUNT;
+}
+
+void lstm_timing_reset(void) {
+    Timing& tm = timing();
+    std::lock_guard<std::mutex> lk(tm.mu);
+    for (const auto& p : tm.pending) {
+        cudaEventSynchronize(p.b);
+        tm.pool.push_back(p.a);
+        tm.pool.push_back(p.b);
+    }
+    tm.pending.clear();
+    for (int k = 0; k < K_COUNT; ++k) {
+        tm.total_ms[k] = 0.0;
+        tm.launches[k] = 0;
+    }
+}
+
+const char* lstm_status_string(lstm_status s) {
+    switch (s) {
+        case LSTM_OK: return "LSTM_OK";
+        case LSTM_ERR_INVALID_ARG: return "LSTM_ERR_INVALID_ARG";
+        case LSTM_ERR_UNSUPPORTED: return "LSTM_ERR_UNSUPPORTED";
+        case LSTM_ERR_WORKSPACE: return "LSTM_ERR_WORKSPACE";
+        case LSTM_ERR_CUDA: return "LSTM_ERR_CUDA";
+        case LSTM_ERR_TIMEOUT: return "LSTM_ERR_TIMEOUT";
+    }
+    return "LSTM_ERR_UNKNOWN";
+}
+
+lstm_status lstm_query_status(void* workspace, cudaStream_t stream) {
+    if (!workspace) return LSTM_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return LSTM_ERR_CUDA;
+    int st = 0;
+    if (cudaMemcpy(&st, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return LSTM_ERR_CUDA;
+    return st == 0 ? LSTM_OK : (lstm_status)st;
+}
+
+lstm_status lstm_forward(const lstm_desc* desc, const void* x, const void* h0, const float* c0,
+                         const void* const* w_ih, const void* const* w_hh,
+                         const void* const* b_ih, const void* const* b_hh,
+                         void* out, void* h_n, float* c_n,
+                         void* workspace, size_t ws_bytes,
+                         void* reserve, size_t rs_bytes, cudaStream_t stream) {
+    if (!valid_desc(desc)) return LSTM_ERR_INVALID_ARG;
+    if (!w_ih || !w_hh) return LSTM_ERR_INVALID_ARG;
+    const int LD = desc->num_layers * (desc->bidirectional ? 2 : 1);
+    for (int i = 0; i < LD; ++i) {
+        if (!w_ih[i] || !w_hh[i]) return LSTM_ERR_INVALID_ARG;
+        if (desc->bias && (!b_ih || !b_hh || !b_ih[i] || !b_hh[i])) return LSTM_ERR_INVALID_ARG;
+    }
+    const long long BT = (long long)desc->batch * desc->seq_len;
+    if (BT > 0 && (!x || !out)) return LSTM_ERR_INVALID_ARG;
+    if (desc->batch > 0 && (!h_n || !c_n)) return LSTM_ERR_INVALID_ARG;
+    if (!workspace) return LSTM_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return LSTM_ERR_INVALID_ARG;
+    if (reserve && reinterpret_cast<uintptr_t>(reserve) % 256 != 0) return LSTM_ERR_INVALID_ARG;
+    Layout l;
+    if (!make_layout(desc, l)) return LSTM_ERR_UNSUPPORTED;
+    if (ws_bytes < l.total) return LSTM_ERR_WORKSPACE;
+    if (reserve && rs_bytes < l.rtotal) return LSTM_ERR_WORKSPACE;
+    if (!device_info().ok) return LSTM_ERR_CUDA;
+
+    const int L = l.L, D = l.D, H = l.H, B = l.B, T = l.T, G = l.G;
+    const size_t es = l.es;
+    const size_t state_elems = (size_t)D * B * H;   // elements per layer slice
+    LSTM_CUDA(cudaMemsetAsync(workspace, 0, l.ctr_b + al(sizeof(unsigned) * (size_t)L * D *
+                                                          (l.bwd_ok ? l.bwd.nbg : 1)),
+                              stream));
+    if (B == 0) return LSTM_OK;
+    if (T == 0) {
+        // no step runs: h_n = h0, c_n = c0 (zeros when absent)
+        const size_t n = (size_t)L * state_elems;
+        if (h0) LSTM_CUDA(cudaMemcpyAsync(h_n, h0, n * es, cudaMemcpyDeviceToDevice, stream));
+        else LSTM_CUDA(cudaMemsetAsync(h_n, 0, n * es, stream));
+        if (c0) LSTM_CUDA(cudaMemcpyAsync(c_n, c0, n * 4, cudaMemcpyDeviceToDevice, stream));
+        else LSTM_CUDA(cudaMemsetAsync(c_n, 0, n * 4, stream));
+        return LSTM_OK;
+    }
+    int* status = reinterpret_cast<int*>(P(workspace, l.status));
+    for (int k = 0; k < L; ++k) {
+        const int in = in_size(l, k);
+        PackIhArgs pk{};
+        pk.H = H; pk.in = in; pk.D = D; pk.dt = l.dt;
+        for (int d = 0; d < D; ++d) {
+            pk.w[d] = w_ih[k * D + d];
+            pk.b_ih[d] = desc->bias ? b_ih[k * D + d] : nullptr;
+            pk.b_hh[d] = desc->bias ? b_hh[k * D + d] : nullptr;
+        }
+        pk.wp = P(workspace, l.wih[k]);
+        pk.bias_p = reinterpret_cast<float*>(P(workspace, l.bias[k]));
+        LSTM_CUDA(timed(K_PACK, stream, [&] { return launch_pack_ih(pk, stream); }));
+    }
+    const void* layer_in = x;
+    for (int k = 0; k < L; ++k) {
+        const int in = in_size(l, k);
+        // time-batched input projection for both directions
+        GemmArgs g{};
+        g.M = B * T; g.N = D * G; g.K = in;
+        g.A = layer_in; g.ta = l.dt; g.sAm = in; g.sAk = 1;
+        g.B = P(workspace, l.wih[k]); g.tb = l.dt; g.sBk = 1; g.sBn = in;
+        g.C = P(workspace, l.gx); g.tc = DType::F32; g.ldc = (long long)D * G;
+        g.bias = reinterpret_cast<const float*>(P(workspace, l.bias[k]));
+        g.accumulate = 0;
+        if (k == 0 && desc->batch_first) { g.remap_T = T; g.remap_B = B; }
+        LSTM_CUDA(timed(K_PROJ, stream, [&] { return launch_gemm(g, stream); }));
+
+        PackHhFwdArgs ph{};
+        ph.H = H; ph.D = D; ph.nu = l.fwd.nu; ph.U = l.fwd.U; ph.dt = l.dt;
+        for (int d = 0; d < D; ++d) ph.w[d] = w_hh[k * D + d];
+        ph.out = P(workspace, l.whh_f);
+        LSTM_CUDA(timed(K_PACK, stream, [&] { return launch_pack_hh_fwd(ph, stream); }));
+
+        FwdRecArgs f{};
+        f.H = H; f.B = B; f.T = T; f.D = D; f.p = l.fwd; f.dt = l.dt;
+        f.gx = reinterpret_cast<const float*>(P(workspace, l.gx));
+        f.wpk = P(workspace, l.whh_f);
+        f.h0 = h0 ? static_cast<const char*>(h0) + (size_t)k * state_elems * es : nullptr;
+        f.c0 = c0 ? c0 + (size_t)k * state_elems : nullptr;
+        void* hseq = reserve ? P(reserve, l.hseq[k]) : P(workspace, l.seq[k & 1]);
+        f.hseq = hseq;
+        if (k == L - 1) {
+            f.out = out;
+            f.out_st = desc->batch_first ? (long long)D * H : (long long)B * D * H;
+            f.out_sb = desc->batch_first ? (long long)T * D * H : (long long)D * H;
+        }
+        f.h_n = static_cast<char*>(h_n) + (size_t)k * state_elems * es;
+        f.c_n = c_n + (size_t)k * state_elems;
+        if (reserve) {
+            f.act = reinterpret_cast<float*>(P(reserve, l.act[k]));
+            f.cst = reinterpret_cast<float*>(P(reserve, l.cst[k]));
+        }
+        f.ctr = reinterpret_cast<unsigned*>(P(workspace, l.ctr_f)) + (size_t)k * D * l.fwd.nbg;
+        f.status = status;
+        f.timeout_ns = timeout_ns();
+        LSTM_CUDA(timed(K_FWD_REC, stream, [&] { return launch_fwd_rec(f, stream); }));
+        layer_in = hseq;
+    }
+    return LSTM_OK;
+}
+
+lstm_status lstm_backward(const lstm_desc* desc, const void* x, const void* h0, const float* c0,
+                          const void* const* w_ih, const void* const* w_hh,
+                          const void* grad_out, const void* grad_hn, const float* grad_cn,
+                          const void* reserve, size_t rs_bytes,
+                          void* workspace, size_t ws_bytes,
+                          void* dx, void* dh0, float* dc0,
+                          float* const* dw_ih, float* const* dw_hh,
+                          float* const* db_ih, float* const* db_hh, cudaStream_t stream) {
+    if (!valid_desc(desc)) return LSTM_ERR_INVALID_ARG;
+    if (!w_ih || !w_hh || !dw_ih || !dw_hh) return LSTM_ERR_INVALID_ARG;
+    const int LD = desc->num_layers * (desc->bidirectional ? 2 : 1);
+    for (int i = 0; i < LD; ++i) {
+        if (!w_ih[i] || !w_hh[i] || !dw_ih[i] || !dw_hh[i]) return LSTM_ERR_INVALID_ARG;
+        if (desc->bias && (!db_ih || !db_hh || !db_ih[i] || !db_hh[i])) return LSTM_ERR_INVALID_ARG;
+    }
+    const long long BT = (long long)desc->batch * desc->seq_len;
+    if (BT > 0 && (!x || !grad_out || !dx || !reserve)) return LSTM_ERR_INVALID_ARG;
+    if (desc->batch > 0 && (!dh0 || !dc0)) return LSTM_ERR_INVALID_ARG;
+    if (!workspace) return LSTM_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return LSTM_ERR_INVALID_ARG;
+    if (reserve && reinterpret_cast<uintptr_t>(reserve) % 256 != 0) return LSTM_ERR_INVALID_ARG;
+    if (desc->dtype != LSTM_F32) return LSTM_ERR_UNSUPPORTED;
+    Layout l;
+    if (!make_layout(desc, l)) return LSTM_ERR_UNSUPPORTED;
+    if (!l.bwd_ok) return LSTM_ERR_UNSUPPORTED;
+    if (ws_bytes < l.total) return LSTM_ERR_WORKSPACE;
+    if (BT > 0 && rs_bytes < l.rtotal) return LSTM_ERR_WORKSPACE;
+    if (!device_info().ok) return LSTM_ERR_CUDA;
+
+    const int L = l.L, D = l.D, H = l.H, B = l.B, T = l.T, G = l.G;
+    const size_t state = (size_t)D * B * H;
+    LSTM_CUDA(cudaMemsetAsync(workspace, 0, l.ctr_b + al(sizeof(unsigned) * (size_t)L * D * l.bwd.nbg),
+                              stream));
+    // weight gradients start from zero (T == 0 or B == 0 leave them zero)
+    for (int k = 0; k < L; ++k) {
+        for (int d = 0; d < D; ++d) {
+            const int i = k * D + d;
+            if (BT == 0) {
+                LSTM_CUDA(cudaMemsetAsync(dw_ih[i], 0, (size_t)G * in_size(l, k) * 4, stream));
+                LSTM_CUDA(cudaMemsetAsync(dw_hh[i], 0, (size_t)G * H * 4, stream));
+                if (desc->bias) {
+                    LSTM_CUDA(cudaMemsetAsync(db_ih[i], 0, (size_t)G * 4, stream));
+                    LSTM_CUDA(cudaMemsetAsync(db_hh[i], 0, (size_t)G * 4, stream));
+                }
+            }
+        }
+    }
+    if (B == 0) return LSTM_OK;
+    if (T == 0) {
+        const size_t n = (size_t)L * state;
+        if (grad_hn) LSTM_CUDA(cudaMemcpyAsync(dh0, grad_hn, n * 4, cudaMemcpyDeviceToDevice, stream));
+        else LSTM_CUDA(cudaMemsetAsync(dh0, 0, n * 4, stream));
+        if (grad_cn) LSTM_CUDA(cudaMemcpyAsync(dc0, grad_cn, n * 4, cudaMemcpyDeviceToDevice, stream));
+        else LSTM_CUDA(cudaMemsetAsync(dc0, 0, n * 4, stream));
+        return LSTM_OK;
+    }
+    int* status = reinterpret_cast<int*>(P(workspace, l.status));
+    float* dG = reinterpret_cast<float*>(P(workspace, l.dG));
+    // time-major copy of x for the layer-0 weight gradient
+    const float* x_tm = static_cast<const float*>(x);
+    if (desc->batch_first) {
+        SeqCopyArgs sc{};
+        sc.T = T; sc.B = B; sc.W = l.I; sc.dt = DType::F32;
+        sc.src = x; sc.s_st = l.I; sc.s_sb = (long long)T * l.I;
+        sc.dst = P(workspace, l.xt); sc.d_st = (long long)B * l.I; sc.d_sb = l.I;
+        LSTM_CUDA(timed(K_COPY, stream, [&] { return launch_seq_copy(sc, stream); }));
+        x_tm = reinterpret_cast<const float*>(P(workspace, l.xt));
+    }
+    const float* dy = static_cast<const float*>(grad_out);
+    long long dy_st = desc->batch_first ? (long long)D * H : (long long)B * D * H;
+    long long dy_sb = desc->batch_first ? (long long)T * D * H : (long long)D * H;
+    int cur = 0;
+    for (int k = L - 1; k >= 0; --k) {
+        const int in = in_size(l, k);
+        PackHhBwdArgs pb{};
+        pb.H = H; pb.D = D; pb.nu = l.bwd.nu; pb.U = l.bwd.U;
+        for (int d = 0; d < D; ++d) pb.w[d] = static_cast<const float*>(w_hh[k * D + d]);
+        pb.out = reinterpret_cast<float*>(P(workspace, l.whh_b));
+        LSTM_CUDA(timed(K_PACK, stream, [&] { return launch_pack_hh_bwd(pb, stream); }));
+
+        BwdRecArgs b{};
+        b.H = H; b.B = B; b.T = T; b.D = D; b.p = l.bwd;
+        b.wt = reinterpret_cast<const float*>(P(workspace, l.whh_b));
+        b.act = reinterpret_cast<const float*>(static_cast<const char*>(reserve) + l.act[k]);
+        b.cst = reinterpret_cast<const float*>(static_cast<const char*>(reserve) + l.cst[k]);
+        b.c0 = c0 ? c0 + (size_t)k * state : nullptr;
+        b.dy = dy; b.dy_st = dy_st; b.dy_sb = dy_sb;
+        b.grad_hn = grad_hn ? static_cast<const float*>(grad_hn) + (size_t)k * state : nullptr;
+        b.grad_cn = grad_cn ? grad_cn + (size_t)k * state : nullptr;
+        b.dG = dG;
+        b.dh0 = static_cast<float*>(dh0) + (size_t)k * state;
+        b.dc0 = dc0 + (size_t)k * state;
+        b.dbpart = reinterpret_cast<float*>(P(workspace, l.dbpart));
+        b.ctr = reinterpret_cast<unsigned*>(P(workspace, l.ctr_b)) + (size_t)k * D * l.bwd.nbg;
+        b.status = status;
+        b.timeout_ns = timeout_ns();
+        LSTM_CUDA(timed(K_BWD_REC, stream, [&] { return launch_bwd_rec(b, stream); }));
+
+        if (desc->bias) {
+            DbArgs db{};
+            db.G = G; db.D = D; db.nbg = l.bwd.nbg; db.dbpart = b.dbpart;
+            for (int d = 0; d < D; ++d) { db.db_ih[d] = db_ih[k * D + d]; db.db_hh[d] = db_hh[k * D + d]; }
+            LSTM_CUDA(timed(K_DB, stream, [&] { return launch_db_reduce(db, stream); }));
+        }
+        const float* layer_in = k == 0 ? x_tm
+                                       : reinterpret_cast<const float*>(static_cast<const char*>(reserve) + l.hseq[k - 1]);
+        const float* hs = reinterpret_cast<const float*>(static_cast<const char*>(reserve) + l.hseq[k]);
+        const long long ldg = (long long)D * G, ldh = (long long)D * H;
+        for (int d = 0; d < D; ++d) {
+            // dW_ih = sum_t dG_t^T x_t
+            GemmArgs g{};
+            g.M = G; g.N = in; g.K = B * T;
+            g.A = dG + (size_t)d * G; g.ta = DType::F32; g.sAm = 1; g.sAk = ldg;
+            g.B = layer_in; g.tb = DType::F32; g.sBk = in; g.sBn = 1;
+            g.C = dw_ih[k * D + d]; g.tc = DType::F32; g.ldc = in;
+            LSTM_CUDA(timed(K_DW, stream, [&] { return launch_gemm(g, stream); }));
+            // dW_hh = sum_t dG_t^T h_{t-1} (h_{-1} = h0)
+            GemmArgs gh{};
+            gh.M = G; gh.N = H; gh.K = B * (T - 1);
+            gh.ta = DType::F32; gh.sAm = 1; gh.sAk = ldg;
+            gh.tb = DType::F32; gh.sBk = ldh; gh.sBn = 1;
+            gh.C = dw_hh[k * D + d]; gh.tc = DType::F32; gh.ldc = H;
+            if (d == 0) {
+                gh.A = dG + (size_t)B * ldg + (size_t)d * G;     // rows t >= 1
+                gh.B = hs + (size_t)d * H;                        // h at t-1
+            } else {
+                gh.A = dG + (size_t)d * G;                        // rows t <= T-2
+                gh.B = hs + (size_t)B * ldh + (size_t)d * H;      // h at t+1
+            }
+            if (T > 1) {
+                LSTM_CUDA(timed(K_DW, stream, [&] { return launch_gemm(gh, stream); }));
+            } else {
+                LSTM_CUDA(cudaMemsetAsync(dw_hh[k * D + d], 0, (size_t)G * H * 4, stream));
+            }
+            if (h0) {
+                GemmArgs g0 = gh;
+                g0.K = B;
+                g0.A = dG + (d == 0 ? 0 : (size_t)(T - 1) * B * ldg) + (size_t)d * G;
+                g0.B = static_cast<const float*>(h0) + ((size_t)k * D + d) * B * H;
+                g0.sBk = H;
+                g0.accumulate = 1;
+                LSTM_CUDA(timed(K_DW, stream, [&] { return launch_gemm(g0, stream); }));
+            }
+        }
+        // gradient w.r.t. the layer input: sum_d dG_d W_ih_d
+        float* din = k == 0 ? static_cast<float*>(dx) : reinterpret_cast<float*>(P(workspace, l.dseq[cur]));
+        for (int d = 0; d < D; ++d) {
+            GemmArgs g{};
+            g.M = B * T; g.N = in; g.K = G;
+            g.A = dG + (size_t)d * G; g.ta = DType::F32; g.sAm = ldg; g.sAk = 1;
+            g.B = w_ih[k * D + d]; g.tb = DType::F32; g.sBk = in; g.sBn = 1;
+            g.C = din; g.tc = DType::F32; g.ldc = in;
+            g.accumulate = d > 0;
+            if (k == 0 && desc->batch_first) { g.remap_T = -T; g.remap_B = B; }
+            LSTM_CUDA(timed(K_DX, stream, [&] { return launch_gemm(g, stream); }));
+        }
+        if (k > 0) {
+            dy = din;
+            dy_st = (long long)B * in;
+            dy_sb = in;
+            cur ^= 1;
+        }
+    }
+    (void)status;
+    return LSTM_OK;
+}
+
+}  // extern "C"

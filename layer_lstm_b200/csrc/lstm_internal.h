@@ -1,0 +1,130 @@
+// Internal interface between the C-ABI/scheduler (lstm_abi.cu) and the
+// kernel launchers.  Not installed; no torch types anywhere.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace lstm {
+
+enum class DType : int { F32 = 0, BF16 = 1 };
+
+inline size_t dtype_size(DType t) { return t == DType::F32 ? 4 : 2; }
+
+// ---------------------------------------------------------------- GEMM
+// C[M x N] (+)= A[M x K] * B[K x N] (+ bias[n]), float32 accumulate.
+// A(m,k) = A[m*sAm + k*sAk], B(k,n) = B[k*sBk + n*sBn]; one of each pair of
+// strides must be 1.  The output row of m is m, or with remap_T > 0 the
+// (b,t) -> (t,b) row map m = b*T + t -> t*B + b (remap_B = B), or with
+// remap_T < 0 the inverse map m = t*B + b -> b*T + t (T = -remap_T).
+struct GemmArgs {
+    int M, N, K;
+    const void* A; long long sAm, sAk; DType ta;
+    const void* B; long long sBk, sBn; DType tb;
+    void* C; long long ldc; DType tc;   // tc: F32 or BF16 output
+    const float* bias;                  // [N] or null
+    int accumulate;                     // 1: C += result (C must be F32)
+    int remap_T, remap_B;
+};
+cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s);
+
+// ---------------------------------------------------------------- packing
+// Gate-interleaved row order used inside the library: packed row p = 4u + q
+// holds standard row q*H + u (q = 0..3 for i, f, g, o).
+struct PackIhArgs {
+    int H, in, D;
+    const void* w[2];          // per direction (G, in), standard order
+    const void* b_ih[2];       // per direction G or null
+    const void* b_hh[2];
+    DType dt;
+    void* wp;                  // [D*G][in] packed, dtype dt
+    float* bias_p;             // [D*G] packed b_ih + b_hh (zeros without bias)
+};
+cudaError_t launch_pack_ih(const PackIhArgs& a, cudaStream_t s);
+
+// Forward recurrent weights: [D][nu][H][4U] (k-major slices), zero padded.
+struct PackHhFwdArgs {
+    int H, D, nu, U;
+    const void* w[2];
+    DType dt;
+    void* out;
+};
+cudaError_t launch_pack_hh_fwd(const PackHhFwdArgs& a, cudaStream_t s);
+
+// Backward recurrent weights (float32): [D][nu][G][U]: element (r, jl) is
+// W_hh[r][j*U + jl], standard row order r, zero padded.
+struct PackHhBwdArgs {
+    int H, D, nu, U;
+    const float* w[2];
+    float* out;
+};
+cudaError_t launch_pack_hh_bwd(const PackHhBwdArgs& a, cudaStream_t s);
+
+// ---------------------------------------------------------------- recurrence
+struct RecPlan {
+    int nbg, Bg, nu, U, Bs, KS, threads;
+    size_t smem;
+    int ctas;
+};
+
+struct FwdRecArgs {
+    int H, B, T, D;
+    RecPlan p;
+    DType dt;
+    const float* gx;            // [T][B][D*G] packed per direction, biases included
+    const void* wpk;            // PackHhFwd layout
+    const void* h0;             // [D][B][H] or null
+    const float* c0;            // [D][B][H] or null
+    void* hseq;                 // [T][B][D*H] layer output, time-major
+    void* out; long long out_st, out_sb;   // user out (top layer) or null; element strides
+    void* h_n; float* c_n;      // [D][B][H]
+    float* act; float* cst;     // [D][T][B][G] packed / [D][T][B][H], or null
+    unsigned* ctr;              // [D*nbg] arrival counters, zero on entry
+    int* status;
+    uint64_t timeout_ns;
+};
+cudaError_t launch_fwd_rec(const FwdRecArgs& a, cudaStream_t s);
+RecPlan plan_fwd_rec(int H, int B, int D, DType dt, int num_sms, size_t smem_max);
+
+struct BwdRecArgs {
+    int H, B, T, D;
+    RecPlan p;
+    const float* wt;            // PackHhBwd layout
+    const float* act;           // [D][T][B][G] packed
+    const float* cst;           // [D][T][B][H]
+    const float* c0;            // [D][B][H] or null
+    const float* dy; long long dy_st, dy_sb;   // dy(t,b,col) = dy[t*st + b*sb + col]
+    const float* grad_hn;       // [D][B][H] or null
+    const float* grad_cn;       // [D][B][H] or null
+    float* dG;                  // [T][B][D*G], standard row order per direction
+    float* dh0; float* dc0;     // [D][B][H]
+    float* dbpart;              // [D][nbg][G]
+    unsigned* ctr;
+    int* status;
+    uint64_t timeout_ns;
+};
+cudaError_t launch_bwd_rec(const BwdRecArgs& a, cudaStream_t s);
+RecPlan plan_bwd_rec(int H, int B, int D, int num_sms, size_t smem_max);
+
+// db[d][r] = sum over groups of dbpart[d][g][r] (fixed order), written to
+// both db_ih[d] and db_hh[d].
+struct DbArgs {
+    int G, D, nbg;
+    const float* dbpart;
+    float* db_ih[2];
+    float* db_hh[2];
+};
+cudaError_t launch_db_reduce(const DbArgs& a, cudaStream_t s);
+
+// dst(t,b,:) = src(t,b,:) for a (rows x width) sequence with arbitrary
+// (t,b) element strides; used to make time-major copies.
+struct SeqCopyArgs {
+    int T, B, W;
+    const void* src; long long s_st, s_sb;
+    void* dst; long long d_st, d_sb;
+    DType dt;
+};
+cudaError_t launch_seq_copy(const SeqCopyArgs& a, cudaStream_t s);
+
+}  // namespace lstm
