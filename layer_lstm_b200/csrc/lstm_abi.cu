@@ -119,8 +119,8 @@ struct Layout {
     RecPlan fwd, bwd;
     bool bwd_ok;
     // workspace offsets
-    size_t status, ctr_f, ctr_b, wih[32], bias[32], whh_f, whh_b, gx, seq[2], dG, dseq[2], xt,
-        dbpart, total;
+    size_t status, ctr_f, ctr_b, wih[32], bias[32], whh_f, whh_b, gx, hT, seq[2], dG, dseq[2], xt,
+        dbpart, P, total;
     // reserve offsets
     size_t act[32], cst[32], hseq[32], rtotal;   // per layer: [D][T][B][G], [D][T][B][H], [T][B][D*H]
 };
@@ -173,8 +173,10 @@ bool make_layout(const lstm_desc* d, Layout& l) {
         l.bias[k] = o; o += al((size_t)l.D * l.G * 4);
     }
     l.whh_f = o; o += al((size_t)l.D * l.fwd.nu * ((l.H + 3) & ~3) * 4 * l.fwd.U * l.es);
-    l.whh_b = o; o += al(l.bwd_ok ? (size_t)l.D * l.bwd.nu * l.G * l.bwd.U * 4 : 0);
+    const size_t Hp = (size_t)((l.H + 3) & ~3);
+    l.whh_b = o; o += al(l.bwd_ok ? (size_t)l.D * l.bwd.nu * 4 * l.bwd.U * Hp * 4 : 0);
     l.gx = o; o += al(TB * l.D * l.G * 4);
+    l.hT = o; o += al(TB * l.D * l.H * l.es);
     l.seq[0] = o; o += al(TB * l.D * l.H * l.es);
     l.seq[1] = o; o += al(TB * l.D * l.H * l.es);
     const size_t maxin = (size_t)(l.I > l.D * l.H ? l.I : l.D * l.H);
@@ -184,8 +186,9 @@ bool make_layout(const lstm_desc* d, Layout& l) {
         l.dseq[1] = o; o += al(TB * maxin * 4);
         l.xt = o; o += al(TB * l.I * 4);
         l.dbpart = o; o += al((size_t)l.D * (l.bwd_ok ? l.bwd.nbg : 1) * l.G * 4);
+        l.P = o; o += al(l.bwd_ok ? (size_t)2 * l.D * l.bwd.nbg * l.bwd.nu * l.bwd.Bg * Hp * 4 : 0);
     } else {
-        l.dG = l.dseq[0] = l.dseq[1] = l.xt = l.dbpart = 0;
+        l.dG = l.dseq[0] = l.dseq[1] = l.xt = l.dbpart = l.P = 0;
     }
     l.total = o;
     size_t r = 0;
@@ -374,7 +377,8 @@ lstm_status lstm_forward(const lstm_desc* desc, const void* x, const void* h0, c
         f.h0 = h0 ? static_cast<const char*>(h0) + (size_t)k * state_elems * es : nullptr;
         f.c0 = c0 ? c0 + (size_t)k * state_elems : nullptr;
         void* hseq = reserve ? P(reserve, l.hseq[k]) : P(workspace, l.seq[k & 1]);
-        f.hseq = hseq;
+        f.hseq = (k < L - 1 || reserve) ? hseq : nullptr;
+        f.hT = P(workspace, l.hT);
         if (k == L - 1) {
             f.out = out;
             f.out_st = desc->batch_first ? (long long)D * H : (long long)B * D * H;
@@ -473,11 +477,12 @@ lstm_status lstm_backward(const lstm_desc* desc, const void* x, const void* h0, 
         pb.H = H; pb.D = D; pb.nu = l.bwd.nu; pb.U = l.bwd.U;
         for (int d = 0; d < D; ++d) pb.w[d] = static_cast<const float*>(w_hh[k * D + d]);
         pb.out = reinterpret_cast<float*>(P(workspace, l.whh_b));
-        LSTM_CUDA(timed(K_PACK, stream, [&] { return launch_pack_hh_bwd(pb, stream); }));
+        LSTM_CUDA(timed(K_PACK, stream, [&] { return launch_pack_hh_rows(pb, stream); }));
 
         BwdRecArgs b{};
         b.H = H; b.B = B; b.T = T; b.D = D; b.p = l.bwd;
-        b.wt = reinterpret_cast<const float*>(P(workspace, l.whh_b));
+        b.wr = reinterpret_cast<const float*>(P(workspace, l.whh_b));
+        b.P = reinterpret_cast<float*>(P(workspace, l.P));
         b.act = reinterpret_cast<const float*>(static_cast<const char*>(reserve) + l.act[k]);
         b.cst = reinterpret_cast<const float*>(static_cast<const char*>(reserve) + l.cst[k]);
         b.c0 = c0 ? c0 + (size_t)k * state : nullptr;

@@ -52,14 +52,14 @@ struct PackHhFwdArgs {
 };
 cudaError_t launch_pack_hh_fwd(const PackHhFwdArgs& a, cudaStream_t s);
 
-// Backward recurrent weights (float32): [D][nu][G][U]: element (r, jl) is
-// W_hh[r][j*U + jl], standard row order r, zero padded.
+// Backward recurrent weights (float32): [D][nu*4U][Hp]; row p = 4u + q holds
+// W_hh[q*H + u][:], zero padded.
 struct PackHhBwdArgs {
     int H, D, nu, U;
     const float* w[2];
     float* out;
 };
-cudaError_t launch_pack_hh_bwd(const PackHhBwdArgs& a, cudaStream_t s);
+cudaError_t launch_pack_hh_rows(const PackHhBwdArgs& a, cudaStream_t s);
 
 // ---------------------------------------------------------------- recurrence
 struct RecPlan {
@@ -76,6 +76,7 @@ struct FwdRecArgs {
     const void* wpk;            // PackHhFwd layout
     const void* h0;             // [D][B][H] or null
     const float* c0;            // [D][B][H] or null
+    void* hT;                   // [D][T][H][B] exchange copy of h (k-major)
     void* hseq;                 // [T][B][D*H] layer output, time-major
     void* out; long long out_st, out_sb;   // user out (top layer) or null; element strides
     void* h_n; float* c_n;      // [D][B][H]
@@ -90,7 +91,7 @@ RecPlan plan_fwd_rec(int H, int B, int D, DType dt, int num_sms, size_t smem_max
 struct BwdRecArgs {
     int H, B, T, D;
     RecPlan p;
-    const float* wt;            // PackHhBwd layout
+    const float* wr;            // [D][nu*4U][Hp] W_hh rows, packed order 4u+q
     const float* act;           // [D][T][B][G] packed
     const float* cst;           // [D][T][B][H]
     const float* c0;            // [D][B][H] or null
@@ -100,6 +101,7 @@ struct BwdRecArgs {
     float* dG;                  // [T][B][D*G], standard row order per direction
     float* dh0; float* dc0;     // [D][B][H]
     float* dbpart;              // [D][nbg][G]
+    float* P;                   // [2][D][nbg][nu][Bg][Hp] partial dh exchange
     unsigned* ctr;
     int* status;
     uint64_t timeout_ns;

@@ -1,0 +1,612 @@
+// Persistent recurrences on the CUDA cores (FFMA): the LSTM forward time loop
+// and the BPTT gate-gradient time loop.
+//
+// Cell: warp_nn "Long Short-Term Memory (LSTM)" page, equation block
+// (i, f, g, o; c' = f*c + i*g; h' = o*tanh(c')).  Backward: reverse-mode
+// differentiation of the unrolled loop ("LSTM Forward Computation", Loop
+// Unroll), weight gradients summed over all steps (pulsatrix LSTMModule,
+// backward()).
+//
+// Both kernels run one cooperative grid of D x nbg x nu blocks: direction d,
+// batch group bg (rows [bg*Bg, bg*Bg+Bg)), and unit slice j (hidden units
+// [j*U, j*U+U)).  A block keeps the 4U rows of W_hh that belong to its units
+// in shared memory for the whole sequence.  Blocks of one (d, bg) group meet
+// once per step on a counter (bounded wait, see lstm_device.cuh).
+//
+//  forward  step: gather h_{t-1} of the group's rows (k-major exchange buffer
+//                 hT[t][k][b]), a = W_slice h + Gx[t], gates, c/h update,
+//                 write h_t (exchange, layer output, user output).
+//  backward step: dh = dy_t + dh_rec for the block's units, gate derivatives
+//                 and the dc carry -> da_t (the block's 4U gate rows); the
+//                 block multiplies its own rows into a partial
+//                 dh_{t-1}[b][0..H) = sum_{r in block} W_hh[r][:] da_t[r]
+//                 and the owners of each unit add the nu partials in a fixed
+//                 order after the step's barrier (a reduce-scatter whose
+//                 traffic equals the forward's all-gather of h).
+#include <algorithm>
+
+#include "lstm_device.cuh"
+#include "lstm_internal.h"
+
+namespace lstm {
+namespace {
+
+__device__ __forceinline__ size_t align16(size_t x) { return (x + 15) & ~size_t(15); }
+inline size_t align16h(size_t x) { return (x + 15) & ~size_t(15); }
+
+// C[r][n] = sum_k A[k*lda + r] * X[k*ldx + n] for r < R, n < N, k < K, with
+// R, N, K multiples of 4.  Each thread computes a 4 x 4 tile over one of KS
+// K-slices and hands it to st(ks, r0, n0, acc).  Lanes of a warp cover an
+// 8 x 4 block of tiles of the same K-slice, so every shared-memory load of a
+// warp touches at most 128 contiguous bytes of A and of X.
+template <typename AT, typename XT, typename St>
+__device__ __forceinline__ void block_mm(const AT* __restrict__ A, int lda, const XT* __restrict__ X,
+                                         int ldx, int R, int N, int K, int KS, St&& st) {
+    const int nRT = R >> 2, nNT = N >> 2;
+    const int wr = nRT >= 8 ? 8 : (nRT >= 4 ? 4 : (nRT >= 2 ? 2 : 1));
+    const int wn = 32 / wr;
+    const int nRB = (nRT + wr - 1) / wr, nNB = (nNT + wn - 1) / wn;
+    const int nblk = nRB * nNB;
+    const int KL = (((K >> 2) + KS - 1) / KS) << 2;
+    const int items = KS * nblk * 32;
+    for (int it = threadIdx.x; it < items; it += blockDim.x) {
+        const int lane = it & 31, wi = it >> 5;
+        const int blk = wi % nblk, ks = wi / nblk;
+        const int rt = (blk % nRB) * wr + lane % wr;
+        const int nt = (blk / nRB) * wn + lane / wr;
+        if (rt >= nRT || nt >= nNT) continue;
+        const int k0 = ks * KL, k1 = min(K, k0 + KL);
+        float acc[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+        const AT* ap = A + rt * 4;
+        const XT* xp = X + nt * 4;
+#pragma unroll 2
+        for (int k = k0; k < k1; k += 4) {
+            float a[4][4], x[4][4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                load4(ap + (size_t)(k + q) * lda, a[q]);
+                load4(xp + (size_t)(k + q) * ldx, x[q]);
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[q][i], x[q][j], acc[i][j]);
+        }
+        st(ks, rt * 4, nt * 4, acc);
+    }
+}
+
+template <typename T> struct Vec4;
+template <> struct Vec4<float> {
+    typedef float4 type;
+    static __device__ __forceinline__ float4 zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
+};
+template <> struct Vec4<bf16> {
+    typedef uint2 type;
+    static __device__ __forceinline__ uint2 zero() { return make_uint2(0u, 0u); }
+};
+
+// dst[r*ncols + c] = src[r*ld + c] for r < nrv, c < ncv, zero elsewhere in the
+// nrows x ncols tile.  L1 is bypassed (rows are written by other blocks during
+// the kernel); 8 loads per thread are in flight before their stores.
+template <typename T>
+__device__ __forceinline__ void copy_tile(T* __restrict__ dst, int nrows, int ncols,
+                                          const T* __restrict__ src, size_t ld, int nrv, int ncv) {
+    constexpr int UN = 8;
+    const int tid = threadIdx.x, nth = blockDim.x;
+    const bool vec = (ncols & 3) == 0 && ncv == ncols && (ld & 3) == 0 &&
+                     (reinterpret_cast<uintptr_t>(src) & (4 * sizeof(T) - 1)) == 0;
+    if (vec) {
+        typedef typename Vec4<T>::type V;
+        const int cv = ncols >> 2;
+        const int total = nrows * cv;
+        for (int base = tid; base < total; base += nth * UN) {
+            V v[UN];
+#pragma unroll
+            for (int u = 0; u < UN; ++u) {
+                const int i = base + u * nth;
+                v[u] = Vec4<T>::zero();
+                if (i < total && i / cv < nrv)
+                    v[u] = __ldcg(reinterpret_cast<const V*>(src + (size_t)(i / cv) * ld) + i % cv);
+            }
+#pragma unroll
+            for (int u = 0; u < UN; ++u) {
+                const int i = base + u * nth;
+                if (i < total) reinterpret_cast<V*>(dst)[i] = v[u];
+            }
+        }
+    } else {
+        const int total = nrows * ncols;
+        for (int base = tid; base < total; base += nth * UN) {
+            T v[UN];
+#pragma unroll
+            for (int u = 0; u < UN; ++u) {
+                const int i = base + u * nth;
+                v[u] = from_f<T>(0.f);
+                const int r = i / ncols, c = i % ncols;
+                if (i < total && r < nrv && c < ncv) v[u] = ld_cg(src + (size_t)r * ld + c);
+            }
+#pragma unroll
+            for (int u = 0; u < UN; ++u) {
+                const int i = base + u * nth;
+                if (i < total) dst[i] = v[u];
+            }
+        }
+    }
+}
+
+inline int pick_ks(int R, int N, int K) {
+    const int nT = (R / 4) * (N / 4);
+    int ks = 1;
+    while (nT * ks * 2 <= 256 && K / (ks * 2) >= 16) ks *= 2;
+    return ks;
+}
+
+// ============================================================== forward
+template <typename WT>
+__global__ void __launch_bounds__(256, 1) fwd_rec_kernel(FwdRecArgs a) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    const RecPlan& p = a.p;
+    const int H = a.H, B = a.B, T = a.T, D = a.D, G = 4 * H;
+    const int Hp = (H + 3) & ~3;
+    const int U = p.U, R = 4 * U, Bs = p.Bs, KS = p.KS;
+    WT* Ws = reinterpret_cast<WT*>(smem);                              // [Hp][R]
+    size_t off = align16((size_t)Hp * R * sizeof(WT));
+    WT* hs = reinterpret_cast<WT*>(smem + off);                        // [Hp][Bs]
+    off += align16((size_t)Hp * Bs * sizeof(WT));
+    float* red = reinterpret_cast<float*>(smem + off);                 // [KS][R][Bs]
+    off += align16((size_t)KS * R * Bs * sizeof(float));
+    float* cs = reinterpret_cast<float*>(smem + off);                  // [U][Bg]
+
+    const int j = blockIdx.x % p.nu;
+    const int bg = (blockIdx.x / p.nu) % p.nbg;
+    const int d = blockIdx.x / (p.nu * p.nbg);
+    const int u0 = j * U, nU = min(U, H - u0);
+    const int b0 = bg * p.Bg, nB = min(p.Bg, B - b0);
+    const WT* h0 = static_cast<const WT*>(a.h0);
+    WT* hT = static_cast<WT*>(a.hT);
+    WT* hseq = static_cast<WT*>(a.hseq);
+    WT* out = static_cast<WT*>(a.out);
+    WT* h_n = static_cast<WT*>(a.h_n);
+    const int tid = threadIdx.x, nth = blockDim.x;
+
+    {
+        typedef typename Vec4<WT>::type V;
+        const V* s4 = reinterpret_cast<const V*>(static_cast<const WT*>(a.wpk) +
+                                                 ((size_t)d * p.nu + j) * Hp * R);
+        V* d4 = reinterpret_cast<V*>(Ws);
+        for (int i = tid; i < Hp * R / 4; i += nth) d4[i] = s4[i];
+    }
+    for (int i = tid; i < U * p.Bg; i += nth) {
+        const int ul = i / p.Bg, bl = i % p.Bg;
+        float c = 0.f;
+        if (a.c0 && ul < nU && bl < nB) c = a.c0[((size_t)d * B + b0 + bl) * H + u0 + ul];
+        cs[i] = c;
+    }
+    __syncthreads();
+    if (nB <= 0) return;   // plans never leave a group empty
+
+    unsigned* ctr = a.ctr + d * p.nbg + bg;
+    const size_t ldseq = (size_t)D * H;
+    const int np0 = nU * min(Bs, nB);
+    auto store_red = [&](int ks, int r0, int n0, float (&acc)[4][4]) {
+        float* rp = red + ((size_t)ks * R + r0) * Bs + n0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            *reinterpret_cast<float4*>(rp + (size_t)i * Bs) =
+                make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+    };
+    for (int s = 0; s < T; ++s) {
+        const int t = d == 0 ? s : T - 1 - s;
+        const int tp = d == 0 ? t - 1 : t + 1;
+        // Gx of this thread's first-sub-tile pairs does not depend on other
+        // blocks: fetch it before waiting.  Pair i: row bl = i % nb, unit ul = i / nb.
+        const int nb0 = min(Bs, nB);
+        float4 gxp[2];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const int i = tid + q * nth;
+            gxp[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (i < np0) {
+                const int bl = i % nb0, ul = i / nb0;
+                gxp[q] = *reinterpret_cast<const float4*>(
+                    a.gx + ((size_t)t * B + b0 + bl) * (size_t)(D * G) + (size_t)d * G + 4 * (u0 + ul));
+            }
+        }
+        if (s > 0 && p.nu > 1) {
+            if (!block_wait_geq(ctr, (unsigned)(p.nu * s), a.status, a.timeout_ns)) return;
+        }
+        for (int bs0 = 0; bs0 < nB; bs0 += Bs) {
+            const int nb = min(Bs, nB - bs0);
+            if (s == 0) {
+                for (int i = tid; i < Hp * Bs; i += nth) {
+                    const int k = i / Bs, bl = i % Bs;
+                    WT v = from_f<WT>(0.f);
+                    if (h0 && k < H && bl < nb) v = h0[((size_t)d * B + b0 + bs0 + bl) * H + k];
+                    hs[i] = v;
+                }
+            } else {
+                copy_tile(hs, Hp, Bs, hT + (((size_t)d * T + tp) * H) * B + b0 + bs0, (size_t)B, H, nb);
+            }
+            __syncthreads();
+            block_mm(Ws, R, hs, Bs, R, Bs, Hp, KS, store_red);
+            __syncthreads();
+            for (int i = tid, q = 0; i < nU * nb; i += nth, ++q) {
+                const int bl = i % nb, ul = i / nb;
+                const int b = b0 + bs0 + bl, u = u0 + ul;
+                float4 gxv;
+                if (bs0 == 0 && q < 2) {
+                    gxv = gxp[q];
+                } else {
+                    gxv = *reinterpret_cast<const float4*>(
+                        a.gx + ((size_t)t * B + b) * (size_t)(D * G) + (size_t)d * G + 4 * u);
+                }
+                float pre[4] = {gxv.x, gxv.y, gxv.z, gxv.w};
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    float acc = 0.f;
+                    for (int ks = 0; ks < KS; ++ks) acc += red[((size_t)ks * R + 4 * ul + g) * Bs + bl];
+                    pre[g] += acc;
+                }
+                const float ig = sigmoidf_(pre[0]);
+                const float fg = sigmoidf_(pre[1]);
+                const float gg = tanhf(pre[2]);
+                const float og = sigmoidf_(pre[3]);
+                float& cref = cs[ul * p.Bg + bs0 + bl];
+                const float c = fg * cref + ig * gg;
+                cref = c;
+                const float h = og * tanhf(c);
+                const WT hv = from_f<WT>(h);
+                hT[(((size_t)d * T + t) * H + u) * B + b] = hv;
+                if (hseq) hseq[((size_t)t * B + b) * ldseq + (size_t)d * H + u] = hv;
+                if (out) out[(size_t)t * a.out_st + (size_t)b * a.out_sb + (size_t)d * H + u] = hv;
+                if (a.act) {
+                    *reinterpret_cast<float4*>(a.act + (((size_t)d * T + t) * B + b) * G + 4 * u) =
+                        make_float4(ig, fg, gg, og);
+                    a.cst[(((size_t)d * T + t) * B + b) * H + u] = c;
+                }
+                if (s == T - 1) {
+                    h_n[((size_t)d * B + b) * H + u] = hv;
+                    a.c_n[((size_t)d * B + b) * H + u] = c;
+                }
+            }
+            __syncthreads();
+        }
+        if (p.nu > 1 && s + 1 < T) block_arrive(ctr);
+    }
+}
+
+// ============================================================== backward
+struct BwdPre {
+    float dy, c, cp;
+    float4 act;
+};
+
+__device__ __forceinline__ BwdPre bwd_fetch(const BwdRecArgs& a, int d, int t, int b, int jj) {
+    const int H = a.H, B = a.B, T = a.T, G = 4 * H;
+    BwdPre r;
+    r.dy = a.dy[(size_t)t * a.dy_st + (size_t)b * a.dy_sb + (size_t)d * H + jj];
+    r.act = *reinterpret_cast<const float4*>(a.act + (((size_t)d * T + t) * B + b) * G + 4 * jj);
+    r.c = a.cst[(((size_t)d * T + t) * B + b) * H + jj];
+    const int tpf = d == 0 ? t - 1 : t + 1;
+    const bool has_prev = d == 0 ? (t >= 1) : (t + 1 < T);
+    r.cp = has_prev ? a.cst[(((size_t)d * T + tpf) * B + b) * H + jj]
+                    : (a.c0 ? a.c0[((size_t)d * B + b) * H + jj] : 0.f);
+    return r;
+}
+
+__global__ void __launch_bounds__(256, 1) bwd_rec_kernel(BwdRecArgs a) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    const RecPlan& p = a.p;
+    const int H = a.H, B = a.B, T = a.T, D = a.D, G = 4 * H;
+    const int Hp = (H + 3) & ~3;
+    const int U = p.U, R4 = 4 * U, Bs = p.Bs, Bg = p.Bg;
+    float* Wr = reinterpret_cast<float*>(smem);                       // [4U][Hp]
+    size_t off = align16((size_t)R4 * Hp * 4);
+    float* daT = reinterpret_cast<float*>(smem + off);                // [4U][Bs]
+    off += align16((size_t)R4 * Bs * 4);
+    float* dcs = reinterpret_cast<float*>(smem + off);                // [U][Bg]
+    off += align16((size_t)U * Bg * 4);
+    float* dhs = reinterpret_cast<float*>(smem + off);                // [U][Bg]
+    off += align16((size_t)U * Bg * 4);
+    float* dbacc = reinterpret_cast<float*>(smem + off);              // [4][U][Bg]
+    off += align16((size_t)4 * U * Bg * 4);
+    float* gpart = reinterpret_cast<float*>(smem + off);              // [CG][U][Bg]
+
+    const int j = blockIdx.x % p.nu;
+    const int bg = (blockIdx.x / p.nu) % p.nbg;
+    const int d = blockIdx.x / (p.nu * p.nbg);
+    const int j0 = j * U, nU = min(U, H - j0);
+    const int b0 = bg * Bg, nB = min(Bg, B - b0);
+    const int tid = threadIdx.x, nth = blockDim.x;
+    {
+        const float4* s4 = reinterpret_cast<const float4*>(a.wr + ((size_t)d * p.nu + j) * R4 * Hp);
+        float4* d4 = reinterpret_cast<float4*>(Wr);
+        for (int i = tid; i < R4 * Hp / 4; i += nth) d4[i] = s4[i];
+    }
+    for (int i = tid; i < U * Bg; i += nth) {
+        const int ul = i / Bg, bl = i % Bg;
+        float dc = 0.f, dh = 0.f;
+        if (ul < nU && bl < nB) {
+            const size_t sidx = ((size_t)d * B + b0 + bl) * H + j0 + ul;
+            if (a.grad_cn) dc = a.grad_cn[sidx];
+            if (a.grad_hn) dh = a.grad_hn[sidx];
+        }
+        dcs[i] = dc;
+        dhs[i] = dh;
+    }
+    for (int i = tid; i < 4 * U * Bg; i += nth) dbacc[i] = 0.f;
+    __syncthreads();
+    if (nB <= 0) return;
+
+    unsigned* ctr = a.ctr + d * p.nbg + bg;
+    const size_t ldg = (size_t)D * G;
+    // partial dh buffers: P[buf][d][bg][c][Bg][Hp]
+    auto Pblk = [&](int buf, int c) {
+        return a.P + ((((size_t)buf * D + d) * p.nbg + bg) * p.nu + c) * (size_t)Bg * Hp;
+    };
+    // gather: dhs[ul][bl] = sum_c P[buf][c][bl][j0+ul] (fixed order over c)
+    const int U4 = U >> 2;
+    const int CG = std::max(1, nth / (U4 * Bg));   // as sized by plan_bwd_rec
+    auto gather = [&](int buf) {
+        for (int i = tid; i < CG * U4 * nB; i += nth) {
+            const int ul4 = i % U4, bl = (i / U4) % nB, cg = i / (U4 * nB);
+            float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+            constexpr int UN = 8;
+            for (int c0 = cg; c0 < p.nu; c0 += CG * UN) {
+                float4 v[UN];
+#pragma unroll
+                for (int u = 0; u < UN; ++u) {
+                    const int c = c0 + u * CG;
+                    v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (c < p.nu)
+                        v[u] = __ldcg(reinterpret_cast<const float4*>(Pblk(buf, c) + (size_t)bl * Hp + j0) + ul4);
+                }
+#pragma unroll
+                for (int u = 0; u < UN; ++u) {
+                    sum.x += v[u].x; sum.y += v[u].y; sum.z += v[u].z; sum.w += v[u].w;
+                }
+            }
+            float* gp = gpart + ((size_t)cg * U + 4 * ul4) * Bg + bl;
+            gp[0] = sum.x; gp[Bg] = sum.y; gp[2 * Bg] = sum.z; gp[3 * Bg] = sum.w;
+        }
+        __syncthreads();
+        for (int i = tid; i < U * nB; i += nth) {
+            const int ul = i / nB, bl = i % nB;
+            float s = 0.f;
+            for (int cg = 0; cg < CG; ++cg) s += gpart[((size_t)cg * U + ul) * Bg + bl];
+            dhs[ul * Bg + bl] = s;
+        }
+        __syncthreads();
+    };
+
+    const int nb0 = min(Bs, nB);
+    const int np0 = nU * nb0;
+    for (int s = 0; s < T; ++s) {
+        const int t = d == 0 ? T - 1 - s : s;
+        BwdPre pre[2];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const int i = tid + q * nth;
+            if (i < np0) pre[q] = bwd_fetch(a, d, t, b0 + i % nb0, j0 + i / nb0);
+        }
+        if (s > 0) {
+            if (p.nu > 1 && !block_wait_geq(ctr, (unsigned)(p.nu * s), a.status, a.timeout_ns)) return;
+            gather((s - 1) & 1);
+        }
+        for (int bs0 = 0; bs0 < nB; bs0 += Bs) {
+            const int nb = min(Bs, nB - bs0);
+            for (int i = tid, q = 0; i < U * Bs; i += nth, ++q) {
+                const int bl = i % Bs, ul = i / Bs;
+                if (ul >= nU || bl >= nb) {
+                    if (ul < U && bl < Bs)
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) daT[(4 * ul + g) * Bs + bl] = 0.f;
+                    continue;
+                }
+                const int b = b0 + bs0 + bl, jj = j0 + ul;
+                const BwdPre v = (bs0 == 0 && i < np0 && nb == nb0 && Bs == nb0 && q < 2)
+                                     ? pre[q] : bwd_fetch(a, d, t, b, jj);
+                const float ig = v.act.x, fg = v.act.y, gg = v.act.z, og = v.act.w;
+                float& dcref = dcs[ul * Bg + bs0 + bl];
+                const float dh = v.dy + dhs[ul * Bg + bs0 + bl];
+                const float th = tanhf(v.c);
+                const float dc = dcref + dh * og * (1.f - th * th);
+                const float da_i = dc * gg * ig * (1.f - ig);
+                const float da_f = dc * v.cp * fg * (1.f - fg);
+                const float da_g = dc * ig * (1.f - gg * gg);
+                const float da_o = dh * th * og * (1.f - og);
+                dcref = dc * fg;
+                float* dgp = a.dG + ((size_t)t * B + b) * ldg + (size_t)d * G + jj;
+                dgp[0] = da_i;
+                dgp[H] = da_f;
+                dgp[2 * H] = da_g;
+                dgp[3 * H] = da_o;
+                daT[(4 * ul + 0) * Bs + bl] = da_i;
+                daT[(4 * ul + 1) * Bs + bl] = da_f;
+                daT[(4 * ul + 2) * Bs + bl] = da_g;
+                daT[(4 * ul + 3) * Bs + bl] = da_o;
+                float* dba = dbacc + (size_t)ul * Bg + bs0 + bl;
+                dba[0] += da_i;
+                dba[(size_t)U * Bg] += da_f;
+                dba[(size_t)2 * U * Bg] += da_g;
+                dba[(size_t)3 * U * Bg] += da_o;
+            }
+            __syncthreads();
+            // partial dh_{t-1}[b][0..Hp) from this block's 4U gate rows
+            float* Pw = Pblk(s & 1, j) + (size_t)bs0 * Hp;
+            auto store_p = [&](int, int r0, int n0, float (&acc)[4][4]) {
+#pragma unroll
+                for (int jn = 0; jn < 4; ++jn) {
+                    if (n0 + jn < nb)
+                        *reinterpret_cast<float4*>(Pw + (size_t)(n0 + jn) * Hp + r0) =
+                            make_float4(acc[0][jn], acc[1][jn], acc[2][jn], acc[3][jn]);
+                }
+            };
+            block_mm(Wr, Hp, daT, Bs, Hp, Bs, R4, 1, store_p);
+            __syncthreads();
+        }
+        if (p.nu > 1) block_arrive(ctr);
+        else __syncthreads();
+    }
+    if (T > 0) {
+        if (p.nu > 1 && !block_wait_geq(ctr, (unsigned)(p.nu * T), a.status, a.timeout_ns)) return;
+        gather((T - 1) & 1);
+    }
+    for (int i = tid; i < nU * nB; i += nth) {
+        const int ul = i / nB, bl = i % nB;
+        const size_t sidx = ((size_t)d * B + b0 + bl) * H + j0 + ul;
+        a.dh0[sidx] = dhs[ul * Bg + bl];
+        a.dc0[sidx] = dcs[ul * Bg + bl];
+    }
+    // bias-gradient partial of this block: sum over its batch rows, fixed order
+    for (int i = tid; i < 4 * nU; i += nth) {
+        const int q = i / nU, ul = i % nU;
+        const float* row = dbacc + ((size_t)q * U + ul) * Bg;
+        float sum = 0.f;
+        for (int bl = 0; bl < nB; ++bl) sum += row[bl];
+        a.dbpart[((size_t)d * p.nbg + bg) * G + (size_t)q * H + j0 + ul] = sum;
+    }
+}
+
+// Backward weight rows: out[d][p][k] (p < nu*4U, k < Hp) = W_hh[(p&3)*H + p/4][k],
+// zero outside the matrix.
+__global__ void pack_hh_rows_kernel(PackHhBwdArgs a) {
+    const int Hp = (a.H + 3) & ~3;
+    const int Rt = 4 * a.U * a.nu;
+    const long long total = (long long)a.D * Rt * Hp;
+    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
+         e += (long long)gridDim.x * blockDim.x) {
+        const int k = (int)(e % Hp);
+        const long long r2 = e / Hp;
+        const int pr = (int)(r2 % Rt), d = (int)(r2 / Rt);
+        const int u = pr >> 2;
+        a.out[e] = (u < a.H && k < a.H) ? a.w[d][((long long)(pr & 3) * a.H + u) * a.H + k] : 0.f;
+    }
+}
+
+}  // namespace
+
+// ================================================================ planning
+RecPlan plan_fwd_rec(int H, int B, int D, DType dt, int num_sms, size_t smem_max) {
+    const size_t es = dtype_size(dt);
+    const int Hp = (H + 3) & ~3;
+    RecPlan best{};
+    double best_cost = 1e300;
+    const int Us[] = {1, 2, 4, 8, 16, 32, 64};
+    for (int U : Us) {
+        const int nu = (H + U - 1) / U;
+        if (U > 1 && (U / 2) >= H) break;
+        for (int nbg = 1; nbg <= std::max(B, 1); ++nbg) {
+            const int ctas = D * nbg * nu;
+            if (ctas > num_sms) break;
+            const int Bg = (B + nbg - 1) / nbg;
+            if (nbg > 1 && (nbg - 1) * Bg >= B) continue;   // a group would be empty
+            int Bs = std::min(((Bg + 3) / 4) * 4, 64);
+            RecPlan pl{};
+            bool ok = false;
+            for (; Bs >= 4; Bs -= 4) {
+                const int R = 4 * U;
+                const int KS = pick_ks(R, Bs, Hp);
+                const size_t smem = align16h((size_t)Hp * R * es) + align16h((size_t)Hp * Bs * es) +
+                                    align16h((size_t)KS * R * Bs * 4) + align16h((size_t)U * Bg * 4);
+                if (smem <= smem_max) {
+                    pl = RecPlan{nbg, Bg, nu, U, Bs, KS, 256, smem, ctas};
+                    ok = true;
+                    break;
+                }
+            }
+            if (!ok) continue;
+            const int nsub = (Bg + pl.Bs - 1) / pl.Bs;
+            // per-step time estimate in SM cycles: FFMA work at ~75% of the SM's
+            // 128 lanes, the exchange read (L2 bytes per block), fixed per-sub-tile
+            // latency, and the group synchronisation
+            const double fma = 4.0 * U * nsub * pl.Bs * (double)Hp;
+            const double l2 = (double)Hp * Bg * es;
+            const double cost = fma / 96.0 + l2 / 64.0 + nsub * 1500.0 + (nu > 1 ? 2500.0 : 0.0) +
+                                (double)ctas * 1e-3;
+            if (cost < best_cost) {
+                best_cost = cost;
+                best = pl;
+            }
+        }
+    }
+    return best;
+}
+
+RecPlan plan_bwd_rec(int H, int B, int D, int num_sms, size_t smem_max) {
+    const int Hp = (H + 3) & ~3;
+    RecPlan best{};
+    double best_cost = 1e300;
+    const int Us[] = {4, 8, 16, 32};
+    for (int U : Us) {
+        const int nu = (H + U - 1) / U;
+        if (U > 4 && (U / 2) >= H) break;
+        for (int nbg = 1; nbg <= std::max(B, 1); ++nbg) {
+            const int ctas = D * nbg * nu;
+            if (ctas > num_sms) break;
+            const int Bg = (B + nbg - 1) / nbg;
+            if (nbg > 1 && (nbg - 1) * Bg >= B) continue;
+            int Bs = std::min(((Bg + 3) / 4) * 4, 64);
+            RecPlan pl{};
+            bool ok = false;
+            for (; Bs >= 4; Bs -= 4) {
+                const int CG = std::max(1, 256 / ((U / 4) * std::min(Bg, 256)));
+                const size_t smem = align16h((size_t)4 * U * Hp * 4) + align16h((size_t)4 * U * Bs * 4) +
+                                    2 * align16h((size_t)U * Bg * 4) + align16h((size_t)4 * U * Bg * 4) +
+                                    align16h((size_t)CG * U * Bg * 4);
+                if (smem <= smem_max) {
+                    pl = RecPlan{nbg, Bg, nu, U, Bs, 1, 256, smem, ctas};
+                    ok = true;
+                    break;
+                }
+            }
+            if (!ok) continue;
+            const int nsub = (Bg + pl.Bs - 1) / pl.Bs;
+            const double fma = 4.0 * U * nsub * pl.Bs * (double)Hp;
+            const double l2 = (double)nu * Bg * U * 4 + (double)Bg * Hp * 4;
+            const double cost = fma / 96.0 + l2 / 64.0 + nsub * 1500.0 + (nu > 1 ? 2500.0 : 0.0) +
+                                (double)ctas * 1e-3;
+            if (cost < best_cost) {
+                best_cost = cost;
+                best = pl;
+            }
+        }
+    }
+    return best;
+}
+
+// ================================================================ launchers
+cudaError_t launch_fwd_rec(const FwdRecArgs& a, cudaStream_t s) {
+    FwdRecArgs args = a;
+    void* params[] = {&args};
+    const void* fn = a.dt == DType::F32 ? reinterpret_cast<const void*>(&fwd_rec_kernel<float>)
+                                        : reinterpret_cast<const void*>(&fwd_rec_kernel<bf16>);
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)a.p.smem);
+    if (e != cudaSuccess) return e;
+    return cudaLaunchCooperativeKernel(fn, dim3(a.p.ctas), dim3(a.p.threads), params, a.p.smem, s);
+}
+
+cudaError_t launch_bwd_rec(const BwdRecArgs& a, cudaStream_t s) {
+    BwdRecArgs args = a;
+    void* params[] = {&args};
+    const void* fn = reinterpret_cast<const void*>(&bwd_rec_kernel);
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)a.p.smem);
+    if (e != cudaSuccess) return e;
+    return cudaLaunchCooperativeKernel(fn, dim3(a.p.ctas), dim3(a.p.threads), params, a.p.smem, s);
+}
+
+cudaError_t launch_pack_hh_rows(const PackHhBwdArgs& a, cudaStream_t s) {
+    const long long total = (long long)a.D * 4 * a.U * a.nu * ((a.H + 3) & ~3);
+    const long long g = std::min<long long>(std::max<long long>((total + 255) / 256, 1), 148LL * 16);
+    pack_hh_rows_kernel<<<(int)g, 256, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace lstm
