@@ -106,6 +106,17 @@ cudaError_t timed(int kind, cudaStream_t s, F&& f) {
     return cudaSuccess;
 }
 
+// GEMM engine: tensor cores where the operands meet TMA's alignment rules,
+// the CUDA-core kernel otherwise.  LSTM_B200_GEMM=simt forces the CUDA-core
+// kernel everywhere (used by the tests to cover both engines).
+bool tc_gemm_enabled() {
+    static const bool v = [] {
+        const char* e = getenv("LSTM_B200_GEMM");
+        return !(e && strcmp(e, "simt") == 0);
+    }();
+    return v;
+}
+
 constexpr size_t kAlign = 256;
 inline size_t al(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 
@@ -120,7 +131,7 @@ struct Layout {
     bool bwd_ok;
     // workspace offsets
     size_t status, ctr_f, ctr_b, wih[32], bias[32], whh_f, whh_b, gx, hT, seq[2], dG, dseq[2], xt,
-        dbpart, P, total;
+        dbpart, P, dGT, bop, wcatT, total;
     // reserve offsets
     size_t act[32], cst[32], hseq[32], rtotal;   // per layer: [D][T][B][G], [D][T][B][H], [T][B][D*H]
 };
@@ -187,8 +198,11 @@ bool make_layout(const lstm_desc* d, Layout& l) {
         l.xt = o; o += al(TB * l.I * 4);
         l.dbpart = o; o += al((size_t)l.D * (l.bwd_ok ? l.bwd.nbg : 1) * l.G * 4);
         l.P = o; o += al(l.bwd_ok ? (size_t)2 * l.D * l.bwd.nbg * l.bwd.nu * l.bwd.Bg * Hp * 4 : 0);
+        l.dGT = o; o += al(TB * l.D * l.G * 4);
+        l.bop = o; o += al((size_t)l.D * (maxin + l.H) * TB * 4);
+        l.wcatT = o; o += al(maxin * l.D * l.G * 4);
     } else {
-        l.dG = l.dseq[0] = l.dseq[1] = l.xt = l.dbpart = l.P = 0;
+        l.dG = l.dseq[0] = l.dseq[1] = l.xt = l.dbpart = l.P = l.dGT = l.bop = l.wcatT = 0;
     }
     l.total = o;
     size_t r = 0;
@@ -362,7 +376,17 @@ lstm_status lstm_forward(const lstm_desc* desc, const void* x, const void* h0, c
         g.bias = reinterpret_cast<const float*>(P(workspace, l.bias[k]));
         g.accumulate = 0;
         if (k == 0 && desc->batch_first) { g.remap_T = T; g.remap_B = B; }
-        LSTM_CUDA(timed(K_PROJ, stream, [&] { return launch_gemm(g, stream); }));
+        TcGemmArgs tg{};
+        tg.M = g.M; tg.N = g.N; tg.K = g.K; tg.dt = l.dt;
+        tg.A = g.A; tg.lda = in; tg.B = g.B; tg.ldb = in;
+        tg.C = static_cast<float*>(g.C); tg.ldc = g.ldc;
+        tg.bias = g.bias; tg.remap_T = g.remap_T; tg.remap_B = g.remap_B;
+        tg.status = status; tg.timeout_ns = timeout_ns();
+        if (tc_gemm_enabled() && tc_gemm_supported(tg)) {
+            LSTM_CUDA(timed(K_PROJ, stream, [&] { return launch_tc_gemm(tg, stream); }));
+        } else {
+            LSTM_CUDA(timed(K_PROJ, stream, [&] { return launch_gemm(g, stream); }));
+        }
 
         PackHhFwdArgs ph{};
         ph.H = H; ph.D = D; ph.nu = l.fwd.nu; ph.U = l.fwd.U; ph.dt = l.dt;
@@ -508,53 +532,111 @@ lstm_status lstm_backward(const lstm_desc* desc, const void* x, const void* h0, 
                                        : reinterpret_cast<const float*>(static_cast<const char*>(reserve) + l.hseq[k - 1]);
         const float* hs = reinterpret_cast<const float*>(static_cast<const char*>(reserve) + l.hseq[k]);
         const long long ldg = (long long)D * G, ldh = (long long)D * H;
-        for (int d = 0; d < D; ++d) {
-            // dW_ih = sum_t dG_t^T x_t
-            GemmArgs g{};
-            g.M = G; g.N = in; g.K = B * T;
-            g.A = dG + (size_t)d * G; g.ta = DType::F32; g.sAm = 1; g.sAk = ldg;
-            g.B = layer_in; g.tb = DType::F32; g.sBk = in; g.sBn = 1;
-            g.C = dw_ih[k * D + d]; g.tc = DType::F32; g.ldc = in;
-            LSTM_CUDA(timed(K_DW, stream, [&] { return launch_gemm(g, stream); }));
-            // dW_hh = sum_t dG_t^T h_{t-1} (h_{-1} = h0)
-            GemmArgs gh{};
-            gh.M = G; gh.N = H; gh.K = B * (T - 1);
-            gh.ta = DType::F32; gh.sAm = 1; gh.sAk = ldg;
-            gh.tb = DType::F32; gh.sBk = ldh; gh.sBn = 1;
-            gh.C = dw_hh[k * D + d]; gh.tc = DType::F32; gh.ldc = H;
-            if (d == 0) {
-                gh.A = dG + (size_t)B * ldg + (size_t)d * G;     // rows t >= 1
-                gh.B = hs + (size_t)d * H;                        // h at t-1
-            } else {
-                gh.A = dG + (size_t)d * G;                        // rows t <= T-2
-                gh.B = hs + (size_t)B * ldh + (size_t)d * H;      // h at t+1
-            }
-            if (T > 1) {
-                LSTM_CUDA(timed(K_DW, stream, [&] { return launch_gemm(gh, stream); }));
-            } else {
-                LSTM_CUDA(cudaMemsetAsync(dw_hh[k * D + d], 0, (size_t)G * H * 4, stream));
-            }
-            if (h0) {
-                GemmArgs g0 = gh;
-                g0.K = B;
-                g0.A = dG + (d == 0 ? 0 : (size_t)(T - 1) * B * ldg) + (size_t)d * G;
-                g0.B = static_cast<const float*>(h0) + ((size_t)k * D + d) * B * H;
-                g0.sBk = H;
-                g0.accumulate = 1;
-                LSTM_CUDA(timed(K_DW, stream, [&] { return launch_gemm(g0, stream); }));
-            }
-        }
-        // gradient w.r.t. the layer input: sum_d dG_d W_ih_d
+        const long long BTl = (long long)B * T;
         float* din = k == 0 ? static_cast<float*>(dx) : reinterpret_cast<float*>(P(workspace, l.dseq[cur]));
-        for (int d = 0; d < D; ++d) {
-            GemmArgs g{};
-            g.M = B * T; g.N = in; g.K = G;
-            g.A = dG + (size_t)d * G; g.ta = DType::F32; g.sAm = ldg; g.sAk = 1;
-            g.B = w_ih[k * D + d]; g.tb = DType::F32; g.sBk = in; g.sBn = 1;
-            g.C = din; g.tc = DType::F32; g.ldc = in;
-            g.accumulate = d > 0;
-            if (k == 0 && desc->batch_first) { g.remap_T = -T; g.remap_B = B; }
-            LSTM_CUDA(timed(K_DX, stream, [&] { return launch_gemm(g, stream); }));
+        // Tensor-core weight phase: dW = dG^T [In | H_prev] per direction over
+        // K = B*T (one GEMM writes dW_ih and dW_hh), dIn = dG [W_ih_0; W_ih_1].
+        float* dGT = reinterpret_cast<float*>(P(workspace, l.dGT));
+        float* bop = reinterpret_cast<float*>(P(workspace, l.bop));
+        float* wcatT = reinterpret_cast<float*>(P(workspace, l.wcatT));
+        TcGemmArgs tw{};
+        tw.M = G; tw.N = in + H; tw.K = (int)BTl; tw.dt = DType::F32;
+        tw.A = dGT; tw.lda = BTl; tw.B = bop; tw.ldb = BTl;
+        tw.C = dw_ih[k * D]; tw.ldc = in; tw.C1 = dw_hh[k * D]; tw.ldc1 = H; tw.n_split = in;
+        tw.status = status; tw.timeout_ns = timeout_ns();
+        TcGemmArgs tx{};
+        tx.M = (int)BTl; tx.N = in; tx.K = D * G; tx.dt = DType::F32;
+        tx.A = dG; tx.lda = ldg; tx.B = wcatT; tx.ldb = (long long)D * G;
+        tx.C = din; tx.ldc = in;
+        if (k == 0 && desc->batch_first) { tx.remap_T = -T; tx.remap_B = B; }
+        tx.status = status; tx.timeout_ns = timeout_ns();
+        const bool tc_ok = tc_gemm_enabled() && tc_gemm_supported(tw) && tc_gemm_supported(tx) &&
+                           (reinterpret_cast<uintptr_t>(dw_ih[k * D]) & 3) == 0;
+        if (tc_ok) {
+            TransposeArgs ta{};
+            ta.M = (int)BTl; ta.C = D * G; ta.mode = 0; ta.src = dG; ta.lds = ldg;
+            ta.dst = dGT; ta.ldd = BTl;
+            LSTM_CUDA(timed(K_COPY, stream, [&] { return launch_transpose(ta, stream); }));
+            for (int d = 0; d < D; ++d) {
+                float* bo = bop + (size_t)d * (in + H) * BTl;
+                TransposeArgs ti{};
+                ti.M = (int)BTl; ti.C = in; ti.mode = 0;
+                if (k == 0) {
+                    ti.src = static_cast<const float*>(x); ti.lds = in;
+                    ti.bt_remap = desc->batch_first; ti.T = T; ti.B = B;
+                } else {
+                    ti.src = reinterpret_cast<const float*>(static_cast<const char*>(reserve) + l.hseq[k - 1]);
+                    ti.lds = in;
+                }
+                ti.dst = bo; ti.ldd = BTl;
+                LSTM_CUDA(timed(K_COPY, stream, [&] { return launch_transpose(ti, stream); }));
+                TransposeArgs th{};
+                th.M = (int)BTl; th.C = H; th.mode = 1;
+                th.src = hs + (size_t)d * H; th.lds = ldh; th.T = T; th.B = B; th.dir = d;
+                th.h0 = h0 ? static_cast<const float*>(h0) + ((size_t)k * D + d) * B * H : nullptr;
+                th.dst = bo + (size_t)in * BTl; th.ldd = BTl;
+                LSTM_CUDA(timed(K_COPY, stream, [&] { return launch_transpose(th, stream); }));
+                TcGemmArgs twd = tw;
+                twd.A = dGT + (size_t)d * G * BTl;
+                twd.B = bo;
+                twd.C = dw_ih[k * D + d];
+                twd.C1 = dw_hh[k * D + d];
+                LSTM_CUDA(timed(K_DW, stream, [&] { return launch_tc_gemm(twd, stream); }));
+                TransposeArgs tww{};
+                tww.M = G; tww.C = in; tww.mode = 0;
+                tww.src = static_cast<const float*>(w_ih[k * D + d]); tww.lds = in;
+                tww.dst = wcatT + (size_t)d * G; tww.ldd = (long long)D * G;
+                LSTM_CUDA(timed(K_COPY, stream, [&] { return launch_transpose(tww, stream); }));
+            }
+            LSTM_CUDA(timed(K_DX, stream, [&] { return launch_tc_gemm(tx, stream); }));
+        } else {
+            for (int d = 0; d < D; ++d) {
+                // dW_ih = sum_t dG_t^T x_t
+                GemmArgs g{};
+                g.M = G; g.N = in; g.K = B * T;
+                g.A = dG + (size_t)d * G; g.ta = DType::F32; g.sAm = 1; g.sAk = ldg;
+                g.B = layer_in; g.tb = DType::F32; g.sBk = in; g.sBn = 1;
+                g.C = dw_ih[k * D + d]; g.tc = DType::F32; g.ldc = in;
+                LSTM_CUDA(timed(K_DW, stream, [&] { return launch_gemm(g, stream); }));
+                // dW_hh = sum_t dG_t^T h_{t-1} (h_{-1} = h0)
+                GemmArgs gh{};
+                gh.M = G; gh.N = H; gh.K = B * (T - 1);
+                gh.ta = DType::F32; gh.sAm = 1; gh.sAk = ldg;
+                gh.tb = DType::F32; gh.sBk = ldh; gh.sBn = 1;
+                gh.C = dw_hh[k * D + d]; gh.tc = DType::F32; gh.ldc = H;
+                if (d == 0) {
+                    gh.A = dG + (size_t)B * ldg + (size_t)d * G;     // rows t >= 1
+                    gh.B = hs + (size_t)d * H;                        // h at t-1
+                } else {
+                    gh.A = dG + (size_t)d * G;                        // rows t <= T-2
+                    gh.B = hs + (size_t)B * ldh + (size_t)d * H;      // h at t+1
+                }
+                if (T > 1) {
+                    LSTM_CUDA(timed(K_DW, stream, [&] { return launch_gemm(gh, stream); }));
+                } else {
+                    LSTM_CUDA(cudaMemsetAsync(dw_hh[k * D + d], 0, (size_t)G * H * 4, stream));
+                }
+                if (h0) {
+                    GemmArgs g0 = gh;
+                    g0.K = B;
+                    g0.A = dG + (d == 0 ? 0 : (size_t)(T - 1) * B * ldg) + (size_t)d * G;
+                    g0.B = static_cast<const float*>(h0) + ((size_t)k * D + d) * B * H;
+                    g0.sBk = H;
+                    g0.accumulate = 1;
+                    LSTM_CUDA(timed(K_DW, stream, [&] { return launch_gemm(g0, stream); }));
+                }
+            }
+            // gradient w.r.t. the layer input: sum_d dG_d W_ih_d
+            for (int d = 0; d < D; ++d) {
+                GemmArgs g{};
+                g.M = B * T; g.N = in; g.K = G;
+                g.A = dG + (size_t)d * G; g.ta = DType::F32; g.sAm = ldg; g.sAk = 1;
+                g.B = w_ih[k * D + d]; g.tb = DType::F32; g.sBk = in; g.sBn = 1;
+                g.C = din; g.tc = DType::F32; g.ldc = in;
+                g.accumulate = d > 0;
+                if (k == 0 && desc->batch_first) { g.remap_T = -T; g.remap_B = B; }
+                LSTM_CUDA(timed(K_DX, stream, [&] { return launch_gemm(g, stream); }));
+            }
         }
         if (k > 0) {
             dy = din;

@@ -29,6 +29,46 @@ struct GemmArgs {
 };
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s);
 
+// Tensor-core GEMM (tcgen05): C[M x N] = A[M x K] * B[N x K]^T (+ bias[n])
+// with both operands K-major (row strides lda, ldb elements, 16-byte
+// multiples).  F32 operands use 3xTF32, BF16 operands kind::f16; the
+// accumulator is float32.  Output column n < n_split goes to
+// C[row*ldc + n], n >= n_split to C1[row*ldc1 + n - n_split] (C1 null: all to
+// C).  Row map as in GemmArgs.  splitk > 1 needs ws (splitk*M*N floats).
+struct TcGemmArgs {
+    int M, N, K;
+    DType dt;
+    const void* A; long long lda;
+    const void* B; long long ldb;
+    float* C; long long ldc;
+    float* C1; long long ldc1; int n_split;
+    const float* bias;
+    int accumulate;
+    int remap_T, remap_B;
+    int splitk;
+    float* ws;
+    int* status;
+    uint64_t timeout_ns;
+};
+bool tc_gemm_supported(const TcGemmArgs& g);
+int tc_gemm_tile_n(DType dt);
+cudaError_t launch_tc_gemm(const TcGemmArgs& g, cudaStream_t s);
+
+// dst[c*ldd + m] = src(m, c) for m < M, c < C (float32).
+//  mode 0: src(m, c) = src[row(m)*lds + c], row(m) = m, or with bt_remap the
+//          time-major index m = t*B + b read from a batch-first (b*T + t) array.
+//  mode 1: h_{t-1} of one direction in its own time order: for m = t*B + b,
+//          src(m, c) = src[(ts*B + b)*lds + c] with ts = t-1 (dir 0) or t+1
+//          (dir 1) when 0 <= ts < T, else h0[b*C + c] (zero if h0 is null).
+struct TransposeArgs {
+    int M, C, mode;
+    const float* src; long long lds;
+    int bt_remap, T, B, dir;
+    const float* h0;
+    float* dst; long long ldd;
+};
+cudaError_t launch_transpose(const TransposeArgs& a, cudaStream_t s);
+
 // ---------------------------------------------------------------- packing
 // Gate-interleaved row order used inside the library: packed row p = 4u + q
 // holds standard row q*H + u (q = 0..3 for i, f, g, o).

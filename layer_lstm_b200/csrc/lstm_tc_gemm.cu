@@ -1,0 +1,369 @@
+// Time-batched GEMMs of the LSTM on the sm_100a tensor cores (tcgen05):
+// the input projection Gx = X W_ih^T + b over all timesteps ("LSTM Forward
+// Computation", Basic Operators: one product with the four gate matrices
+// stacked), the weight gradients dW_ih = sum_t da_t x_t^T, dW_hh =
+// sum_t da_t h_{t-1}^T (pulsatrix LSTMModule, backward()), and the
+// layer-input gradient dX = dG W_ih.
+//
+// C[M x N] = A[M x K] * B[N x K]^T with both operands K-major in global
+// memory.  One CTA computes a 128 x BN tile; warp 0 issues TMA tile loads
+// into a ring of shared-memory stages, warp 1 (one thread) issues tcgen05.mma
+// into a TMEM accumulator, warps 4-7 drain TMEM through registers to global
+// memory.  bf16 operands use kind::f16.  float32 operands use three
+// kind::tf32 products per K step, hi*hi + hi*lo + lo*hi with hi = x with its
+// low 13 mantissa bits cleared and lo = x - hi (exact in fp32); warps 2-3
+// split each stage in shared memory before the MMAs read it.  This is the
+// error-compensated 3xTF32 scheme of Ootomo & Yokota (2022), "Recovering
+// single precision accuracy from Tensor Cores while surpassing the FP32
+// theoretical peak performance"; the dropped lo*lo term and the truncation
+// of lo keep the product error near 2^-21 relative.
+#include <mutex>
+
+#include "lstm_device.cuh"
+#include "lstm_internal.h"
+#include "lstm_tc.cuh"
+
+namespace lstm {
+namespace {
+
+template <int KIND> struct Cfg;
+template <> struct Cfg<0> {   // bf16
+    static constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4, FMT = 1;
+    static constexpr int A_BYTES = BM * 128, B_BYTES = BN * 128;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+};
+template <> struct Cfg<1> {   // 3xTF32
+    static constexpr int BM = 128, BN = 128, BK = 32, STAGES = 3, FMT = 2;
+    static constexpr int A_BYTES = BM * 128, B_BYTES = BN * 128;
+    static constexpr int STAGE_BYTES = 2 * (A_BYTES + B_BYTES);   // hi tiles, then lo tiles
+};
+
+template <int KIND>
+constexpr size_t smem_bytes() {
+    return (size_t)Cfg<KIND>::STAGES * Cfg<KIND>::STAGE_BYTES + 1024 + 256;
+}
+
+struct TcEpi {
+    int M, N, K, k_per_split;
+    float* C; long long ldc;
+    float* C1; long long ldc1; int n_split;
+    const float* bias;
+    int accumulate;
+    int remap_T, remap_B;
+    float* ws;                 // split-K partials [splits][M][N] or null
+    int* status;
+    uint64_t timeout_ns;
+};
+
+__device__ __forceinline__ long long out_row(const TcEpi& e, int m) {
+    if (e.remap_T > 0) return (long long)(m % e.remap_T) * e.remap_B + m / e.remap_T;
+    if (e.remap_T < 0) return (long long)(m % e.remap_B) * (-e.remap_T) + m / e.remap_B;
+    return m;
+}
+
+// Drain wait used on the abort path only: ignores the abort flag.
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!tc::mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > 100000000ull) break;   // 0.1 s
+    }
+}
+
+template <int KIND>
+__global__ void __launch_bounds__(256, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, TcEpi e) {
+    using Cf = Cfg<KIND>;
+    constexpr int S = Cf::STAGES, BM = Cf::BM, BN = Cf::BN, BK = Cf::BK;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * Cf::STAGE_BYTES);
+    uint64_t* lofull = full + S;
+    uint64_t* empty = lofull + S;
+    uint64_t* tmem_full = empty + S;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_full + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN, split = blockIdx.z;
+    const int kbeg = split * e.k_per_split;
+    const int kend = min(e.K, kbeg + e.k_per_split);
+    const int nk = kend > kbeg ? (kend - kbeg + BK - 1) / BK : 0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            tc::mbar_init(&full[s], 1);
+            tc::mbar_init(&lofull[s], 64);
+            tc::mbar_init(&empty[s], 1);
+        }
+        tc::mbar_init(tmem_full, 1);
+        *abort_flag = 0;
+        tc::fence_mbar_init();
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(tmem_slot, BN);
+        tc::tmem_relinquish();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tc::prefetch_tmap(&tmA);
+            tc::prefetch_tmap(&tmB);
+            int issued = 0;
+            for (int kt = 0; kt < nk; ++kt) {
+                const int s = kt % S, r = kt / S;
+                if (!tc::mbar_wait(&empty[s], (r & 1) ^ 1, abort_flag, e.status, e.timeout_ns)) break;
+                unsigned char* st = smem + s * Cf::STAGE_BYTES;
+                tc::mbar_arrive_expect_tx(&full[s], Cf::A_BYTES + Cf::B_BYTES);
+                const int kx = kbeg + kt * BK;
+                tc::tma_load_2d(st, &tmA, kx, m0, &full[s]);
+                tc::tma_load_2d(st + Cf::A_BYTES, &tmB, kx, n0, &full[s]);
+                issued = kt + 1;
+            }
+            if (*abort_flag) {   // let this block's copies land before shared memory is released
+                for (int kt = issued > S ? issued - S : 0; kt < issued; ++kt) mbar_drain(&full[kt % S], (kt / S) & 1);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = tc::instr_desc(Cf::FMT, BM, BN);
+            int last = -1;
+            for (int kt = 0; kt < nk; ++kt) {
+                const int s = kt % S, r = kt / S;
+                uint64_t* ready = KIND == 1 ? &lofull[s] : &full[s];
+                if (!tc::mbar_wait(ready, r & 1, abort_flag, e.status, e.timeout_ns)) break;
+                tc::tc_fence_after();
+                unsigned char* st = smem + s * Cf::STAGE_BYTES;
+                const uint32_t a_base = tc::smem_u32(st);
+                const uint32_t b_base = a_base + Cf::A_BYTES;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint64_t ad = tc::smem_desc_sw128(a_base + j * 32);
+                    const uint64_t bd = tc::smem_desc_sw128(b_base + j * 32);
+                    const uint32_t acc = (kt | j) != 0;
+                    if (KIND == 0) {
+                        tc::mma_bf16(tmem, ad, bd, idesc, acc);
+                    } else {
+                        const uint32_t lo_off = Cf::A_BYTES + Cf::B_BYTES;
+                        const uint64_t adl = tc::smem_desc_sw128(a_base + lo_off + j * 32);
+                        const uint64_t bdl = tc::smem_desc_sw128(b_base + lo_off + j * 32);
+                        tc::mma_tf32(tmem, adl, bd, idesc, acc);    // lo * hi
+                        tc::mma_tf32(tmem, ad, bdl, idesc, 1);      // hi * lo
+                        tc::mma_tf32(tmem, ad, bd, idesc, 1);       // hi * hi
+                    }
+                }
+                tc::mma_commit(&empty[s]);
+                last = kt;
+            }
+            tc::mma_commit(tmem_full);
+            if (*abort_flag && last >= 0) mbar_drain(&empty[last % S], (last / S) & 1);
+        }
+    } else if (KIND == 1 && warp < 4) {
+        // hi/lo split of each stage (64 threads), in place for hi.
+        const int ct = threadIdx.x - 64;
+        for (int kt = 0; kt < nk; ++kt) {
+            const int s = kt % S, r = kt / S;
+            if (!tc::mbar_wait(&full[s], r & 1, abort_flag, e.status, e.timeout_ns)) break;
+            float4* hi = reinterpret_cast<float4*>(smem + s * Cf::STAGE_BYTES);
+            float4* lo = reinterpret_cast<float4*>(smem + s * Cf::STAGE_BYTES + Cf::A_BYTES + Cf::B_BYTES);
+            constexpr int NV = (Cf::A_BYTES + Cf::B_BYTES) / 16;
+#pragma unroll 4
+            for (int i = ct; i < NV; i += 64) {
+                const float4 x = hi[i];
+                float4 h, l;
+                h.x = __uint_as_float(__float_as_uint(x.x) & 0xFFFFE000u); l.x = x.x - h.x;
+                h.y = __uint_as_float(__float_as_uint(x.y) & 0xFFFFE000u); l.y = x.y - h.y;
+                h.z = __uint_as_float(__float_as_uint(x.z) & 0xFFFFE000u); l.z = x.z - h.z;
+                h.w = __uint_as_float(__float_as_uint(x.w) & 0xFFFFE000u); l.w = x.w - h.w;
+                hi[i] = h;
+                lo[i] = l;
+            }
+            tc::fence_proxy_async_smem();
+            tc::mbar_arrive(&lofull[s]);
+        }
+    } else if (warp >= 4) {
+        const int q = warp & 3;
+        const bool ok = tc::mbar_wait(tmem_full, 0, abort_flag, e.status, e.timeout_ns);
+        tc::tc_fence_after();
+        const int m = m0 + q * 32 + lane;
+        if (ok) {
+            for (int c = 0; c < BN; c += 16) {
+                float v[16];
+                tc::tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c, v);
+                tc::tmem_ld_wait();
+                if (m >= e.M) continue;
+                if (nk == 0) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] = 0.f;
+                }
+                if (e.ws) {
+                    float* dst = e.ws + ((size_t)split * e.M + m) * e.N;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        if (n0 + c + i < e.N) dst[n0 + c + i] = v[i];
+                } else {
+                    const long long row = out_row(e, m);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int n = n0 + c + i;
+                        if (n >= e.N) continue;
+                        float val = v[i] + (e.bias ? e.bias[n] : 0.f);
+                        float* dst = n < e.n_split ? e.C + row * e.ldc + n : e.C1 + row * e.ldc1 + (n - e.n_split);
+                        if (e.accumulate) val += *dst;
+                        *dst = val;
+                    }
+                }
+            }
+        }
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem, BN);
+    }
+}
+
+__global__ void splitk_reduce_kernel(TcEpi e, int splits) {
+    const long long total = (long long)e.M * e.N;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        const int m = (int)(i / e.N), n = (int)(i % e.N);
+        float val = 0.f;
+        for (int z = 0; z < splits; ++z) val += e.ws[(size_t)z * total + i];
+        val += e.bias ? e.bias[n] : 0.f;
+        const long long row = out_row(e, m);
+        float* dst = n < e.n_split ? e.C + row * e.ldc + n : e.C1 + row * e.ldc1 + (n - e.n_split);
+        if (e.accumulate) val += *dst;
+        *dst = val;
+    }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+bool make_map(CUtensorMap* map, DType dt, const void* base, long long rows, long long cols, long long ld,
+              int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const size_t es = dtype_size(dt);
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(ld * es)};
+    cuuint32_t box[2] = {(cuuint32_t)(128 / es), (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, dt == DType::F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                     2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int KIND>
+cudaError_t launch_kind(const TcGemmArgs& g, cudaStream_t s) {
+    using Cf = Cfg<KIND>;
+    CUtensorMap ta, tb;
+    if (!make_map(&ta, g.dt, g.A, g.M, g.K, g.lda, Cf::BM)) return cudaErrorInvalidValue;
+    if (!make_map(&tb, g.dt, g.B, g.N, g.K, g.ldb, Cf::BN)) return cudaErrorInvalidValue;
+    TcEpi e{};
+    e.M = g.M; e.N = g.N; e.K = g.K;
+    const int splits = g.splitk > 1 && g.ws ? g.splitk : 1;
+    const int kchunks = (g.K + Cf::BK - 1) / Cf::BK;
+    e.k_per_split = ((kchunks + splits - 1) / splits) * Cf::BK;
+    e.C = g.C; e.ldc = g.ldc;
+    e.C1 = g.C1 ? g.C1 : g.C; e.ldc1 = g.C1 ? g.ldc1 : g.ldc;
+    e.n_split = g.C1 ? g.n_split : g.N;
+    e.bias = g.bias; e.accumulate = g.accumulate;
+    e.remap_T = g.remap_T; e.remap_B = g.remap_B;
+    e.ws = splits > 1 ? g.ws : nullptr;
+    e.status = g.status; e.timeout_ns = g.timeout_ns;
+    const size_t smem = smem_bytes<KIND>();
+    cudaError_t err = cudaFuncSetAttribute(tc_gemm_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)smem);
+    if (err != cudaSuccess) return err;
+    dim3 grid((g.N + Cf::BN - 1) / Cf::BN, (g.M + Cf::BM - 1) / Cf::BM, splits);
+    tc_gemm_kernel<KIND><<<grid, 256, smem, s>>>(ta, tb, e);
+    err = cudaGetLastError();
+    if (err != cudaSuccess || splits == 1) return err;
+    const long long total = (long long)g.M * g.N;
+    const int blocks = (int)std::min<long long>((total + 255) / 256, 148LL * 8);
+    splitk_reduce_kernel<<<blocks, 256, 0, s>>>(e, splits);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_gemm_supported(const TcGemmArgs& g) {
+    if (g.M <= 0 || g.N <= 0 || g.K <= 0) return false;
+    if (!encode_fn()) return false;
+    const size_t es = dtype_size(g.dt);
+    if ((g.lda * es) % 16 != 0 || (g.ldb * es) % 16 != 0) return false;
+    if ((reinterpret_cast<uintptr_t>(g.A) & 15) || (reinterpret_cast<uintptr_t>(g.B) & 15)) return false;
+    if (g.K < (long long)(128 / es)) return false;   // at least one full 128-byte K chunk
+    return true;
+}
+
+int tc_gemm_tile_n(DType dt) { return dt == DType::F32 ? Cfg<1>::BN : Cfg<0>::BN; }
+
+cudaError_t launch_tc_gemm(const TcGemmArgs& g, cudaStream_t s) {
+    return g.dt == DType::F32 ? launch_kind<1>(g, s) : launch_kind<0>(g, s);
+}
+
+// ---------------------------------------------------------------- transposes
+namespace {
+
+__global__ void transpose_kernel(TransposeArgs a) {
+    __shared__ float tile[32][33];
+    const int m0 = blockIdx.x * 32, c0 = blockIdx.y * 32;
+    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 32 x 8 threads
+    for (int i = ty; i < 32; i += 8) {
+        const int m = m0 + i, c = c0 + tx;
+        float v = 0.f;
+        if (m < a.M && c < a.C) {
+            if (a.mode == 0) {
+                long long row = m;
+                if (a.bt_remap) row = (long long)(m % a.B) * a.T + m / a.B;   // m = t*B + b -> b*T + t
+                v = a.src[row * a.lds + c];
+            } else {
+                const int t = m / a.B, b = m % a.B;
+                const int ts = a.dir == 0 ? t - 1 : t + 1;
+                if (ts >= 0 && ts < a.T) v = a.src[((long long)ts * a.B + b) * a.lds + c];
+                else if (a.h0) v = a.h0[(long long)b * a.C + c];
+            }
+        }
+        tile[i][tx] = v;
+    }
+    __syncthreads();
+    for (int i = ty; i < 32; i += 8) {
+        const int c = c0 + i, m = m0 + tx;
+        if (m < a.M && c < a.C) a.dst[(long long)c * a.ldd + m] = tile[tx][i];
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_transpose(const TransposeArgs& a, cudaStream_t s) {
+    if (a.M <= 0 || a.C <= 0) return cudaSuccess;
+    dim3 grid((a.M + 31) / 32, (a.C + 31) / 32);
+    transpose_kernel<<<grid, 256, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace lstm
