@@ -141,6 +141,35 @@ lstm_status lstm_backward(const lstm_desc* desc, const void* x, const void* h0, 
                           float* const* dw_ih, float* const* dw_hh,
                           float* const* db_ih, float* const* db_hh, cudaStream_t stream);
 
+/*
+ * Inference forward that allocates nothing and takes no workspace.  The pages
+ * have no counterpart: this is an integration aid.  It exists for callers
+ * that cannot call cudaMalloc or size a workspace for us, such as a plugin
+ * running inside a host application that owns every byte of device memory
+ * and forbids its plugins to allocate, or a loop on a fixed memory budget
+ * where an allocation could fail or stall at an unpredictable moment.
+ *
+ * Same arguments and results as lstm_forward with reserve == NULL; the caller
+ * still passes every input and output.  The scratch is one fixed array of
+ * LSTM_NOALLOC_SCRATCH_BYTES (32 MiB) of device memory inside the library,
+ * present on every GPU where the library's device code is loaded until the
+ * process exits.  Problems whose inference workspace exceeds it return
+ * LSTM_ERR_WORKSPACE; use lstm_forward with your own workspace for those.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  Every call shares the one array: calls that may overlap on the
+ * GPU (other streams, other host threads) race and must be serialised by the
+ * caller.  The status word read by lstm_query_status lives in the array too;
+ * lstm_query_status cannot reach it, so a bounded-wait failure surfaces only
+ * through the outputs of the call.
+ */
+#define LSTM_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+lstm_status lstm_forward_noalloc(const lstm_desc* desc, const void* x, const void* h0,
+                                 const float* c0, const void* const* w_ih, const void* const* w_hh,
+                                 const void* const* b_ih, const void* const* b_hh,
+                                 void* out, void* h_n, float* c_n, cudaStream_t stream);
+
 /* Synchronises `stream` and returns the kernel-side status recorded in
  * `workspace` by the last call that used it (LSTM_OK or LSTM_ERR_TIMEOUT), or
  * LSTM_ERR_CUDA if the stream reports an error. */

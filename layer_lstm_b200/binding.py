@@ -23,7 +23,8 @@ LSTM_BF16 = 1
 
 EXPORTED = ("lstm_workspace_size", "lstm_reserve_size", "lstm_forward", "lstm_backward",
             "lstm_query_status", "lstm_status_string", "lstm_timing_enable", "lstm_timing_read",
-            "lstm_timing_reset")
+            "lstm_timing_reset", "lstm_forward_noalloc")
+LSTM_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class lstm_kernel_time(ctypes.Structure):
@@ -92,6 +93,8 @@ def load(build_if_stale: bool = True):
     lib.lstm_timing_read.restype = ctypes.c_int
     lib.lstm_timing_reset.argtypes = []
     lib.lstm_timing_reset.restype = None
+    lib.lstm_forward_noalloc.argtypes = [dp, vp, vp, vp, vpp, vpp, vpp, vpp, vp, vp, vp, vp]
+    lib.lstm_forward_noalloc.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -161,6 +164,14 @@ def lstm_backward(desc, x, h0, c0, w_ih, w_hh, grad_out, grad_hn, grad_cn, reser
                              _p(workspace), _nbytes(workspace) if ws_bytes is None else ws_bytes,
                              _p(dx), _p(dh0), _p(dc0), _parr(dw_ih), _parr(dw_hh),
                              _parr(db_ih), _parr(db_hh), _stream(stream))
+
+
+def lstm_forward_noalloc(desc, x, h0, c0, w_ih, w_hh, b_ih, b_hh, out, h_n, c_n,
+                         stream=None) -> int:
+    lib = load()
+    return lib.lstm_forward_noalloc(ctypes.byref(desc), _p(x), _p(h0), _p(c0), _parr(w_ih),
+                                    _parr(w_hh), _parr(b_ih), _parr(b_hh), _p(out), _p(h_n),
+                                    _p(c_n), _stream(stream))
 
 
 def lstm_query_status(workspace, stream=None) -> int:

@@ -223,6 +223,18 @@ inline char* P(void* base, size_t off) { return static_cast<char*>(base) + off; 
     } while (0)
 
 }  // namespace
+
+// Bytes at the start of the workspace that an inference forward
+// (reserve == NULL) reads or writes: the status word, the counters, the
+// packed weights, the projection output and the exchange / layer-output
+// buffers all lie in front of the buffers only the backward uses.
+// 0 for an invalid description.
+size_t forward_workspace_prefix(const lstm_desc* desc) {
+    Layout l;
+    if (!make_layout(desc, l)) return 0;
+    return l.seq[1] + al((size_t)l.T * l.B * l.D * l.H * l.es);
+}
+
 }  // namespace lstm
 
 using namespace lstm;
