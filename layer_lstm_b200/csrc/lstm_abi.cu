@@ -13,6 +13,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <algorithm>
 #include <mutex>
 #include <vector>
 
@@ -117,6 +118,16 @@ bool tc_gemm_enabled() {
     return v;
 }
 
+// Recurrence engine for bf16 inference: tensor cores when the plan fits,
+// otherwise the CUDA-core kernel.  LSTM_B200_REC=simt forces the latter.
+bool tc_rec_enabled() {
+    static const bool v = [] {
+        const char* e = getenv("LSTM_B200_REC");
+        return !(e && strcmp(e, "simt") == 0);
+    }();
+    return v;
+}
+
 constexpr size_t kAlign = 256;
 inline size_t al(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 
@@ -128,10 +139,12 @@ struct Layout {
     DType dt;
     size_t es;
     RecPlan fwd, bwd;
+    TcRecPlan tcr;
+    int nbg_ctr;       // counter stride per (layer, direction): max over the forward plans
     bool bwd_ok;
     // workspace offsets
     size_t status, ctr_f, ctr_b, wih[32], bias[32], whh_f, whh_b, gx, hT, seq[2], dG, dseq[2], xt,
-        dbpart, P, dGT, bop, wcatT, total;
+        dbpart, P, dGT, bop, wcatT, hx, whh_tc, bias_dummy, total;
     // reserve offsets
     size_t act[32], cst[32], hseq[32], rtotal;   // per layer: [D][T][B][G], [D][T][B][H], [T][B][D*H]
 };
@@ -174,10 +187,12 @@ bool make_layout(const lstm_desc* d, Layout& l) {
     if (l.fwd.ctas == 0) return false;
     l.bwd = plan_bwd_rec(l.H, Bp, l.D, dev.sms, smem_max);
     l.bwd_ok = l.bwd.ctas > 0;
+    l.tcr = l.dt == DType::BF16 ? plan_tc_rec(l.H, Bp, l.D, dev.sms, smem_max) : TcRecPlan{};
     const size_t TB = (size_t)l.T * l.B;
     size_t o = 0;
     l.status = o; o += al(sizeof(int));
-    l.ctr_f = o; o += al(sizeof(unsigned) * (size_t)l.L * l.D * l.fwd.nbg);
+    l.nbg_ctr = std::max(l.fwd.nbg, l.tcr.ok ? l.tcr.nbg : 0);
+    l.ctr_f = o; o += al(sizeof(unsigned) * (size_t)l.L * l.D * l.nbg_ctr);
     l.ctr_b = o; o += al(sizeof(unsigned) * (size_t)l.L * l.D * (l.bwd_ok ? l.bwd.nbg : 1));
     for (int k = 0; k < l.L; ++k) {
         l.wih[k] = o; o += al((size_t)l.D * l.G * in_size(l, k) * l.es);
@@ -190,6 +205,13 @@ bool make_layout(const lstm_desc* d, Layout& l) {
     l.hT = o; o += al(TB * l.D * l.H * l.es);
     l.seq[0] = o; o += al(TB * l.D * l.H * l.es);
     l.seq[1] = o; o += al(TB * l.D * l.H * l.es);
+    if (l.tcr.ok) {
+        l.hx = o; o += al((size_t)l.D * (l.T + 1) * l.B * l.H * 2);
+        l.whh_tc = o; o += al((size_t)l.D * l.G * l.H * 2);
+        l.bias_dummy = o; o += al((size_t)l.D * l.G * 4);
+    } else {
+        l.hx = l.whh_tc = l.bias_dummy = 0;
+    }
     const size_t maxin = (size_t)(l.I > l.D * l.H ? l.I : l.D * l.H);
     if (l.dt == DType::F32) {
         l.dG = o; o += al(TB * l.D * l.G * 4);
@@ -232,6 +254,7 @@ inline char* P(void* base, size_t off) { return static_cast<char*>(base) + off; 
 size_t forward_workspace_prefix(const lstm_desc* desc) {
     Layout l;
     if (!make_layout(desc, l)) return 0;
+    if (l.tcr.ok) return l.bias_dummy + al((size_t)l.D * l.G * 4);
     return l.seq[1] + al((size_t)l.T * l.B * l.D * l.H * l.es);
 }
 
@@ -400,6 +423,45 @@ lstm_status lstm_forward(const lstm_desc* desc, const void* x, const void* h0, c
             LSTM_CUDA(timed(K_PROJ, stream, [&] { return launch_gemm(g, stream); }));
         }
 
+        void* hseq_tc = reserve ? P(reserve, l.hseq[k]) : P(workspace, l.seq[k & 1]);
+        if (!reserve && l.tcr.ok && tc_rec_enabled()) {
+            // tensor-core recurrence: packed W_hh rows, h0 into exchange slot 0
+            PackIhArgs pw{};
+            pw.H = H; pw.in = H; pw.D = D; pw.dt = l.dt;
+            for (int d = 0; d < D; ++d) pw.w[d] = w_hh[k * D + d];
+            pw.wp = P(workspace, l.whh_tc);
+            pw.bias_p = reinterpret_cast<float*>(P(workspace, l.bias_dummy));
+            LSTM_CUDA(timed(K_PACK, stream, [&] { return launch_pack_ih(pw, stream); }));
+            for (int d = 0; d < D; ++d) {
+                char* slot0 = P(workspace, l.hx) + (size_t)d * (T + 1) * B * H * 2;
+                if (h0)
+                    LSTM_CUDA(cudaMemcpyAsync(slot0, static_cast<const char*>(h0) + ((size_t)k * D + d) * B * H * 2,
+                                              (size_t)B * H * 2, cudaMemcpyDeviceToDevice, stream));
+                else
+                    LSTM_CUDA(cudaMemsetAsync(slot0, 0, (size_t)B * H * 2, stream));
+            }
+            TcRecArgs tr{};
+            tr.H = H; tr.B = B; tr.T = T; tr.D = D; tr.p = l.tcr;
+            tr.gx = reinterpret_cast<const float*>(P(workspace, l.gx));
+            tr.wpk = P(workspace, l.whh_tc);
+            tr.c0 = c0 ? c0 + (size_t)k * state_elems : nullptr;
+            tr.hx = P(workspace, l.hx);
+            tr.hseq = k < L - 1 ? hseq_tc : nullptr;
+            if (k == L - 1) {
+                tr.out = out;
+                tr.out_st = desc->batch_first ? (long long)D * H : (long long)B * D * H;
+                tr.out_sb = desc->batch_first ? (long long)T * D * H : (long long)D * H;
+            }
+            tr.h_n = static_cast<char*>(h_n) + (size_t)k * state_elems * es;
+            tr.c_n = c_n + (size_t)k * state_elems;
+            tr.ctr = reinterpret_cast<unsigned*>(P(workspace, l.ctr_f)) + (size_t)k * D * l.nbg_ctr;
+            tr.status = status;
+            tr.timeout_ns = timeout_ns();
+            LSTM_CUDA(timed(K_FWD_REC, stream, [&] { return launch_tc_rec(tr, stream); }));
+            layer_in = hseq_tc;
+            continue;
+        }
+
         PackHhFwdArgs ph{};
         ph.H = H; ph.D = D; ph.nu = l.fwd.nu; ph.U = l.fwd.U; ph.dt = l.dt;
         for (int d = 0; d < D; ++d) ph.w[d] = w_hh[k * D + d];
@@ -426,7 +488,7 @@ lstm_status lstm_forward(const lstm_desc* desc, const void* x, const void* h0, c
             f.act = reinterpret_cast<float*>(P(reserve, l.act[k]));
             f.cst = reinterpret_cast<float*>(P(reserve, l.cst[k]));
         }
-        f.ctr = reinterpret_cast<unsigned*>(P(workspace, l.ctr_f)) + (size_t)k * D * l.fwd.nbg;
+        f.ctr = reinterpret_cast<unsigned*>(P(workspace, l.ctr_f)) + (size_t)k * D * l.nbg_ctr;
         f.status = status;
         f.timeout_ns = timeout_ns();
         LSTM_CUDA(timed(K_FWD_REC, stream, [&] { return launch_fwd_rec(f, stream); }));

@@ -128,6 +128,32 @@ struct FwdRecArgs {
 cudaError_t launch_fwd_rec(const FwdRecArgs& a, cudaStream_t s);
 RecPlan plan_fwd_rec(int H, int B, int D, DType dt, int num_sms, size_t smem_max);
 
+// Tensor-core forward recurrence (bf16, inference).  W_hh packed rows
+// [D*4H][H] bf16 (order 4u+q); hx exchange [D][T+1][B][H] bf16 with slot 0 =
+// h0 (or zeros) filled before the launch.
+struct TcRecPlan {
+    bool ok;
+    int nbg, Bg, N, nu, kc_smem, stages, ctas;
+    size_t smem;
+};
+TcRecPlan plan_tc_rec(int H, int B, int D, int num_sms, size_t smem_max);
+
+struct TcRecArgs {
+    int H, B, T, D;
+    TcRecPlan p;
+    const float* gx;
+    const void* wpk;
+    const float* c0;
+    void* hx;
+    void* hseq;
+    void* out; long long out_st, out_sb;
+    void* h_n; float* c_n;
+    unsigned* ctr;
+    int* status;
+    uint64_t timeout_ns;
+};
+cudaError_t launch_tc_rec(const TcRecArgs& a, cudaStream_t s);
+
 struct BwdRecArgs {
     int H, B, T, D;
     RecPlan p;

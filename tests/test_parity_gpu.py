@@ -80,6 +80,14 @@ SMALL = {
                                state_std=0.3, seed=105),
     "bf16_uni": Workload("s", L=1, D=1, I=50, H=130, T=8, B=70, dtype="bf16", seed=106),
     "B1_T1": Workload("s", L=2, D=2, I=5, H=12, T=1, B=1, dtype="f32", state_std=0.5, seed=107),
+    # tensor-core recurrence: W_hh slice fully in tensor memory (H=128), split
+    # between shared and tensor memory (H=576), ragged batch groups
+    "bf16_tc_h128_bi": Workload("s", L=2, D=2, I=64, H=128, T=9, B=40, dtype="bf16",
+                                state_std=0.3, seed=111),
+    "bf16_tc_h576": Workload("s", L=1, D=1, I=128, H=576, T=5, B=20, dtype="bf16",
+                             state_std=0.3, seed=112),
+    "bf16_tc_seqfirst": Workload("s", L=1, D=2, I=64, H=256, T=6, B=130, dtype="bf16",
+                                 batch_first=False, seed=113),
     "H1": Workload("s", L=1, D=1, I=3, H=1, T=4, B=3, dtype="f32", state_std=0.5, seed=108),
 }
 
@@ -191,3 +199,18 @@ def test_workload_training_full_size(cuda_lib):
         for i, (g, o) in enumerate(zip(gpu2[k], ref2[k])):
             e = _relerr(g, o)
             assert e <= RTOL_GRAD, f"{k}[{i}]: max-rel {e:.3e}"
+
+
+@pytest.mark.parametrize("env", ["LSTM_B200_REC=simt", "LSTM_B200_GEMM=simt"])
+def test_cuda_core_engines(env, cuda_lib):
+    """Re-runs shapes that normally take the tensor-core kernels with the
+    CUDA-core kernels forced (engine choice is read once per process)."""
+    import os
+    import subprocess
+    import sys
+    k, v = env.split("=")
+    e = dict(os.environ)
+    e[k] = v
+    script = os.path.join(os.path.dirname(__file__), "engine_check.py")
+    r = subprocess.run([sys.executable, script], env=e, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout + r.stderr
