@@ -75,8 +75,7 @@ __global__ void __launch_bounds__(256, 1)
     using Cf = Cfg<KIND>;
     constexpr int S = Cf::STAGES, BM = Cf::BM, BN = Cf::BN, BK = Cf::BK;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    unsigned char* smem = reinterpret_cast<unsigned char*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    unsigned char* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * Cf::STAGE_BYTES);
     uint64_t* lofull = full + S;
     uint64_t* empty = lofull + S;
@@ -186,37 +185,57 @@ __global__ void __launch_bounds__(256, 1)
             tc::mbar_arrive(&lofull[s]);
         }
     } else if (warp >= 4) {
+        // Epilogue: each warp drains its 32 accumulator rows in 32 x 32
+        // blocks staged through shared memory (the pipeline stages are idle
+        // once every MMA has completed), so each global store instruction
+        // writes one contiguous 128-byte row segment.
         const int q = warp & 3;
         const bool ok = tc::mbar_wait(tmem_full, 0, abort_flag, e.status, e.timeout_ns);
         tc::tc_fence_after();
-        const int m = m0 + q * 32 + lane;
+        float* stg = reinterpret_cast<float*>(smem) + q * (32 * 33);
+        // Output row of accumulator row (q*32 + lane), computed once per tile
+        // and broadcast inside the row loop.
+        const int mrow = m0 + q * 32 + lane;
+        const long long my_row = e.ws ? (long long)mrow : out_row(e, mrow);
+        const int rows_here = min(32, e.M - (m0 + q * 32));
         if (ok) {
-            for (int c = 0; c < BN; c += 16) {
-                float v[16];
+            for (int c = 0; c < BN; c += 32) {
+                float v[16], w[16];
                 tc::tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c, v);
+                tc::tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(c + 16), w);
                 tc::tmem_ld_wait();
-                if (m >= e.M) continue;
-                if (nk == 0) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) v[i] = 0.f;
+                for (int i = 0; i < 16; ++i) {
+                    stg[lane * 33 + i] = nk ? v[i] : 0.f;
+                    stg[lane * 33 + 16 + i] = nk ? w[i] : 0.f;
                 }
+                __syncwarp();
+                const int n = n0 + c + lane;
+                const bool ncol = n < e.N;
+                const float bn = (!e.ws && e.bias && ncol) ? e.bias[n] : 0.f;
+                float* base;
+                long long ld;
                 if (e.ws) {
-                    float* dst = e.ws + ((size_t)split * e.M + m) * e.N;
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        if (n0 + c + i < e.N) dst[n0 + c + i] = v[i];
+                    base = e.ws + (size_t)split * e.M * e.N + n;
+                    ld = e.N;
+                } else if (n < e.n_split) {
+                    base = e.C + n;
+                    ld = e.ldc;
                 } else {
-                    const long long row = out_row(e, m);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int n = n0 + c + i;
-                        if (n >= e.N) continue;
-                        float val = v[i] + (e.bias ? e.bias[n] : 0.f);
-                        float* dst = n < e.n_split ? e.C + row * e.ldc + n : e.C1 + row * e.ldc1 + (n - e.n_split);
+                    base = e.C1 + (n - e.n_split);
+                    ld = e.ldc1;
+                }
+#pragma unroll 8
+                for (int rr = 0; rr < 32; ++rr) {
+                    const long long row = __shfl_sync(0xffffffffu, my_row, rr);
+                    if (rr < rows_here && ncol) {
+                        float* dst = base + row * ld;
+                        float val = stg[rr * 33 + lane] + bn;
                         if (e.accumulate) val += *dst;
                         *dst = val;
                     }
                 }
+                __syncwarp();
             }
         }
     }

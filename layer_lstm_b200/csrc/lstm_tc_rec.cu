@@ -56,8 +56,30 @@ struct TcRecParams {
     uint64_t timeout_ns;
 };
 
+// Branch-free choice among four registers by a lane-dependent index k in
+// [0, 4): two levels of selp, so a warp never diverges on it.
+__device__ __forceinline__ float selp_f(float a, float b, uint32_t take_b) {
+    float r;
+    asm("{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %3, 0;\n\tselp.f32 %0, %2, %1, p;\n\t}"
+        : "=f"(r) : "f"(a), "f"(b), "r"(take_b));
+    return r;
+}
+
 __device__ __forceinline__ float sel4(float a0, float a1, float a2, float a3, int k) {
-    return k == 0 ? a0 : (k == 1 ? a1 : (k == 2 ? a2 : a3));
+    const float lo = selp_f(a0, a1, (uint32_t)k & 1u);
+    const float hi = selp_f(a2, a3, (uint32_t)k & 1u);
+    return selp_f(lo, hi, (uint32_t)k & 2u);
+}
+
+// Gate nonlinearities of this bf16-only kernel: CUDA's fast intrinsics and the
+// hardware tanh approximation (relative error near 2^-11, far inside the bf16
+// path's 2e-2 tolerance).
+__device__ __forceinline__ float sigmoid_fast(float z) { return __fdividef(1.f, 1.f + __expf(-z)); }
+
+__device__ __forceinline__ float tanh_fast(float z) {
+    float r;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(r) : "f"(z));
+    return r;
 }
 
 __device__ __forceinline__ bool named_bar_or(int id, int n, bool pred) {
@@ -132,8 +154,7 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 __global__ void __launch_bounds__(kThreads, 1)
     tc_rec_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmW, TcRecParams a) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    unsigned char* smem = reinterpret_cast<unsigned char*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    unsigned char* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
     const int H = a.H, B = a.B, T = a.T, D = a.D, G = 4 * H;
     const int KT = H / 64, S = a.stages, N = a.N;
     const int hstage = N * 128;
@@ -320,10 +341,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int col = cbase + 16 * cc + 4 * gq + i;
                     if (col >= nB) continue;
                     const int b = b0 + col;
-                    const float ig = sigmoidf_(pi), fg = sigmoidf_(pf), gg = tanhf(pgg), og = sigmoidf_(po);
+                    const float ig = sigmoid_fast(pi), fg = sigmoid_fast(pf), gg = tanh_fast(pgg);
+                    const float og = sigmoid_fast(po);
                     const float c = fg * creg[cc][i] + ig * gg;
                     creg[cc][i] = c;
-                    const bf16 hv = __float2bfloat16_rn(og * tanhf(c));
+                    const bf16 hv = __float2bfloat16_rn(og * tanh_fast(c));
                     hxo[(size_t)b * H + u] = hv;
                     if (a.hseq) a.hseq[((size_t)t * B + b) * ldseq + (size_t)d * H + u] = hv;
                     if (a.out) a.out[(size_t)t * a.out_st + (size_t)b * a.out_sb + (size_t)d * H + u] = hv;
