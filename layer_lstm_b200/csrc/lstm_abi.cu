@@ -202,7 +202,7 @@ bool make_layout(const lstm_desc* d, Layout& l) {
     const size_t Hp = (size_t)((l.H + 3) & ~3);
     l.whh_b = o; o += al(l.bwd_ok ? (size_t)l.D * l.bwd.nu * 4 * l.bwd.U * Hp * 4 : 0);
     l.gx = o; o += al(TB * l.D * l.G * 4);
-    l.hT = o; o += al(TB * l.D * l.H * l.es);
+    l.hT = o; o += al((size_t)l.T * l.D * l.fwd.nbg * l.fwd.Bg * l.H * l.es);   // [D][T][nbg][H][Bg]
     l.seq[0] = o; o += al(TB * l.D * l.H * l.es);
     l.seq[1] = o; o += al(TB * l.D * l.H * l.es);
     if (l.tcr.ok) {

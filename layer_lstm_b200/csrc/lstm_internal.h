@@ -116,7 +116,7 @@ struct FwdRecArgs {
     const void* wpk;            // PackHhFwd layout
     const void* h0;             // [D][B][H] or null
     const float* c0;            // [D][B][H] or null
-    void* hT;                   // [D][T][H][B] exchange copy of h (k-major)
+    void* hT;                   // [D][T][nbg][H][Bg] exchange copy of h (group-major, k-major)
     void* hseq;                 // [T][B][D*H] layer output, time-major
     void* out; long long out_st, out_sb;   // user out (top layer) or null; element strides
     void* h_n; float* c_n;      // [D][B][H]

@@ -13,8 +13,10 @@
 // in shared memory for the whole sequence.  Blocks of one (d, bg) group meet
 // once per step on a counter (bounded wait, see lstm_device.cuh).
 //
-//  forward  step: gather h_{t-1} of the group's rows (k-major exchange buffer
-//                 hT[t][k][b]), a = W_slice h + Gx[t], gates, c/h update,
+//  forward  step: gather h_{t-1} of the group's rows from the exchange
+//                 buffer hT[d][t][bg][k][bl] (group-major and k-major, so the
+//                 group's tile is one contiguous block fetched with a single
+//                 bulk async copy), a = W_slice h + Gx[t], gates, c/h update,
 //                 write h_t (exchange, layer output, user output).
 //  backward step: dh = dy_t + dh_rec for the block's units, gate derivatives
 //                 and the dc carry -> da_t (the block's 4U gate rows); the
@@ -27,6 +29,7 @@
 
 #include "lstm_device.cuh"
 #include "lstm_internal.h"
+#include "lstm_tc.cuh"
 
 namespace lstm {
 namespace {
@@ -141,16 +144,18 @@ __device__ __forceinline__ void copy_tile(T* __restrict__ dst, int nrows, int nc
     }
 }
 
+constexpr int kRecThreads = 256;   // threads per recurrent block
+
 inline int pick_ks(int R, int N, int K) {
     const int nT = (R / 4) * (N / 4);
     int ks = 1;
-    while (nT * ks * 2 <= 256 && K / (ks * 2) >= 16) ks *= 2;
+    while (nT * ks * 2 <= kRecThreads && K / (ks * 2) >= 16) ks *= 2;
     return ks;
 }
 
 // ============================================================== forward
 template <typename WT>
-__global__ void __launch_bounds__(256, 1) fwd_rec_kernel(FwdRecArgs a) {
+__global__ void __launch_bounds__(kRecThreads, 1) fwd_rec_kernel(FwdRecArgs a) {
     extern __shared__ __align__(16) unsigned char smem[];
     const RecPlan& p = a.p;
     const int H = a.H, B = a.B, T = a.T, D = a.D, G = 4 * H;
@@ -163,6 +168,8 @@ __global__ void __launch_bounds__(256, 1) fwd_rec_kernel(FwdRecArgs a) {
     float* red = reinterpret_cast<float*>(smem + off);                 // [KS][R][Bs]
     off += align16((size_t)KS * R * Bs * sizeof(float));
     float* cs = reinterpret_cast<float*>(smem + off);                  // [U][Bg]
+    off += align16((size_t)U * p.Bg * sizeof(float));
+    uint64_t* hbar = reinterpret_cast<uint64_t*>(smem + ((off + 7) & ~size_t(7)));
 
     const int j = blockIdx.x % p.nu;
     const int bg = (blockIdx.x / p.nu) % p.nbg;
@@ -189,11 +196,22 @@ __global__ void __launch_bounds__(256, 1) fwd_rec_kernel(FwdRecArgs a) {
         if (a.c0 && ul < nU && bl < nB) c = a.c0[((size_t)d * B + b0 + bl) * H + u0 + ul];
         cs[i] = c;
     }
+    if (tid == 0) {
+        tc::mbar_init(hbar, 1);
+        tc::fence_mbar_init();
+    }
     __syncthreads();
     if (nB <= 0) return;   // plans never leave a group empty
 
     unsigned* ctr = a.ctr + d * p.nbg + bg;
     const size_t ldseq = (size_t)D * H;
+    const size_t tile = (size_t)H * p.Bg;                       // exchange elements per (t, group)
+    WT* hT_grp = hT + (size_t)bg * tile;                        // + (d*T + t) * nbg * tile
+    const size_t hT_tstride = (size_t)p.nbg * tile;
+    // one bulk copy per step when the group's tile is the whole shared tile
+    const bool bulk = Bs == p.Bg && Hp == H && ((tile * sizeof(WT)) & 15) == 0 &&
+                      ((reinterpret_cast<uintptr_t>(hT) & 15) == 0);
+    uint32_t hphase = 0;
     const int np0 = nU * min(Bs, nB);
     auto store_red = [&](int ks, int r0, int n0, float (&acc)[4][4]) {
         float* rp = red + ((size_t)ks * R + r0) * Bs + n0;
@@ -231,8 +249,20 @@ __global__ void __launch_bounds__(256, 1) fwd_rec_kernel(FwdRecArgs a) {
                     if (h0 && k < H && bl < nb) v = h0[((size_t)d * B + b0 + bs0 + bl) * H + k];
                     hs[i] = v;
                 }
+            } else if (bulk) {
+                if (tid == 0) {
+                    // order the previous step's generic reads of hs and the
+                    // other blocks' generic writes of hT before the async copy
+                    tc::fence_proxy_async_smem();
+                    tc::fence_proxy_async_global();
+                    tc::mbar_arrive_expect_tx(hbar, (uint32_t)(tile * sizeof(WT)));
+                    tc::bulk_load(hs, hT_grp + ((size_t)d * T + tp) * hT_tstride, (uint32_t)(tile * sizeof(WT)), hbar);
+                }
+                volatile int never = 0;
+                if (!tc::mbar_wait(hbar, hphase, &never, a.status, a.timeout_ns)) return;
+                hphase ^= 1;
             } else {
-                copy_tile(hs, Hp, Bs, hT + (((size_t)d * T + tp) * H) * B + b0 + bs0, (size_t)B, H, nb);
+                copy_tile(hs, Hp, Bs, hT_grp + ((size_t)d * T + tp) * hT_tstride + bs0, (size_t)p.Bg, H, nb);
             }
             __syncthreads();
             block_mm(Ws, R, hs, Bs, R, Bs, Hp, KS, store_red);
@@ -263,7 +293,7 @@ __global__ void __launch_bounds__(256, 1) fwd_rec_kernel(FwdRecArgs a) {
                 cref = c;
                 const float h = og * tanhf(c);
                 const WT hv = from_f<WT>(h);
-                hT[(((size_t)d * T + t) * H + u) * B + b] = hv;
+                hT_grp[((size_t)d * T + t) * hT_tstride + (size_t)u * p.Bg + bs0 + bl] = hv;
                 if (hseq) hseq[((size_t)t * B + b) * ldseq + (size_t)d * H + u] = hv;
                 if (out) out[(size_t)t * a.out_st + (size_t)b * a.out_sb + (size_t)d * H + u] = hv;
                 if (a.act) {
@@ -278,7 +308,10 @@ __global__ void __launch_bounds__(256, 1) fwd_rec_kernel(FwdRecArgs a) {
             }
             __syncthreads();
         }
-        if (p.nu > 1 && s + 1 < T) block_arrive(ctr);
+        if (p.nu > 1 && s + 1 < T) {
+            if (bulk) tc::fence_proxy_async_global();   // h_t is read by bulk copies
+            block_arrive(ctr);
+        }
     }
 }
 
@@ -301,7 +334,7 @@ __device__ __forceinline__ BwdPre bwd_fetch(const BwdRecArgs& a, int d, int t, i
     return r;
 }
 
-__global__ void __launch_bounds__(256, 1) bwd_rec_kernel(BwdRecArgs a) {
+__global__ void __launch_bounds__(kRecThreads, 1) bwd_rec_kernel(BwdRecArgs a) {
     extern __shared__ __align__(16) unsigned char smem[];
     const RecPlan& p = a.p;
     const int H = a.H, B = a.B, T = a.T, D = a.D, G = 4 * H;
@@ -515,9 +548,9 @@ RecPlan plan_fwd_rec(int H, int B, int D, DType dt, int num_sms, size_t smem_max
                 const int R = 4 * U;
                 const int KS = pick_ks(R, Bs, Hp);
                 const size_t smem = align16h((size_t)Hp * R * es) + align16h((size_t)Hp * Bs * es) +
-                                    align16h((size_t)KS * R * Bs * 4) + align16h((size_t)U * Bg * 4);
+                                    align16h((size_t)KS * R * Bs * 4) + align16h((size_t)U * Bg * 4) + 16;
                 if (smem <= smem_max) {
-                    pl = RecPlan{nbg, Bg, nu, U, Bs, KS, 256, smem, ctas};
+                    pl = RecPlan{nbg, Bg, nu, U, Bs, KS, kRecThreads, smem, ctas};
                     ok = true;
                     break;
                 }
@@ -557,12 +590,12 @@ RecPlan plan_bwd_rec(int H, int B, int D, int num_sms, size_t smem_max) {
             RecPlan pl{};
             bool ok = false;
             for (; Bs >= 4; Bs -= 4) {
-                const int CG = std::max(1, 256 / ((U / 4) * std::min(Bg, 256)));
+                const int CG = std::max(1, kRecThreads / ((U / 4) * std::min(Bg, kRecThreads)));
                 const size_t smem = align16h((size_t)4 * U * Hp * 4) + align16h((size_t)4 * U * Bs * 4) +
                                     2 * align16h((size_t)U * Bg * 4) + align16h((size_t)4 * U * Bg * 4) +
                                     align16h((size_t)CG * U * Bg * 4);
                 if (smem <= smem_max) {
-                    pl = RecPlan{nbg, Bg, nu, U, Bs, 1, 256, smem, ctas};
+                    pl = RecPlan{nbg, Bg, nu, U, Bs, 1, kRecThreads, smem, ctas};
                     ok = true;
                     break;
                 }
