@@ -140,10 +140,10 @@ struct Layout {
     size_t es;
     RecPlan fwd, bwd;
     TcRecPlan tcr;
-    int nbg_ctr;       // counter stride per (layer, direction): max over the forward plans
+    int nbg_ctr;       // counter stride per (layer, direction) of the FFMA forward recurrence
     bool bwd_ok;
     // workspace offsets
-    size_t status, ctr_f, ctr_b, wih[32], bias[32], whh_f, whh_b, gx, hT, seq[2], dG, dseq[2], xt,
+    size_t status, ctr_f, ctr_b, ctr_tc, ctr_end, wih[32], bias[32], whh_f, whh_b, gx, hT, seq[2], dG, dseq[2], xt,
         dbpart, P, dGT, bop, wcatT, hx, whh_tc, bias_dummy, total;
     // reserve offsets
     size_t act[32], cst[32], hseq[32], rtotal;   // per layer: [D][T][B][G], [D][T][B][H], [T][B][D*H]
@@ -191,9 +191,13 @@ bool make_layout(const lstm_desc* d, Layout& l) {
     const size_t TB = (size_t)l.T * l.B;
     size_t o = 0;
     l.status = o; o += al(sizeof(int));
-    l.nbg_ctr = std::max(l.fwd.nbg, l.tcr.ok ? l.tcr.nbg : 0);
+    l.nbg_ctr = l.fwd.nbg;
     l.ctr_f = o; o += al(sizeof(unsigned) * (size_t)l.L * l.D * l.nbg_ctr);
     l.ctr_b = o; o += al(sizeof(unsigned) * (size_t)l.L * l.D * (l.bwd_ok ? l.bwd.nbg : 1));
+    // tensor-core recurrence: one counter per (layer, direction, group), each
+    // on its own 128-byte line
+    l.ctr_tc = o; o += al(l.tcr.ok ? sizeof(unsigned) * 32 * (size_t)l.L * l.D * l.tcr.nbg : 0);
+    l.ctr_end = o;
     for (int k = 0; k < l.L; ++k) {
         l.wih[k] = o; o += al((size_t)l.D * l.G * in_size(l, k) * l.es);
         l.bias[k] = o; o += al((size_t)l.D * l.G * 4);
@@ -372,9 +376,7 @@ lstm_status lstm_forward(const lstm_desc* desc, const void* x, const void* h0, c
     const int L = l.L, D = l.D, H = l.H, B = l.B, T = l.T, G = l.G;
     const size_t es = l.es;
     const size_t state_elems = (size_t)D * B * H;   // elements per layer slice
-    LSTM_CUDA(cudaMemsetAsync(workspace, 0, l.ctr_b + al(sizeof(unsigned) * (size_t)L * D *
-                                                          (l.bwd_ok ? l.bwd.nbg : 1)),
-                              stream));
+    LSTM_CUDA(cudaMemsetAsync(workspace, 0, l.ctr_end, stream));   // status word and all counters
     if (B == 0) return LSTM_OK;
     if (T == 0) {
         // no step runs: h_n = h0, c_n = c0 (zeros when absent)
@@ -454,7 +456,7 @@ lstm_status lstm_forward(const lstm_desc* desc, const void* x, const void* h0, c
             }
             tr.h_n = static_cast<char*>(h_n) + (size_t)k * state_elems * es;
             tr.c_n = c_n + (size_t)k * state_elems;
-            tr.ctr = reinterpret_cast<unsigned*>(P(workspace, l.ctr_f)) + (size_t)k * D * l.nbg_ctr;
+            tr.ctr = reinterpret_cast<unsigned*>(P(workspace, l.ctr_tc)) + (size_t)k * D * l.tcr.nbg * 32;
             tr.status = status;
             tr.timeout_ns = timeout_ns();
             LSTM_CUDA(timed(K_FWD_REC, stream, [&] { return launch_tc_rec(tr, stream); }));
@@ -528,8 +530,7 @@ lstm_status lstm_backward(const lstm_desc* desc, const void* x, const void* h0, 
 
     const int L = l.L, D = l.D, H = l.H, B = l.B, T = l.T, G = l.G;
     const size_t state = (size_t)D * B * H;
-    LSTM_CUDA(cudaMemsetAsync(workspace, 0, l.ctr_b + al(sizeof(unsigned) * (size_t)L * D * l.bwd.nbg),
-                              stream));
+    LSTM_CUDA(cudaMemsetAsync(workspace, 0, l.ctr_end, stream));   // status word and all counters
     // weight gradients start from zero (T == 0 or B == 0 leave them zero)
     for (int k = 0; k < L; ++k) {
         for (int d = 0; d < D; ++d) {

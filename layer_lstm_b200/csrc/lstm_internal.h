@@ -133,7 +133,7 @@ RecPlan plan_fwd_rec(int H, int B, int D, DType dt, int num_sms, size_t smem_max
 // h0 (or zeros) filled before the launch.
 struct TcRecPlan {
     bool ok;
-    int nbg, Bg, N, nu, kc_smem, stages, ctas;
+    int nbg, Bg, N, nu, KH, kc_smem, stages, ctas;   // ctas = 2 per (d, bg, unit slice)
     size_t smem;
 };
 TcRecPlan plan_tc_rec(int H, int B, int D, int num_sms, size_t smem_max);
@@ -148,7 +148,7 @@ struct TcRecArgs {
     void* hseq;
     void* out; long long out_st, out_sb;
     void* h_n; float* c_n;
-    unsigned* ctr;
+    unsigned* ctr;              // [D][nbg] group counters, 32 words apart, zeroed
     int* status;
     uint64_t timeout_ns;
 };

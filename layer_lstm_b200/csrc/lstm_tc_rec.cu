@@ -6,24 +6,30 @@
 // W_ih x_t + b_ih + b_hh from the time-batched projection) and the cell
 // update c = f c + i g, h = o tanh(c).
 //
-// Block (d, bg, j) owns 128 packed gate rows p = 4u + q of units
-// [32j, 32j+32) and the batch rows of group bg, and keeps its whole W_hh
-// slice resident for the sequence: K chunks [0, kc_smem) in shared memory
-// (128-byte-swizzled K-major tiles loaded once by TMA) and the remaining
-// chunks in tensor memory, where tcgen05.mma reads them as the A operand.
-// The accumulator (128 lanes x N batch columns, fp32) also lives in tensor
-// memory.  One step:
-//   warp 0:         wait for the group's h_{t-1}, TMA it (N rows x 64 k per
-//                   chunk) through a ring of shared-memory stages
-//   warp 1:         once the accumulator holds Gx[t] (d_ready), one thread
-//                   issues M=128 x N x K=16 MMAs over all of K
-//   epilogue warps: (two per tensor-memory lane quarter, each half of the
-//                   batch columns) tcgen05.ld the pre-activations, exchange
-//                   the four gates of each unit inside 4-lane groups
-//                   (shuffles), update c (registers) and h, write h_t and
-//                   arrive on the counter; then load Gx[t+1] and store it
-//                   into the accumulator (tcgen05.st) and signal d_ready.
-// Only bf16 inference uses this kernel; every wait is bounded.
+// A cluster of two blocks owns 128 packed gate rows p = 4u + q (units
+// [32j, 32j+32)) and the N batch columns of group bg.  The pair splits K:
+// block rank r keeps the K chunks [r*KH, r*KH + KH) of the 128-row W_hh slice
+// resident for the whole sequence (tensor memory, where tcgen05.mma reads it
+// as the A operand; chunks beyond its capacity in shared memory) and issues
+// the MMAs of its half only, so the serial chain of MMA instructions per step
+// is half as long as with one block per slice.  Each block owns half of the N
+// columns: it sends its partial sums of the partner's columns into the
+// partner's shared memory (distributed shared memory stores, then a remote
+// mbarrier arrive), adds the partner's partial sums of its own columns, and
+// updates c and h there.  One step:
+//   warp 0:     wait for the group's h_{t-1}, TMA this block's K chunks of it
+//               (N rows x 64 k each) through a ring of shared-memory stages
+//   warp 1:     once the accumulator holds Gx[t] in the own columns and zero
+//               in the partner's (d_ready), one thread issues M=128 x N x
+//               K=16 MMAs over the block's K chunks
+//   warps 2-9:  (two per tensor-memory lane quarter) exchange partial sums
+//               with the partner, exchange the four gates of each unit inside
+//               4-lane groups (shuffles), update c (registers) and h, write
+//               h_t and arrive on the group counter; then load Gx[t+1] (L2
+//               prefetched one step ahead) into the accumulator and signal
+//               d_ready.
+// Only bf16 inference uses this kernel.  Every wait is bounded: on a timeout
+// the kernel records LSTM_ERR_TIMEOUT in the status word and returns.
 #include <algorithm>
 
 #include "lstm_device.cuh"
@@ -35,23 +41,29 @@ namespace {
 
 constexpr int kRows = 128;             // gate rows per block
 constexpr int kChunkW = kRows * 128;   // bytes of one 64-wide K chunk of W
-constexpr int kMaxNcc = 8;             // N <= 128 batch columns per block
-constexpr int kNccHalf = kMaxNcc / 2;  // 16-column chunks per epilogue half
+constexpr int kMaxN = 256;             // batch columns per cluster
+constexpr int kCcPerHalf = 4;          // own 16-column chunks per epilogue thread (N/2 <= 128)
 constexpr int kEpi = 256;              // epilogue threads: warps 2-9, two per lane quarter
 constexpr int kThreads = 64 + kEpi;    // warp 0 TMA, warp 1 MMA
 constexpr uint32_t kAcol = 256;        // tensor-memory column of the resident W part
+constexpr int kMaxTmemChunks = 8;      // 8 x 32 columns of W in tensor memory
+// Shared memory requested per block is at least this, so that two blocks
+// never share an SM (each allocates all 512 tensor-memory columns).
+constexpr size_t kMinSmem = 120 * 1024;
+constexpr int kCtrStride = 32;         // unsigned words between group counters (one 128-byte line each)
 
 struct TcRecParams {
     int H, B, T, D;
-    int nbg, Bg, N, nu, kc_smem, stages;
+    int nbg, Bg, N, nu, KH, kc_smem, stages;
     const float* gx;          // [T][B][D*G] packed rows, biases included
     const float* c0;          // [D][B][H] or null
     bf16* hx;                 // [D][T+1][B][H]; slot 0 holds h0
     bf16* hseq;               // [T][B][D*H] or null
     bf16* out; long long out_st, out_sb;
+    int out_vec;              // out is 16-byte aligned: h leaves in 16-byte stores
     bf16* h_n; float* c_n;    // [D][B][H]
     const bf16* wpk;          // [D*G][H] packed rows
-    unsigned* ctr;            // [D*nbg]
+    unsigned* ctr;            // [D][nbg] group counters, kCtrStride apart
     int* status;
     uint64_t timeout_ns;
 };
@@ -71,16 +83,18 @@ __device__ __forceinline__ float sel4(float a0, float a1, float a2, float a3, in
     return selp_f(lo, hi, (uint32_t)k & 2u);
 }
 
-// Gate nonlinearities of this bf16-only kernel: CUDA's fast intrinsics and the
-// hardware tanh approximation (relative error near 2^-11, far inside the bf16
-// path's 2e-2 tolerance).
-__device__ __forceinline__ float sigmoid_fast(float z) { return __fdividef(1.f, 1.f + __expf(-z)); }
-
+// Gate nonlinearities of this bf16-only kernel: the hardware tanh
+// approximation (relative error near 2^-11, far inside the bf16 path's 2e-2
+// tolerance).
 __device__ __forceinline__ float tanh_fast(float z) {
     float r;
     asm("tanh.approx.f32 %0, %1;" : "=f"(r) : "f"(z));
     return r;
 }
+
+// sigma(z) = (1 + tanh(z/2)) / 2: one special-function op instead of an
+// exponential and a reciprocal
+__device__ __forceinline__ float sigmoid_fast(float z) { return fmaf(0.5f, tanh_fast(0.5f * z), 0.5f); }
 
 __device__ __forceinline__ bool named_bar_or(int id, int n, bool pred) {
     uint32_t r;
@@ -93,6 +107,69 @@ __device__ __forceinline__ bool named_bar_or(int id, int n, bool pred) {
         : "r"((uint32_t)pred), "r"(id), "r"(n)
         : "memory");
     return r != 0;
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Shared-memory address of the same offset in block `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_rank(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+
+// Arrive on an mbarrier of another block of the cluster, releasing this
+// thread's earlier distributed-shared-memory stores at cluster scope.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t remote_bar) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(tc::smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for the partner's partial sums: gives up on this block's abort
+// flag, on an error anywhere in the grid, or after timeout_ns.
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort, int* status,
+                                                  uint64_t timeout_ns) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    uint32_t it = 0;
+    while (!mbar_try_wait_cluster(bar, parity)) {
+        if ((++it & 255u) == 0) {
+            if (*abort || ld_volatile(status) != kStatusOk) {
+                *abort = 1;
+                return false;
+            }
+            if (globaltimer_ns() - t0 > timeout_ns) {
+                atomicCAS(status, kStatusOk, kStatusTimeout);
+                *abort = 1;
+                return false;
+            }
+        }
+    }
+    return true;
 }
 
 // Bounded wait until *ctr >= target (single thread).
@@ -117,33 +194,6 @@ __device__ __forceinline__ bool ctr_wait(const unsigned* ctr, unsigned target, v
     return true;
 }
 
-// Gx[t] of accumulator row `prow - prow0` (packed row prow) for columns
-// [cbase, cbase + NH) of this thread's half, written into the accumulator
-// (zeros outside the batch), then d_ready.  Two groups of 32 columns: each
-// group's loads are all in flight before its tensor-memory stores.
-__device__ __forceinline__ void preload_gx(const float* gx, int t, int B, size_t ldgx, int prow, int b0,
-                                           int cbase, int NH, int nB, uint32_t trow, uint64_t* d_ready) {
-    const float* gxp = gx + (size_t)t * B * ldgx + (size_t)prow;
-#pragma unroll
-    for (int g = 0; g < kNccHalf / 2; ++g) {
-        if (32 * g >= NH) break;
-        uint32_t v[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int col = cbase + 32 * g + i;
-            v[i] = (32 * g + i < NH && col < nB) ? __float_as_uint(__ldg(gxp + (size_t)(b0 + col) * ldgx)) : 0u;
-        }
-        uint32_t lo[16], hi[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) { lo[i] = v[i]; hi[i] = v[16 + i]; }
-        tc::tmem_st16(trow + (uint32_t)(cbase + 32 * g), lo);
-        if (32 * g + 16 < NH) tc::tmem_st16(trow + (uint32_t)(cbase + 32 * g + 16), hi);
-    }
-    tc::tmem_st_wait();
-    tc::tc_fence_before();
-    tc::mbar_arrive(d_ready);
-}
-
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     const uint64_t t0 = globaltimer_ns();
     while (!tc::mbar_try_wait(bar, parity)) {
@@ -151,30 +201,90 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     }
 }
 
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
+                 : "memory");
+}
+
+// Accumulator initialisation for one step: Gx[t] of packed row `prow` in the
+// own columns (chunks cc = half, half + 2, ... of [own0, own0 + NH); zero past
+// the batch), zero in the partner's columns; then d_ready.  Two own chunks'
+// loads are in flight before their tensor-memory stores.
+__device__ __forceinline__ void preload_gx(const float* gx, int t, int B, size_t ldgx, int prow, int b0, int own0,
+                                           int pcol0, int ncc, int nB, int half, uint32_t trow, uint64_t* d_ready) {
+    const float* gxp = gx + (size_t)t * B * ldgx + (size_t)prow;
+    uint32_t zero[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) zero[i] = 0u;
+#pragma unroll
+    for (int k = 0; k < kCcPerHalf; k += 2) {
+        const int cc0 = half + 2 * k, cc1 = cc0 + 2;
+        if (cc0 >= ncc) break;
+        uint32_t v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int cc = i < 16 ? cc0 : cc1;
+            const int col = own0 + 16 * cc + (i & 15);
+            v[i] = (cc < ncc && col < nB) ? __float_as_uint(__ldg(gxp + (size_t)(b0 + col) * ldgx)) : 0u;
+        }
+        uint32_t lo[16], hi[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) { lo[i] = v[i]; hi[i] = v[16 + i]; }
+        tc::tmem_st16(trow + (uint32_t)(own0 + 16 * cc0), lo);
+        tc::tmem_st16(trow + (uint32_t)(pcol0 + 16 * cc0), zero);
+        if (cc1 < ncc) {
+            tc::tmem_st16(trow + (uint32_t)(own0 + 16 * cc1), hi);
+            tc::tmem_st16(trow + (uint32_t)(pcol0 + 16 * cc1), zero);
+        }
+    }
+    tc::tmem_st_wait();
+    tc::tc_fence_before();
+    tc::mbar_arrive(d_ready);
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     tc_rec_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmW, TcRecParams a) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
     const int H = a.H, B = a.B, T = a.T, D = a.D, G = 4 * H;
-    const int KT = H / 64, S = a.stages, N = a.N;
+    const int S = a.stages, N = a.N, NH = N / 2;
     const int hstage = N * 128;
+    const uint32_t rank = cluster_rank();
+    const int KT = H / 64;
+    const int c_beg = (int)rank * a.KH, c_end = min(KT, c_beg + a.KH);
+    const int nch = c_end - c_beg;                     // K chunks of this block (>= 1)
+    const int kc_smem = min(nch, a.kc_smem);           // of which in shared memory
     unsigned char* sW = smem;
     unsigned char* sH = smem + a.kc_smem * kChunkW;
-    uint64_t* full = reinterpret_cast<uint64_t*>(sH + S * hstage);
+    // partner's partial sums of the own columns, [NH/4][128 rows] float4 (a
+    // warp's store of one column quad is 512 contiguous bytes)
+    float4* recv = reinterpret_cast<float4*>(sH + S * hstage);
+    // h of the own columns, [NH][32 units] bf16, 16-byte unit octets swizzled
+    bf16* sh = reinterpret_cast<bf16*>(recv + (size_t)(NH / 4) * kRows);
+    uint64_t* full = reinterpret_cast<uint64_t*>(sh + (size_t)NH * 32);
     uint64_t* empty = full + S;
     uint64_t* d_ready = empty + S;
     uint64_t* mma_done = d_ready + 1;
     uint64_t* w_full = mma_done + 1;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(w_full + 1);
+    uint64_t* recv_full = w_full + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(recv_full + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int j = blockIdx.x % a.nu;
-    const int bg = (blockIdx.x / a.nu) % a.nbg;
-    const int d = blockIdx.x / (a.nu * a.nbg);
+    const int cl = blockIdx.x >> 1;                    // cluster index; rank == blockIdx.x & 1
+    const int j = cl % a.nu;
+    const int bg = (cl / a.nu) % a.nbg;
+    const int d = cl / (a.nu * a.nbg);
     const int b0 = bg * a.Bg, nB = min(a.Bg, B - b0);
     const int prow0 = d * G + j * kRows;
-    unsigned* ctr = a.ctr + d * a.nbg + bg;
+    const int own0 = (int)rank * NH;                   // first own column
+    const int pcol0 = (int)(rank ^ 1u) * NH;           // first column of the partner
+    // group counter of (d, bg): every block of the group adds 1 when its h_t
+    // columns are out, so h_t is complete at 2 nu (s + 1)
+    unsigned* ctr = a.ctr + (size_t)(d * a.nbg + bg) * kCtrStride;
+    // K chunks in rotated order, so the blocks of a group spread their reads
+    // of h over the chunks
+    const int rot = j % nch;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -184,6 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mbar_init(d_ready, kEpi);
         tc::mbar_init(mma_done, 1);
         tc::mbar_init(w_full, 1);
+        tc::mbar_init(recv_full, kEpi);               // one arrive per epilogue thread of the partner
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
@@ -194,24 +305,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
+    cluster_sync();                                    // the partner's barriers exist before any remote arrive
     const uint32_t tmem = *tmem_slot;
 
-    // Resident weights: shared-memory part by TMA, tensor-memory part by the
-    // epilogue warps (row r of the block on lane r; two bf16 per column).
+    // Resident weights of this block's K chunks: the first kc_smem in shared
+    // memory by TMA, the rest in tensor memory (row r of the slice on lane r,
+    // two bf16 per column) by the first four epilogue warps.
     if (warp == 0 && lane == 0) {
         tc::prefetch_tmap(&tmH);
         tc::prefetch_tmap(&tmW);
-        if (a.kc_smem > 0) {
-            tc::mbar_arrive_expect_tx(w_full, (uint32_t)(a.kc_smem * kChunkW));
-            for (int c = 0; c < a.kc_smem; ++c) tc::tma_load_2d(sW + c * kChunkW, &tmW, 64 * c, prow0, w_full);
+        if (kc_smem > 0) {
+            tc::mbar_arrive_expect_tx(w_full, (uint32_t)(kc_smem * kChunkW));
+            for (int c = 0; c < kc_smem; ++c) tc::tma_load_2d(sW + c * kChunkW, &tmW, 64 * (c_beg + c), prow0, w_full);
         }
     }
     const int q = warp & 3;                 // lane quarter of an epilogue warp
     const int r = q * 32 + lane;            // accumulator row of this epilogue thread
-    const int half = (warp - 2) >> 2;       // batch-column half of an epilogue warp
+    const int half = (warp - 2) >> 2;       // 0 or 1 for epilogue warps
+    const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
     if (warp >= 2 && half == 0) {
         const bf16* wrow = a.wpk + (size_t)(prow0 + r) * H;
-        for (int c = a.kc_smem; c < KT; ++c) {
+        for (int c = c_beg + kc_smem; c < c_end; ++c) {
             const uint4* src = reinterpret_cast<const uint4*>(wrow + 64 * c);
             uint32_t v0[16], v1[16];
 #pragma unroll
@@ -221,9 +335,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint4 y = src[4 + i];
                 v1[4 * i] = y.x; v1[4 * i + 1] = y.y; v1[4 * i + 2] = y.z; v1[4 * i + 3] = y.w;
             }
-            const uint32_t col = kAcol + (uint32_t)(c - a.kc_smem) * 32;
-            tc::tmem_st16(tmem + ((uint32_t)(q * 32) << 16) + col, v0);
-            tc::tmem_st16(tmem + ((uint32_t)(q * 32) << 16) + col + 16, v1);
+            const uint32_t col = kAcol + (uint32_t)(c - c_beg - kc_smem) * 32;
+            tc::tmem_st16(trow + col, v0);
+            tc::tmem_st16(trow + col + 16, v1);
         }
         tc::tmem_st_wait();
     }
@@ -238,19 +352,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             for (int s = 0; s < T && ok; ++s) {
                 if (s > 0) {
-                    if (!ctr_wait(ctr, (unsigned)(a.nu * s), abort_flag, a.status, a.timeout_ns)) break;
+                    if (!ctr_wait(ctr, (unsigned)(2 * a.nu * s), abort_flag, a.status, a.timeout_ns)) break;
                     tc::fence_proxy_async_global();
                 }
                 const int row0 = (d * (T + 1) + s) * B + b0;
-                for (int c = 0; c < KT; ++c) {
-                    const int idx = s * KT + c, st = idx % S, rnd = idx / S;
+                for (int i = 0; i < nch; ++i) {
+                    const int c = rot + i < nch ? rot + i : rot + i - nch;
+                    const int st = issued % S, rnd = issued / S;
                     if (!tc::mbar_wait(&empty[st], (rnd & 1) ^ 1, abort_flag, a.status, a.timeout_ns)) {
                         ok = false;
                         break;
                     }
                     tc::mbar_arrive_expect_tx(&full[st], (uint32_t)hstage);
-                    tc::tma_load_2d(sH + st * hstage, &tmH, 64 * c, row0, &full[st]);
-                    issued = idx + 1;
+                    tc::tma_load_2d(sH + st * hstage, &tmH, 64 * (c_beg + c), row0, &full[st]);
+                    ++issued;
                 }
             }
             if (*abort_flag) {
@@ -262,27 +377,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ MMA
         if (lane == 0) {
             const uint32_t idesc = tc::instr_desc(1, kRows, N);
-            bool ok = a.kc_smem == 0 || tc::mbar_wait(w_full, 0, abort_flag, a.status, a.timeout_ns);
+            bool ok = kc_smem == 0 || tc::mbar_wait(w_full, 0, abort_flag, a.status, a.timeout_ns);
             int last = -1;
             for (int s = 0; s < T && ok; ++s) {
                 if (!tc::mbar_wait(d_ready, s & 1, abort_flag, a.status, a.timeout_ns)) break;
                 tc::tc_fence_after();
-                for (int c = 0; c < KT; ++c) {
-                    const int idx = s * KT + c, st = idx % S, rnd = idx / S;
+                for (int i = 0; i < nch; ++i) {
+                    const int idx = s * nch + i, st = idx % S, rnd = idx / S;
                     if (!tc::mbar_wait(&full[st], rnd & 1, abort_flag, a.status, a.timeout_ns)) {
                         ok = false;
                         break;
                     }
                     tc::tc_fence_after();
+                    const int c = rot + i < nch ? rot + i : rot + i - nch;
                     const uint32_t b_base = tc::smem_u32(sH + st * hstage);
 #pragma unroll
                     for (int jj = 0; jj < 4; ++jj) {
                         const uint64_t bd = tc::smem_desc_sw128(b_base + 32 * jj);
-                        if (c < a.kc_smem) {
+                        if (c < kc_smem) {
                             const uint64_t ad = tc::smem_desc_sw128(tc::smem_u32(sW + c * kChunkW) + 32 * jj);
                             tc::mma_bf16(tmem, ad, bd, idesc, 1);
                         } else {
-                            const uint32_t at = tmem + kAcol + (uint32_t)(c - a.kc_smem) * 32 + 8 * jj;
+                            const uint32_t at = tmem + kAcol + (uint32_t)(c - kc_smem) * 32 + 8 * jj;
                             tc::mma_bf16_ts(tmem, at, bd, idesc, 1);
                         }
                     }
@@ -296,76 +412,153 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------------- epilogue
+        const int e = threadIdx.x - 64;             // epilogue thread index
         const int gq = lane & 3;                    // gate of this lane's row
         const int u = j * 32 + q * 8 + (lane >> 2); // unit of this lane's row group
-        const int NH = N / 2;                       // columns of this half (multiple of 16)
-        const int cbase = half * NH;                // first column of this half
-        float creg[kNccHalf][4];
-#pragma unroll
-        for (int cc = 0; cc < kNccHalf; ++cc)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int col = cbase + 16 * cc + 4 * gq + i;
-                creg[cc][i] = (16 * cc < NH && col < nB && a.c0) ? a.c0[((size_t)d * B + b0 + col) * H + u] : 0.f;
-            }
+        const int ncc = NH / 16;                    // own 16-column chunks
+        const uint32_t partner = rank ^ 1u;
+        const uint32_t recv_remote = map_rank(tc::smem_u32(recv), partner);
+        const uint32_t recv_bar_remote = map_rank(tc::smem_u32(recv_full), partner);
         const size_t ldgx = (size_t)D * G;
         const size_t ldseq = (size_t)D * H;
-        const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
-        preload_gx(a.gx, d == 0 ? 0 : T - 1, B, ldgx, prow0 + r, b0, cbase, NH, nB, trow, d_ready);
+        float creg[kCcPerHalf][4];
+#pragma unroll
+        for (int k = 0; k < kCcPerHalf; ++k)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int cc = half + 2 * k;
+                const int col = own0 + 16 * cc + 4 * gq + i;
+                creg[k][i] = (cc < ncc && col < nB && a.c0) ? a.c0[((size_t)d * B + b0 + col) * H + u] : 0.f;
+            }
+        preload_gx(a.gx, d == 0 ? 0 : T - 1, B, ldgx, prow0 + r, b0, own0, pcol0, ncc, nB, half, trow, d_ready);
         for (int s = 0; s < T; ++s) {
             const int t = d == 0 ? s : T - 1 - s;
+            // Gx[t_next] of the own columns into L2 while the MMAs run
+            if (s + 1 < T && e < NH && own0 + e < nB) {
+                const int tn = d == 0 ? s + 1 : T - 2 - s;
+                prefetch_l2(a.gx + ((size_t)tn * B + b0 + own0 + e) * ldgx + prow0, kRows * 4);
+            }
             const bool ok = tc::mbar_wait(mma_done, s & 1, abort_flag, a.status, a.timeout_ns);
             if (named_bar_or(1, kEpi, !ok)) break;   // every epilogue thread leaves together
             tc::tc_fence_after();
-            bf16* hxo = a.hx + ((size_t)(d * (T + 1) + s + 1) * B) * H;
+            // 1) this block's partial sums of the partner's columns -> partner,
+            //    two 16-column chunks at a time
 #pragma unroll
-            for (int cc = 0; cc < kNccHalf; ++cc) {
-                if (16 * cc >= NH) break;
-                float v[16];
-                tc::tmem_ld16(trow + (uint32_t)(cbase + 16 * cc), v);
+            for (int k0 = 0; k0 < kCcPerHalf; k0 += 2) {
+                if (half + 2 * k0 >= ncc) break;
+                float pv[2][16];
+#pragma unroll
+                for (int kk = 0; kk < 2; ++kk) {
+                    const int cc = half + 2 * (k0 + kk);
+                    if (cc < ncc) tc::tmem_ld16(trow + (uint32_t)(pcol0 + 16 * cc), pv[kk]);
+                }
                 tc::tmem_ld_wait();
-                // v[4k + i]: gate gq at column 16cc + 4k + i.  Three xor
-                // exchanges inside each 4-lane group give lane gq all four
-                // gates at column 16cc + 4gq + i (gate X arrives in round gq ^ X).
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    float rcv[4];
-                    rcv[0] = sel4(v[i], v[4 + i], v[8 + i], v[12 + i], gq);
+                for (int kk = 0; kk < 2; ++kk) {
+                    const int cc = half + 2 * (k0 + kk);
+                    if (cc >= ncc) break;
 #pragma unroll
-                    for (int rr = 1; rr < 4; ++rr)
-                        rcv[rr] = __shfl_xor_sync(0xffffffffu, sel4(v[i], v[4 + i], v[8 + i], v[12 + i], gq ^ rr), rr);
-                    const float pi = sel4(rcv[0], rcv[1], rcv[2], rcv[3], gq ^ 0);
-                    const float pf = sel4(rcv[0], rcv[1], rcv[2], rcv[3], gq ^ 1);
-                    const float pgg = sel4(rcv[0], rcv[1], rcv[2], rcv[3], gq ^ 2);
-                    const float po = sel4(rcv[0], rcv[1], rcv[2], rcv[3], gq ^ 3);
-                    const int col = cbase + 16 * cc + 4 * gq + i;
-                    if (col >= nB) continue;
-                    const int b = b0 + col;
-                    const float ig = sigmoid_fast(pi), fg = sigmoid_fast(pf), gg = tanh_fast(pgg);
-                    const float og = sigmoid_fast(po);
-                    const float c = fg * creg[cc][i] + ig * gg;
-                    creg[cc][i] = c;
-                    const bf16 hv = __float2bfloat16_rn(og * tanh_fast(c));
-                    hxo[(size_t)b * H + u] = hv;
-                    if (a.hseq) a.hseq[((size_t)t * B + b) * ldseq + (size_t)d * H + u] = hv;
-                    if (a.out) a.out[(size_t)t * a.out_st + (size_t)b * a.out_sb + (size_t)d * H + u] = hv;
-                    if (s == T - 1) {
-                        a.h_n[((size_t)d * B + b) * H + u] = hv;
-                        a.c_n[((size_t)d * B + b) * H + u] = c;
+                    for (int m = 0; m < 4; ++m)
+                        st_cluster_v4(recv_remote + (uint32_t)(((4 * cc + m) * kRows + r) * 16), pv[kk][4 * m],
+                                      pv[kk][4 * m + 1], pv[kk][4 * m + 2], pv[kk][4 * m + 3]);
+                }
+            }
+            mbar_arrive_remote(recv_bar_remote);
+            // 2) the partner's partial sums of the own columns
+            const bool got = mbar_wait_cluster(recv_full, s & 1, abort_flag, a.status, a.timeout_ns);
+            if (named_bar_or(1, kEpi, !got)) break;
+            // 3) gates, cell update and h for the own columns, two chunks at a time
+#pragma unroll
+            for (int k0 = 0; k0 < kCcPerHalf; k0 += 2) {
+                if (half + 2 * k0 >= ncc) break;
+                float ov[2][16];
+#pragma unroll
+                for (int kk = 0; kk < 2; ++kk) {
+                    const int cc = half + 2 * (k0 + kk);
+                    if (cc < ncc) tc::tmem_ld16(trow + (uint32_t)(own0 + 16 * cc), ov[kk]);
+                }
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int kk = 0; kk < 2; ++kk) {
+                    const int k = k0 + kk;
+                    const int cc = half + 2 * k;
+                    if (cc >= ncc) break;
+                    float* v = ov[kk];
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const float4 p4 = recv[(4 * cc + m) * kRows + r];
+                        v[4 * m] += p4.x; v[4 * m + 1] += p4.y; v[4 * m + 2] += p4.z; v[4 * m + 3] += p4.w;
+                    }
+                    // v[4m + i]: gate gq at column 16cc + 4m + i.  Three xor
+                    // exchanges inside each 4-lane group give lane gq all four
+                    // gates at column 16cc + 4gq + i (gate X arrives in round gq ^ X).
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        float rcv[4];
+                        rcv[0] = sel4(v[i], v[4 + i], v[8 + i], v[12 + i], gq);
+#pragma unroll
+                        for (int rr = 1; rr < 4; ++rr)
+                            rcv[rr] =
+                                __shfl_xor_sync(0xffffffffu, sel4(v[i], v[4 + i], v[8 + i], v[12 + i], gq ^ rr), rr);
+                        const float pi = sel4(rcv[0], rcv[1], rcv[2], rcv[3], gq ^ 0);
+                        const float pf = sel4(rcv[0], rcv[1], rcv[2], rcv[3], gq ^ 1);
+                        const float pgg = sel4(rcv[0], rcv[1], rcv[2], rcv[3], gq ^ 2);
+                        const float po = sel4(rcv[0], rcv[1], rcv[2], rcv[3], gq ^ 3);
+                        const int lc = 16 * cc + 4 * gq + i;   // column within the own half
+                        const int col = own0 + lc;
+                        if (col >= nB) continue;
+                        const float ig = sigmoid_fast(pi), fg = sigmoid_fast(pf), gg = tanh_fast(pgg);
+                        const float og = sigmoid_fast(po);
+                        const float c = fg * creg[k][i] + ig * gg;
+                        creg[k][i] = c;
+                        const bf16 hv = __float2bfloat16_rn(og * tanh_fast(c));
+                        // unit octet q of column lc, stored at octet q ^ gq
+                        // ((lc >> 2) & 3 == gq): the four columns of a warp's
+                        // store fall in different banks
+                        sh[lc * 32 + 8 * (q ^ gq) + (lane >> 2)] = hv;
+                        if (s == T - 1) {
+                            const int b = b0 + col;
+                            a.h_n[((size_t)d * B + b) * H + u] = hv;
+                            a.c_n[((size_t)d * B + b) * H + u] = c;
+                        }
                     }
                 }
             }
-            // publish h_t to the group, then hand the accumulator Gx[t+1]
+            // 4) h_t of the own columns to global memory in 16-byte pieces
+            //    (32 units of a column are 64 contiguous bytes), publish it
+            //    to the group, then hand the accumulator Gx[t+1]
+            tc::named_bar_sync(1, kEpi);
+            {
+                bf16* hxo = a.hx + ((size_t)(d * (T + 1) + s + 1) * B) * H + 32 * j;
+                for (int idx = e; idx < NH * 4; idx += kEpi) {
+                    const int lc = idx >> 2, oct = idx & 3;
+                    if (own0 + lc >= nB) continue;
+                    const int b = b0 + own0 + lc;
+                    const uint4 val = *reinterpret_cast<const uint4*>(sh + lc * 32 + 8 * (oct ^ ((lc >> 2) & 3)));
+                    *reinterpret_cast<uint4*>(hxo + (size_t)b * H + 8 * oct) = val;
+                    const size_t uo = (size_t)d * H + 32 * j + 8 * oct;
+                    if (a.hseq) *reinterpret_cast<uint4*>(a.hseq + ((size_t)t * B + b) * ldseq + uo) = val;
+                    if (a.out) {
+                        bf16* dst = a.out + (size_t)t * a.out_st + (size_t)b * a.out_sb + uo;
+                        if (a.out_vec) {
+                            *reinterpret_cast<uint4*>(dst) = val;
+                        } else {
+                            const bf16* sv = reinterpret_cast<const bf16*>(&val);
+#pragma unroll
+                            for (int x = 0; x < 8; ++x) dst[x] = sv[x];
+                        }
+                    }
+                }
+            }
             tc::fence_proxy_async_global();
             tc::named_bar_sync(1, kEpi);
             if (warp == 2 && lane == 0) {
                 __threadfence();
                 atomicAdd(ctr, 1u);
             }
-            // Gx[t+1]: its load latency overlaps the group barrier and the h
-            // TMA that the next step's MMAs wait for anyway
             if (s + 1 < T)
-                preload_gx(a.gx, d == 0 ? s + 1 : T - 2 - s, B, ldgx, prow0 + r, b0, cbase, NH, nB, trow, d_ready);
+                preload_gx(a.gx, d == 0 ? s + 1 : T - 2 - s, B, ldgx, prow0 + r, b0, own0, pcol0, ncc, nB, half, trow,
+                           d_ready);
         }
     }
     tc::tc_fence_before();
@@ -374,35 +567,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::tc_fence_after();
         tc::tmem_dealloc(tmem, 512);
     }
+    cluster_sync();   // neither block leaves while its partner may still write into it
 }
 
 }  // namespace
 
 TcRecPlan plan_tc_rec(int H, int B, int D, int num_sms, size_t smem_max) {
     TcRecPlan p{};
-    if (H % 64 != 0 || B < 1) return p;
+    if (H % 64 != 0 || H < 128 || B < 1) return p;
     const int KT = H / 64;
+    const int KH = (KT + 1) / 2;                      // K chunks of the first block of a pair
     const int nu = 4 * H / kRows;
-    const int kc_smem = std::max(0, KT - 8);
-    const int max_groups = num_sms / (D * nu);
+    const int kc_smem = std::max(0, KH - kMaxTmemChunks);
+    const int max_groups = num_sms / (2 * D * nu);
     if (max_groups < 1) return p;
     int nbg = std::min(max_groups, std::max(1, (B + 31) / 32));
     int Bg = (B + nbg - 1) / nbg;
-    while (((Bg + 31) / 32) * 32 > 16 * kMaxNcc && nbg < max_groups) {
+    while (((Bg + 31) / 32) * 32 > kMaxN && nbg < max_groups) {
         ++nbg;
         Bg = (B + nbg - 1) / nbg;
     }
-    const int N = ((Bg + 31) / 32) * 32;   // two halves of whole 16-column chunks
-    if (N > 16 * kMaxNcc) return p;
+    const int N = ((Bg + 31) / 32) * 32;               // two halves of whole 16-column chunks
+    if (N > kMaxN) return p;
     if (nbg > 1 && (nbg - 1) * Bg >= B) return p;
-    const size_t fixed = (size_t)kc_smem * kChunkW + 1024 + 256;
+    const size_t recv = (size_t)kRows * (N / 2) * 4 + (size_t)(N / 2) * 32 * 2;   // partial sums, h staging
+    const size_t fixed = (size_t)kc_smem * kChunkW + recv + 1024 + 256;
     int stages = 8;
     while (stages >= 2 && fixed + (size_t)stages * N * 128 > smem_max) --stages;
     if (stages < 2) return p;
     p.ok = true;
-    p.nbg = nbg; p.Bg = Bg; p.N = N; p.nu = nu; p.kc_smem = kc_smem; p.stages = stages;
-    p.ctas = D * nbg * nu;
-    p.smem = fixed + (size_t)stages * N * 128;
+    p.nbg = nbg; p.Bg = Bg; p.N = N; p.nu = nu; p.KH = KH; p.kc_smem = kc_smem; p.stages = stages;
+    p.ctas = 2 * D * nbg * nu;
+    p.smem = std::min(smem_max, std::max(kMinSmem, fixed + (size_t)stages * N * 128));
     return p;
 }
 
@@ -439,19 +635,40 @@ cudaError_t launch_tc_rec(const TcRecArgs& a, cudaStream_t s) {
     if (!make_map_bf16(&tmW, a.wpk, (long long)a.D * 4 * a.H, a.H, kRows)) return cudaErrorInvalidValue;
     TcRecParams prm{};
     prm.H = a.H; prm.B = a.B; prm.T = a.T; prm.D = a.D;
-    prm.nbg = p.nbg; prm.Bg = p.Bg; prm.N = p.N; prm.nu = p.nu; prm.kc_smem = p.kc_smem; prm.stages = p.stages;
+    prm.nbg = p.nbg; prm.Bg = p.Bg; prm.N = p.N; prm.nu = p.nu; prm.KH = p.KH;
+    prm.kc_smem = p.kc_smem; prm.stages = p.stages;
     prm.gx = a.gx; prm.c0 = a.c0;
     prm.hx = static_cast<bf16*>(a.hx);
     prm.hseq = static_cast<bf16*>(a.hseq);
     prm.out = static_cast<bf16*>(a.out); prm.out_st = a.out_st; prm.out_sb = a.out_sb;
+    prm.out_vec = (reinterpret_cast<uintptr_t>(a.out) & 15) == 0;
     prm.h_n = static_cast<bf16*>(a.h_n); prm.c_n = a.c_n;
     prm.wpk = static_cast<const bf16*>(a.wpk);
     prm.ctr = a.ctr; prm.status = a.status; prm.timeout_ns = a.timeout_ns;
     cudaError_t e = cudaFuncSetAttribute(tc_rec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
     if (e != cudaSuccess) return e;
-    void* params[] = {&tmH, &tmW, &prm};
-    return cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(&tc_rec_kernel), dim3(p.ctas), dim3(kThreads),
-                                       params, p.smem, s);
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(p.ctas);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = p.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // every block waits on the others of its group: the whole grid must be
+    // resident at once
+    int clusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&clusters, tc_rec_kernel, &cfg);
+    if (e != cudaSuccess) return e;
+    if (2 * clusters < p.ctas) return cudaErrorCooperativeLaunchTooLarge;
+    attr[1].id = cudaLaunchAttributeCooperative;
+    attr[1].val.cooperative = 1;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, tc_rec_kernel, tmH, tmW, prm);
 }
 
 }  // namespace lstm
