@@ -63,11 +63,23 @@ def load_peaks():
 
 
 # --------------------------------------------------------------- work model
+ENGINE_SUFFIXES = ("_tc", "_ffma", "_simt")
+
+
+def kind_base(kind):
+    """Kernel kind without its engine suffix (fwd_rec_tc -> fwd_rec)."""
+    for suf in ENGINE_SUFFIXES:
+        if kind.endswith(suf):
+            return kind[: -len(suf)]
+    return kind
+
+
 def kernel_work(wl, kind):
     """Algorithmic work of all launches of `kind` in one step: (units, amount).
 
     Recurrences and GEMMs count 2 flops per multiply-add of the matrix
     products the method defines (elementwise gate math is not counted)."""
+    kind = kind_base(kind)
     B, T, H, D, L, G = wl.B, wl.T, wl.H, wl.D, wl.L, 4 * wl.H
     ins = [wl.in_size(k) for k in range(L)]
     if kind == "fwd_rec":
@@ -83,11 +95,18 @@ def kernel_work(wl, kind):
     return None, 0.0
 
 
-# Bound and peak of each kernel kind as the library implements it.
+# Bound of each kernel kind, from the engine suffix the library reports:
 #   alu:    FP32 FMA on the CUDA cores, 148 SMs x 128 lanes x 2 flop x max SM clock
-#   tensor: tcgen05 tensor cores (peak from the measured cuBLAS bf16 figure)
-KIND_BOUND = {"fwd_rec": "alu", "bwd_rec": "alu", "proj_gemm": "alu", "dw_gemm": "alu",
-              "dx_gemm": "alu"}
+#   tensor: tcgen05 tensor cores.  bf16 operands: the measured cuBLAS bf16 burst
+#           peak.  fp32 operands run as 3xTF32 (three tf32 products per fp32
+#           product): the bf16 peak x 1.1/2.25 (nominal tf32/bf16 dense ratio) / 3.
+COUNTED_KINDS = ("fwd_rec", "bwd_rec", "proj_gemm", "dw_gemm", "dx_gemm")
+
+
+def kind_bound(kind):
+    if kind_base(kind) not in COUNTED_KINDS:
+        return None
+    return "tensor" if kind.endswith("_tc") else "alu"
 
 
 def alu_peak_tflops():
@@ -362,20 +381,24 @@ def run_ours(args):
     # ------------------------------------------------------------- roofline
     peaks = load_peaks()
     roof = None
-    dom = max(((k, v) for k, v in kern.items() if v[0] > 0 and KIND_BOUND.get(k)),
+    dom = max(((k, v) for k, v in kern.items() if v[0] > 0 and kind_bound(k)),
               key=lambda kv: kv[1][1], default=None)
     if dom is not None:
         kind, (launches, kms) = dom
         unit, work_step = kernel_work(wl, kind)
         per_launch = work_step * args.steps / launches
         avg_s = kms / launches / 1e3
-        bound = KIND_BOUND[kind]
+        bound = kind_bound(kind)
         if bound == "alu":
             peak = alu_peak_tflops()
             peak_note = "derived: 148 SMs x 128 FP32 lanes x 2 flop x 1965 MHz"
+        elif wl.dtype == "bf16":
+            peak = peaks["bf16_tflops"]
+            peak_note = f"{peaks['source']} bf16 burst"
         else:
-            peak = peaks["bf16_tflops_sustained"]
-            peak_note = f"{peaks['source']} bf16 sustained"
+            peak = peaks["bf16_tflops"] * 1.1 / 2.25 / 3.0
+            peak_note = (f"{peaks['source']} bf16 burst x 1.1/2.25 (tf32) / 3 (3xTF32 products "
+                         "per fp32 product)")
         achieved = per_launch / avg_s / 1e12
         traffic = traffic_for(kind, wl.name)
         roof = {"bound": bound, "kernel": kind, "achieved": achieved, "peak": peak,

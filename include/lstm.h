@@ -185,8 +185,11 @@ const char* lstm_status_string(lstm_status status);
  * events, adds their durations to per-kind totals and copies up to
  * max_entries {name, launches, total_ms} records into `out` (a host array);
  * it returns the number of records written (the number of kinds when out is
- * NULL), or -1 if an event could not be read.  Kinds: pack, proj_gemm,
- * fwd_rec, bwd_rec, dw_gemm, dx_gemm, db_reduce, seq_copy.  lstm_timing_reset
+ * NULL), or -1 if an event could not be read.  Kinds (the suffix names the
+ * engine: _tc tensor cores, _ffma / _simt CUDA cores): pack, proj_gemm_tc,
+ * proj_gemm_simt, fwd_rec_tc, fwd_rec_ffma, bwd_rec_ffma, dw_gemm_tc,
+ * dw_gemm_simt, dx_gemm_tc, dx_gemm_simt, db_reduce, seq_copy, transpose.
+ * lstm_timing_reset
  * zeroes the totals.  Process-wide and thread-safe; event recording adds a
  * few microseconds per launch, so leave it off outside measurements.
  */

@@ -60,9 +60,16 @@ uint64_t timeout_ns() {
 // When enabled, every kernel the library launches is bracketed by a pair of
 // CUDA events on its stream; lstm_timing_read() resolves them into per-kind
 // launch counts and summed device durations.
-enum Kind { K_PACK = 0, K_PROJ, K_FWD_REC, K_BWD_REC, K_DW, K_DX, K_DB, K_COPY, K_COUNT };
-const char* const kKindNames[K_COUNT] = {"pack", "proj_gemm", "fwd_rec", "bwd_rec",
-                                         "dw_gemm", "dx_gemm", "db_reduce", "seq_copy"};
+// Kind names carry the engine: _tc tensor cores (tcgen05), _ffma / _simt the
+// CUDA cores.
+enum Kind {
+    K_PACK = 0, K_PROJ_TC, K_PROJ_SIMT, K_FWD_REC_TC, K_FWD_REC_FFMA, K_BWD_REC_FFMA, K_DW_TC, K_DW_SIMT,
+    K_DX_TC, K_DX_SIMT, K_DB, K_COPY, K_TRANSPOSE, K_COUNT
+};
+const char* const kKindNames[K_COUNT] = {"pack",       "proj_gemm_tc", "proj_gemm_simt", "fwd_rec_tc",
+                                         "fwd_rec_ffma", "bwd_rec_ffma", "dw_gemm_tc",   "dw_gemm_simt",
+                                         "dx_gemm_tc", "dx_gemm_simt", "db_reduce",    "seq_copy",
+                                         "transpose"};
 
 struct Timing {
     std::mutex mu;
@@ -418,11 +425,11 @@ lstm_status lstm_forward(const lstm_desc* desc, const void* x, const void* h0, c
         tg.A = g.A; tg.lda = in; tg.B = g.B; tg.ldb = in;
         tg.C = static_cast<float*>(g.C); tg.ldc = g.ldc;
         tg.bias = g.bias; tg.remap_T = g.remap_T; tg.remap_B = g.remap_B;
-        tg.status = status; tg.timeout_ns = timeout_ns();
+        tg.status = status; tg.timeout_ns = timeout_ns(); tg.num_sms = device_info().sms;
         if (tc_gemm_enabled() && tc_gemm_supported(tg)) {
-            LSTM_CUDA(timed(K_PROJ, stream, [&] { return launch_tc_gemm(tg, stream); }));
+            LSTM_CUDA(timed(K_PROJ_TC, stream, [&] { return launch_tc_gemm(tg, stream); }));
         } else {
-            LSTM_CUDA(timed(K_PROJ, stream, [&] { return launch_gemm(g, stream); }));
+            LSTM_CUDA(timed(K_PROJ_SIMT, stream, [&] { return launch_gemm(g, stream); }));
         }
 
         void* hseq_tc = reserve ? P(reserve, l.hseq[k]) : P(workspace, l.seq[k & 1]);
@@ -459,7 +466,7 @@ lstm_status lstm_forward(const lstm_desc* desc, const void* x, const void* h0, c
             tr.ctr = reinterpret_cast<unsigned*>(P(workspace, l.ctr_tc)) + (size_t)k * D * l.tcr.nbg * 32;
             tr.status = status;
             tr.timeout_ns = timeout_ns();
-            LSTM_CUDA(timed(K_FWD_REC, stream, [&] { return launch_tc_rec(tr, stream); }));
+            LSTM_CUDA(timed(K_FWD_REC_TC, stream, [&] { return launch_tc_rec(tr, stream); }));
             layer_in = hseq_tc;
             continue;
         }
@@ -493,7 +500,7 @@ lstm_status lstm_forward(const lstm_desc* desc, const void* x, const void* h0, c
         f.ctr = reinterpret_cast<unsigned*>(P(workspace, l.ctr_f)) + (size_t)k * D * l.nbg_ctr;
         f.status = status;
         f.timeout_ns = timeout_ns();
-        LSTM_CUDA(timed(K_FWD_REC, stream, [&] { return launch_fwd_rec(f, stream); }));
+        LSTM_CUDA(timed(K_FWD_REC_FFMA, stream, [&] { return launch_fwd_rec(f, stream); }));
         layer_in = hseq;
     }
     return LSTM_OK;
@@ -595,7 +602,7 @@ lstm_status lstm_backward(const lstm_desc* desc, const void* x, const void* h0, 
         b.ctr = reinterpret_cast<unsigned*>(P(workspace, l.ctr_b)) + (size_t)k * D * l.bwd.nbg;
         b.status = status;
         b.timeout_ns = timeout_ns();
-        LSTM_CUDA(timed(K_BWD_REC, stream, [&] { return launch_bwd_rec(b, stream); }));
+        LSTM_CUDA(timed(K_BWD_REC_FFMA, stream, [&] { return launch_bwd_rec(b, stream); }));
 
         if (desc->bias) {
             DbArgs db{};
@@ -618,20 +625,20 @@ lstm_status lstm_backward(const lstm_desc* desc, const void* x, const void* h0, 
         tw.M = G; tw.N = in + H; tw.K = (int)BTl; tw.dt = DType::F32;
         tw.A = dGT; tw.lda = BTl; tw.B = bop; tw.ldb = BTl;
         tw.C = dw_ih[k * D]; tw.ldc = in; tw.C1 = dw_hh[k * D]; tw.ldc1 = H; tw.n_split = in;
-        tw.status = status; tw.timeout_ns = timeout_ns();
+        tw.status = status; tw.timeout_ns = timeout_ns(); tw.num_sms = device_info().sms;
         TcGemmArgs tx{};
         tx.M = (int)BTl; tx.N = in; tx.K = D * G; tx.dt = DType::F32;
         tx.A = dG; tx.lda = ldg; tx.B = wcatT; tx.ldb = (long long)D * G;
         tx.C = din; tx.ldc = in;
         if (k == 0 && desc->batch_first) { tx.remap_T = -T; tx.remap_B = B; }
-        tx.status = status; tx.timeout_ns = timeout_ns();
+        tx.status = status; tx.timeout_ns = timeout_ns(); tx.num_sms = device_info().sms;
         const bool tc_ok = tc_gemm_enabled() && tc_gemm_supported(tw) && tc_gemm_supported(tx) &&
                            (reinterpret_cast<uintptr_t>(dw_ih[k * D]) & 3) == 0;
         if (tc_ok) {
             TransposeArgs ta{};
             ta.M = (int)BTl; ta.C = D * G; ta.mode = 0; ta.src = dG; ta.lds = ldg;
             ta.dst = dGT; ta.ldd = BTl;
-            LSTM_CUDA(timed(K_COPY, stream, [&] { return launch_transpose(ta, stream); }));
+            LSTM_CUDA(timed(K_TRANSPOSE, stream, [&] { return launch_transpose(ta, stream); }));
             for (int d = 0; d < D; ++d) {
                 float* bo = bop + (size_t)d * (in + H) * BTl;
                 TransposeArgs ti{};
@@ -644,26 +651,26 @@ lstm_status lstm_backward(const lstm_desc* desc, const void* x, const void* h0, 
                     ti.lds = in;
                 }
                 ti.dst = bo; ti.ldd = BTl;
-                LSTM_CUDA(timed(K_COPY, stream, [&] { return launch_transpose(ti, stream); }));
+                LSTM_CUDA(timed(K_TRANSPOSE, stream, [&] { return launch_transpose(ti, stream); }));
                 TransposeArgs th{};
                 th.M = (int)BTl; th.C = H; th.mode = 1;
                 th.src = hs + (size_t)d * H; th.lds = ldh; th.T = T; th.B = B; th.dir = d;
                 th.h0 = h0 ? static_cast<const float*>(h0) + ((size_t)k * D + d) * B * H : nullptr;
                 th.dst = bo + (size_t)in * BTl; th.ldd = BTl;
-                LSTM_CUDA(timed(K_COPY, stream, [&] { return launch_transpose(th, stream); }));
+                LSTM_CUDA(timed(K_TRANSPOSE, stream, [&] { return launch_transpose(th, stream); }));
                 TcGemmArgs twd = tw;
                 twd.A = dGT + (size_t)d * G * BTl;
                 twd.B = bo;
                 twd.C = dw_ih[k * D + d];
                 twd.C1 = dw_hh[k * D + d];
-                LSTM_CUDA(timed(K_DW, stream, [&] { return launch_tc_gemm(twd, stream); }));
+                LSTM_CUDA(timed(K_DW_TC, stream, [&] { return launch_tc_gemm(twd, stream); }));
                 TransposeArgs tww{};
                 tww.M = G; tww.C = in; tww.mode = 0;
                 tww.src = static_cast<const float*>(w_ih[k * D + d]); tww.lds = in;
                 tww.dst = wcatT + (size_t)d * G; tww.ldd = (long long)D * G;
-                LSTM_CUDA(timed(K_COPY, stream, [&] { return launch_transpose(tww, stream); }));
+                LSTM_CUDA(timed(K_TRANSPOSE, stream, [&] { return launch_transpose(tww, stream); }));
             }
-            LSTM_CUDA(timed(K_DX, stream, [&] { return launch_tc_gemm(tx, stream); }));
+            LSTM_CUDA(timed(K_DX_TC, stream, [&] { return launch_tc_gemm(tx, stream); }));
         } else {
             for (int d = 0; d < D; ++d) {
                 // dW_ih = sum_t dG_t^T x_t
@@ -672,7 +679,7 @@ lstm_status lstm_backward(const lstm_desc* desc, const void* x, const void* h0, 
                 g.A = dG + (size_t)d * G; g.ta = DType::F32; g.sAm = 1; g.sAk = ldg;
                 g.B = layer_in; g.tb = DType::F32; g.sBk = in; g.sBn = 1;
                 g.C = dw_ih[k * D + d]; g.tc = DType::F32; g.ldc = in;
-                LSTM_CUDA(timed(K_DW, stream, [&] { return launch_gemm(g, stream); }));
+                LSTM_CUDA(timed(K_DW_SIMT, stream, [&] { return launch_gemm(g, stream); }));
                 // dW_hh = sum_t dG_t^T h_{t-1} (h_{-1} = h0)
                 GemmArgs gh{};
                 gh.M = G; gh.N = H; gh.K = B * (T - 1);
@@ -687,7 +694,7 @@ lstm_status lstm_backward(const lstm_desc* desc, const void* x, const void* h0, 
                     gh.B = hs + (size_t)B * ldh + (size_t)d * H;      // h at t+1
                 }
                 if (T > 1) {
-                    LSTM_CUDA(timed(K_DW, stream, [&] { return launch_gemm(gh, stream); }));
+                    LSTM_CUDA(timed(K_DW_SIMT, stream, [&] { return launch_gemm(gh, stream); }));
                 } else {
                     LSTM_CUDA(cudaMemsetAsync(dw_hh[k * D + d], 0, (size_t)G * H * 4, stream));
                 }
@@ -698,7 +705,7 @@ lstm_status lstm_backward(const lstm_desc* desc, const void* x, const void* h0, 
                     g0.B = static_cast<const float*>(h0) + ((size_t)k * D + d) * B * H;
                     g0.sBk = H;
                     g0.accumulate = 1;
-                    LSTM_CUDA(timed(K_DW, stream, [&] { return launch_gemm(g0, stream); }));
+                    LSTM_CUDA(timed(K_DW_SIMT, stream, [&] { return launch_gemm(g0, stream); }));
                 }
             }
             // gradient w.r.t. the layer input: sum_d dG_d W_ih_d
@@ -710,7 +717,7 @@ lstm_status lstm_backward(const lstm_desc* desc, const void* x, const void* h0, 
                 g.C = din; g.tc = DType::F32; g.ldc = in;
                 g.accumulate = d > 0;
                 if (k == 0 && desc->batch_first) { g.remap_T = -T; g.remap_B = B; }
-                LSTM_CUDA(timed(K_DX, stream, [&] { return launch_gemm(g, stream); }));
+                LSTM_CUDA(timed(K_DX_SIMT, stream, [&] { return launch_gemm(g, stream); }));
             }
         }
         if (k > 0) {

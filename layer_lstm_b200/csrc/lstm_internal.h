@@ -49,6 +49,7 @@ struct TcGemmArgs {
     float* ws;
     int* status;
     uint64_t timeout_ns;
+    int num_sms;                // persistent grid size (SMs of the device)
 };
 bool tc_gemm_supported(const TcGemmArgs& g);
 int tc_gemm_tile_n(DType dt);

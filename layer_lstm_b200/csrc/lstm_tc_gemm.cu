@@ -6,10 +6,11 @@
 // layer-input gradient dX = dG W_ih.
 //
 // C[M x N] = A[M x K] * B[N x K]^T with both operands K-major in global
-// memory.  One CTA computes a 128 x BN tile; warp 0 issues TMA tile loads
-// into a ring of shared-memory stages, warp 1 (one thread) issues tcgen05.mma
-// into a TMEM accumulator, warps 4-7 drain TMEM through registers to global
-// memory.  bf16 operands use kind::f16.  float32 operands use three
+// memory.  A persistent grid (one CTA per SM) walks the 128 x BN output tiles;
+// warp 0 issues TMA tile loads into a ring of shared-memory stages, warp 1
+// (one thread) issues tcgen05.mma into one of two TMEM accumulators, warps
+// 4-7 drain the other accumulator through registers to global memory while
+// the next tile's MMAs run.  bf16 operands use kind::f16.  float32 operands use three
 // kind::tf32 products per K step, hi*hi + hi*lo + lo*hi with hi = x with its
 // low 13 mantissa bits cleared and lo = x - hi (exact in fp32); warps 2-3
 // split each stage in shared memory before the MMAs read it.  This is the
@@ -38,13 +39,16 @@ template <> struct Cfg<1> {   // 3xTF32
     static constexpr int STAGE_BYTES = 2 * (A_BYTES + B_BYTES);   // hi tiles, then lo tiles
 };
 
+constexpr int kStageFloats = 4 * 32 * 33;   // epilogue staging: one 32 x 33 block per epilogue warp
+
 template <int KIND>
 constexpr size_t smem_bytes() {
-    return (size_t)Cfg<KIND>::STAGES * Cfg<KIND>::STAGE_BYTES + 1024 + 256;
+    return (size_t)Cfg<KIND>::STAGES * Cfg<KIND>::STAGE_BYTES + (size_t)kStageFloats * 4 + 1024 + 256;
 }
 
 struct TcEpi {
     int M, N, K, k_per_split;
+    int tiles_n, tiles_m, splits;   // tile t: n-tile t % tiles_n, then m-tile, then split
     float* C; long long ldc;
     float* C1; long long ldc1; int n_split;
     const float* bias;
@@ -69,6 +73,28 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
     }
 }
 
+struct TileCoord {
+    int m0, n0, split, kbeg, nk;
+};
+
+template <int KIND>
+__device__ __forceinline__ TileCoord tile_coord(const TcEpi& e, int t) {
+    using Cf = Cfg<KIND>;
+    TileCoord c;
+    const int tn = t % e.tiles_n;
+    const int tm = (t / e.tiles_n) % e.tiles_m;
+    c.split = t / (e.tiles_n * e.tiles_m);
+    c.m0 = tm * Cf::BM;
+    c.n0 = tn * Cf::BN;
+    c.kbeg = c.split * e.k_per_split;
+    const int kend = min(e.K, c.kbeg + e.k_per_split);
+    c.nk = kend > c.kbeg ? (kend - c.kbeg + Cf::BK - 1) / Cf::BK : 0;
+    return c;
+}
+
+// Persistent: block b computes tiles b, b + gridDim.x, ...  Two accumulators
+// of BN tensor-memory columns alternate between tiles, so the epilogue of
+// one tile overlaps the loads and MMAs of the next.
 template <int KIND>
 __global__ void __launch_bounds__(256, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, TcEpi e) {
@@ -76,18 +102,17 @@ __global__ void __launch_bounds__(256, 1)
     constexpr int S = Cf::STAGES, BM = Cf::BM, BN = Cf::BN, BK = Cf::BK;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * Cf::STAGE_BYTES);
+    float* stage_out = reinterpret_cast<float*>(smem + S * Cf::STAGE_BYTES);
+    uint64_t* full = reinterpret_cast<uint64_t*>(stage_out + kStageFloats);
     uint64_t* lofull = full + S;
     uint64_t* empty = lofull + S;
-    uint64_t* tmem_full = empty + S;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_full + 1);
+    uint64_t* tmem_full = empty + S;       // [2]
+    uint64_t* tmem_empty = tmem_full + 2;  // [2]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_empty + 2);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN, split = blockIdx.z;
-    const int kbeg = split * e.k_per_split;
-    const int kend = min(e.K, kbeg + e.k_per_split);
-    const int nk = kend > kbeg ? (kend - kbeg + BK - 1) / BK : 0;
+    const int ntiles = e.tiles_n * e.tiles_m * e.splits;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -95,12 +120,15 @@ __global__ void __launch_bounds__(256, 1)
             tc::mbar_init(&lofull[s], 64);
             tc::mbar_init(&empty[s], 1);
         }
-        tc::mbar_init(tmem_full, 1);
+        for (int b = 0; b < 2; ++b) {
+            tc::mbar_init(&tmem_full[b], 1);
+            tc::mbar_init(&tmem_empty[b], 4);   // one arrive per epilogue warp
+        }
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
     if (warp == 1) {
-        tc::tmem_alloc(tmem_slot, BN);
+        tc::tmem_alloc(tmem_slot, 2 * BN);
         tc::tmem_relinquish();
     }
     tc::tc_fence_before();
@@ -112,111 +140,149 @@ __global__ void __launch_bounds__(256, 1)
         if (lane == 0) {
             tc::prefetch_tmap(&tmA);
             tc::prefetch_tmap(&tmB);
-            int issued = 0;
-            for (int kt = 0; kt < nk; ++kt) {
-                const int s = kt % S, r = kt / S;
-                if (!tc::mbar_wait(&empty[s], (r & 1) ^ 1, abort_flag, e.status, e.timeout_ns)) break;
-                unsigned char* st = smem + s * Cf::STAGE_BYTES;
-                tc::mbar_arrive_expect_tx(&full[s], Cf::A_BYTES + Cf::B_BYTES);
-                const int kx = kbeg + kt * BK;
-                tc::tma_load_2d(st, &tmA, kx, m0, &full[s]);
-                tc::tma_load_2d(st + Cf::A_BYTES, &tmB, kx, n0, &full[s]);
-                issued = kt + 1;
+            int it = 0;   // k-chunks issued so far, over all tiles of this block
+            bool ok = true;
+            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+                const TileCoord c = tile_coord<KIND>(e, t);
+                for (int kt = 0; kt < c.nk; ++kt, ++it) {
+                    const int s = it % S, r = it / S;
+                    if (!tc::mbar_wait(&empty[s], (r & 1) ^ 1, abort_flag, e.status, e.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    unsigned char* st = smem + s * Cf::STAGE_BYTES;
+                    tc::mbar_arrive_expect_tx(&full[s], Cf::A_BYTES + Cf::B_BYTES);
+                    const int kx = c.kbeg + kt * BK;
+                    tc::tma_load_2d(st, &tmA, kx, c.m0, &full[s]);
+                    tc::tma_load_2d(st + Cf::A_BYTES, &tmB, kx, c.n0, &full[s]);
+                }
             }
             if (*abort_flag) {   // let this block's copies land before shared memory is released
-                for (int kt = issued > S ? issued - S : 0; kt < issued; ++kt) mbar_drain(&full[kt % S], (kt / S) & 1);
+                for (int k = it > S ? it - S : 0; k < it; ++k) mbar_drain(&full[k % S], (k / S) & 1);
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
             constexpr uint32_t idesc = tc::instr_desc(Cf::FMT, BM, BN);
-            int last = -1;
-            for (int kt = 0; kt < nk; ++kt) {
-                const int s = kt % S, r = kt / S;
-                uint64_t* ready = KIND == 1 ? &lofull[s] : &full[s];
-                if (!tc::mbar_wait(ready, r & 1, abort_flag, e.status, e.timeout_ns)) break;
+            int it = 0, last = -1, i = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++i) {
+                const TileCoord c = tile_coord<KIND>(e, t);
+                const int ab = i & 1;
+                // the epilogue has drained this accumulator (tile i - 2)
+                if (!tc::mbar_wait(&tmem_empty[ab], ((i >> 1) & 1) ^ 1, abort_flag, e.status, e.timeout_ns)) break;
                 tc::tc_fence_after();
-                unsigned char* st = smem + s * Cf::STAGE_BYTES;
-                const uint32_t a_base = tc::smem_u32(st);
-                const uint32_t b_base = a_base + Cf::A_BYTES;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint64_t ad = tc::smem_desc_sw128(a_base + j * 32);
-                    const uint64_t bd = tc::smem_desc_sw128(b_base + j * 32);
-                    const uint32_t acc = (kt | j) != 0;
-                    if (KIND == 0) {
-                        tc::mma_bf16(tmem, ad, bd, idesc, acc);
-                    } else {
-                        const uint32_t lo_off = Cf::A_BYTES + Cf::B_BYTES;
-                        const uint64_t adl = tc::smem_desc_sw128(a_base + lo_off + j * 32);
-                        const uint64_t bdl = tc::smem_desc_sw128(b_base + lo_off + j * 32);
-                        tc::mma_tf32(tmem, adl, bd, idesc, acc);    // lo * hi
-                        tc::mma_tf32(tmem, ad, bdl, idesc, 1);      // hi * lo
-                        tc::mma_tf32(tmem, ad, bd, idesc, 1);       // hi * hi
+                const uint32_t acc_t = tmem + (uint32_t)(ab * BN);
+                for (int kt = 0; kt < c.nk; ++kt, ++it) {
+                    const int s = it % S, r = it / S;
+                    uint64_t* ready = KIND == 1 ? &lofull[s] : &full[s];
+                    if (!tc::mbar_wait(ready, r & 1, abort_flag, e.status, e.timeout_ns)) {
+                        ok = false;
+                        break;
                     }
+                    tc::tc_fence_after();
+                    unsigned char* st = smem + s * Cf::STAGE_BYTES;
+                    const uint32_t a_base = tc::smem_u32(st);
+                    const uint32_t b_base = a_base + Cf::A_BYTES;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint64_t ad = tc::smem_desc_sw128(a_base + j * 32);
+                        const uint64_t bd = tc::smem_desc_sw128(b_base + j * 32);
+                        const uint32_t acc = (kt | j) != 0;
+                        if (KIND == 0) {
+                            tc::mma_bf16(acc_t, ad, bd, idesc, acc);
+                        } else {
+                            const uint32_t lo_off = Cf::A_BYTES + Cf::B_BYTES;
+                            const uint64_t adl = tc::smem_desc_sw128(a_base + lo_off + j * 32);
+                            const uint64_t bdl = tc::smem_desc_sw128(b_base + lo_off + j * 32);
+                            tc::mma_tf32(acc_t, adl, bd, idesc, acc);   // lo * hi
+                            tc::mma_tf32(acc_t, ad, bdl, idesc, 1);     // hi * lo
+                            tc::mma_tf32(acc_t, ad, bd, idesc, 1);      // hi * hi
+                        }
+                    }
+                    tc::mma_commit(&empty[s]);
+                    last = it;
                 }
-                tc::mma_commit(&empty[s]);
-                last = kt;
+                if (!ok) break;
+                tc::mma_commit(&tmem_full[ab]);
             }
-            tc::mma_commit(tmem_full);
             if (*abort_flag && last >= 0) mbar_drain(&empty[last % S], (last / S) & 1);
         }
     } else if (KIND == 1 && warp < 4) {
         // hi/lo split of each stage (64 threads), in place for hi.
         const int ct = threadIdx.x - 64;
-        for (int kt = 0; kt < nk; ++kt) {
-            const int s = kt % S, r = kt / S;
-            if (!tc::mbar_wait(&full[s], r & 1, abort_flag, e.status, e.timeout_ns)) break;
-            float4* hi = reinterpret_cast<float4*>(smem + s * Cf::STAGE_BYTES);
-            float4* lo = reinterpret_cast<float4*>(smem + s * Cf::STAGE_BYTES + Cf::A_BYTES + Cf::B_BYTES);
-            constexpr int NV = (Cf::A_BYTES + Cf::B_BYTES) / 16;
+        int it = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            const TileCoord c = tile_coord<KIND>(e, t);
+            for (int kt = 0; kt < c.nk; ++kt, ++it) {
+                const int s = it % S, r = it / S;
+                if (!tc::mbar_wait(&full[s], r & 1, abort_flag, e.status, e.timeout_ns)) {
+                    ok = false;
+                    break;
+                }
+                float4* hi = reinterpret_cast<float4*>(smem + s * Cf::STAGE_BYTES);
+                float4* lo = reinterpret_cast<float4*>(smem + s * Cf::STAGE_BYTES + Cf::A_BYTES + Cf::B_BYTES);
+                constexpr int NV = (Cf::A_BYTES + Cf::B_BYTES) / 16;
 #pragma unroll 4
-            for (int i = ct; i < NV; i += 64) {
-                const float4 x = hi[i];
-                float4 h, l;
-                h.x = __uint_as_float(__float_as_uint(x.x) & 0xFFFFE000u); l.x = x.x - h.x;
-                h.y = __uint_as_float(__float_as_uint(x.y) & 0xFFFFE000u); l.y = x.y - h.y;
-                h.z = __uint_as_float(__float_as_uint(x.z) & 0xFFFFE000u); l.z = x.z - h.z;
-                h.w = __uint_as_float(__float_as_uint(x.w) & 0xFFFFE000u); l.w = x.w - h.w;
-                hi[i] = h;
-                lo[i] = l;
+                for (int i = ct; i < NV; i += 64) {
+                    const float4 x = hi[i];
+                    float4 h, l;
+                    h.x = __uint_as_float(__float_as_uint(x.x) & 0xFFFFE000u); l.x = x.x - h.x;
+                    h.y = __uint_as_float(__float_as_uint(x.y) & 0xFFFFE000u); l.y = x.y - h.y;
+                    h.z = __uint_as_float(__float_as_uint(x.z) & 0xFFFFE000u); l.z = x.z - h.z;
+                    h.w = __uint_as_float(__float_as_uint(x.w) & 0xFFFFE000u); l.w = x.w - h.w;
+                    hi[i] = h;
+                    lo[i] = l;
+                }
+                tc::fence_proxy_async_smem();
+                tc::mbar_arrive(&lofull[s]);
             }
-            tc::fence_proxy_async_smem();
-            tc::mbar_arrive(&lofull[s]);
         }
     } else if (warp >= 4) {
         // Epilogue: each warp drains its 32 accumulator rows in 32 x 32
-        // blocks staged through shared memory (the pipeline stages are idle
-        // once every MMA has completed), so each global store instruction
-        // writes one contiguous 128-byte row segment.
+        // blocks staged through its own shared-memory block, so each global
+        // store instruction writes one contiguous 128-byte row segment.
         const int q = warp & 3;
-        const bool ok = tc::mbar_wait(tmem_full, 0, abort_flag, e.status, e.timeout_ns);
-        tc::tc_fence_after();
-        float* stg = reinterpret_cast<float*>(smem) + q * (32 * 33);
-        // Output row of accumulator row (q*32 + lane), computed once per tile
-        // and broadcast inside the row loop.
-        const int mrow = m0 + q * 32 + lane;
-        const long long my_row = e.ws ? (long long)mrow : out_row(e, mrow);
-        const int rows_here = min(32, e.M - (m0 + q * 32));
-        if (ok) {
-            for (int c = 0; c < BN; c += 32) {
+        float* stg = stage_out + q * (32 * 33);
+        int i = 0;
+        for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++i) {
+            const TileCoord c = tile_coord<KIND>(e, t);
+            const int ab = i & 1;
+            const bool ok = tc::mbar_wait(&tmem_full[ab], (i >> 1) & 1, abort_flag, e.status, e.timeout_ns);
+            if (!ok) break;
+            tc::tc_fence_after();
+            const uint32_t acc_t = tmem + (uint32_t)(ab * BN) + ((uint32_t)(q * 32) << 16);
+            // Output row of accumulator row (q*32 + lane), computed once per
+            // tile and broadcast inside the row loop.
+            const int mrow = c.m0 + q * 32 + lane;
+            const long long my_row = e.ws ? (long long)mrow : out_row(e, mrow);
+            const int rows_here = min(32, e.M - (c.m0 + q * 32));
+            for (int cc = 0; cc < BN; cc += 32) {
                 float v[16], w[16];
-                tc::tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c, v);
-                tc::tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(c + 16), w);
+                tc::tmem_ld16(acc_t + (uint32_t)cc, v);
+                tc::tmem_ld16(acc_t + (uint32_t)(cc + 16), w);
                 tc::tmem_ld_wait();
+                if (cc + 32 >= BN) {
+                    // every column of this accumulator is in registers: hand
+                    // it back to the MMA warp before the stores
+                    tc::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(&tmem_empty[ab]);
+                }
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    stg[lane * 33 + i] = nk ? v[i] : 0.f;
-                    stg[lane * 33 + 16 + i] = nk ? w[i] : 0.f;
+                for (int k = 0; k < 16; ++k) {
+                    stg[lane * 33 + k] = c.nk ? v[k] : 0.f;
+                    stg[lane * 33 + 16 + k] = c.nk ? w[k] : 0.f;
                 }
                 __syncwarp();
-                const int n = n0 + c + lane;
+                const int n = c.n0 + cc + lane;
                 const bool ncol = n < e.N;
                 const float bn = (!e.ws && e.bias && ncol) ? e.bias[n] : 0.f;
                 float* base;
                 long long ld;
                 if (e.ws) {
-                    base = e.ws + (size_t)split * e.M * e.N + n;
+                    base = e.ws + (size_t)c.split * e.M * e.N + n;
                     ld = e.N;
                 } else if (n < e.n_split) {
                     base = e.C + n;
@@ -243,7 +309,7 @@ __global__ void __launch_bounds__(256, 1)
     __syncthreads();
     if (warp == 1) {
         tc::tc_fence_after();
-        tc::tmem_dealloc(tmem, BN);
+        tc::tmem_dealloc(tmem, 2 * BN);
     }
 }
 
@@ -317,7 +383,11 @@ cudaError_t launch_kind(const TcGemmArgs& g, cudaStream_t s) {
     cudaError_t err = cudaFuncSetAttribute(tc_gemm_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)smem);
     if (err != cudaSuccess) return err;
-    dim3 grid((g.N + Cf::BN - 1) / Cf::BN, (g.M + Cf::BM - 1) / Cf::BM, splits);
+    e.tiles_n = (g.N + Cf::BN - 1) / Cf::BN;
+    e.tiles_m = (g.M + Cf::BM - 1) / Cf::BM;
+    e.splits = splits;
+    const long long ntiles = (long long)e.tiles_n * e.tiles_m * splits;
+    const int grid = (int)std::min<long long>(ntiles, g.num_sms > 0 ? g.num_sms : 148);
     tc_gemm_kernel<KIND><<<grid, 256, smem, s>>>(ta, tb, e);
     err = cudaGetLastError();
     if (err != cudaSuccess || splits == 1) return err;
