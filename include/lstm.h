@@ -203,6 +203,39 @@ lstm_status lstm_timing_enable(int enable);
 int lstm_timing_read(lstm_kernel_time* out, int max_entries);
 void lstm_timing_reset(void);
 
+/*
+ * Per-step timeline of a recurrent kernel (instrumentation; the pages define
+ * no counterpart).  While enabled, every recurrent launch has thread(s) of
+ * block 0 stamp %globaltimer (ns) at fixed points of each step into a static
+ * device buffer of LSTM_TRACE_MAX_STEPS x LSTM_TRACE_EVENTS entries, zeroed
+ * before the launch; each launch overwrites the previous one, so after a
+ * multi-layer call the buffer holds the last recurrent launch.
+ * lstm_trace_read copies min(max_steps, steps of that launch) rows of
+ * LSTM_TRACE_EVENTS values into `out` (host memory) and returns the number of
+ * rows (0 if nothing was traced, -1 on a CUDA error); *kind (if non-null)
+ * receives the kernel, LSTM_TRACE_*.  The caller synchronises the launch's
+ * stream first.  Unused events stay 0.  Events by kernel:
+ *   LSTM_TRACE_FWD_REC_FFMA: 0 step start, 1 group wait done, 2 h tile in
+ *     shared memory, 3 matvec done (first batch sub-tile), 4 cell update
+ *     done, 5 arrival published.
+ *   LSTM_TRACE_BWD_REC_FFMA: 0 step start, 1 group wait done, 2 partial-dh
+ *     gather done, 3 gate gradients done (first sub-tile), 4 partial dh
+ *     products done, 5 arrival published.
+ *   LSTM_TRACE_FWD_REC_TC: 0 producer passed the group wait, 1 last h TMA
+ *     issued, 2 accumulator initialised (MMA thread), 9 first h chunk landed,
+ *     3 MMAs committed, 4 epilogue saw the MMAs complete, 5 partial sums sent
+ *     to the partner block, 6 partner's partial sums received, 7 cell update
+ *     done, 8 h_t published, 10 Gx of this step loaded into the accumulator
+ *     (stamped at the end of the previous step).
+ * Process-wide; tracing adds one timer read and store per event to block 0.
+ */
+#define LSTM_TRACE_MAX_STEPS 512
+#define LSTM_TRACE_EVENTS 16
+enum { LSTM_TRACE_FWD_REC_FFMA = 1, LSTM_TRACE_BWD_REC_FFMA = 2, LSTM_TRACE_FWD_REC_TC = 3 };
+
+lstm_status lstm_trace_enable(int enable);
+int lstm_trace_read(unsigned long long* out, int max_steps, int* kind);
+
 #ifdef __cplusplus
 }
 #endif

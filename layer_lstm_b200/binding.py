@@ -23,8 +23,13 @@ LSTM_BF16 = 1
 
 EXPORTED = ("lstm_workspace_size", "lstm_reserve_size", "lstm_forward", "lstm_backward",
             "lstm_query_status", "lstm_status_string", "lstm_timing_enable", "lstm_timing_read",
-            "lstm_timing_reset", "lstm_forward_noalloc")
+            "lstm_timing_reset", "lstm_forward_noalloc", "lstm_trace_enable", "lstm_trace_read")
 LSTM_NOALLOC_SCRATCH_BYTES = 32 << 20
+LSTM_TRACE_MAX_STEPS = 512
+LSTM_TRACE_EVENTS = 16
+LSTM_TRACE_FWD_REC_FFMA = 1
+LSTM_TRACE_BWD_REC_FFMA = 2
+LSTM_TRACE_FWD_REC_TC = 3
 
 
 class lstm_kernel_time(ctypes.Structure):
@@ -95,6 +100,10 @@ def load(build_if_stale: bool = True):
     lib.lstm_timing_reset.restype = None
     lib.lstm_forward_noalloc.argtypes = [dp, vp, vp, vp, vpp, vpp, vpp, vpp, vp, vp, vp, vp]
     lib.lstm_forward_noalloc.restype = ctypes.c_int
+    lib.lstm_trace_enable.argtypes = [ctypes.c_int]
+    lib.lstm_trace_enable.restype = ctypes.c_int
+    lib.lstm_trace_read.argtypes = [ctypes.POINTER(ctypes.c_ulonglong), ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
+    lib.lstm_trace_read.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -195,6 +204,23 @@ def lstm_timing_read() -> dict:
     if got < 0:
         raise LstmError(LSTM_ERR_CUDA, "lstm_timing_read")
     return {arr[i].name.decode(): (int(arr[i].launches), float(arr[i].total_ms)) for i in range(got)}
+
+
+def lstm_trace_enable(enable: bool) -> int:
+    return int(load().lstm_trace_enable(int(bool(enable))))
+
+
+def lstm_trace_read(max_steps: int = LSTM_TRACE_MAX_STEPS):
+    """(kind, rows): rows is a list of LSTM_TRACE_EVENTS-long lists of
+    %globaltimer stamps (ns) of the last traced recurrent launch."""
+    lib = load()
+    buf = (ctypes.c_ulonglong * (max_steps * LSTM_TRACE_EVENTS))()
+    kind = ctypes.c_int(0)
+    n = lib.lstm_trace_read(buf, max_steps, ctypes.byref(kind))
+    if n < 0:
+        raise LstmError(LSTM_ERR_CUDA, "lstm_trace_read")
+    rows = [list(buf[i * LSTM_TRACE_EVENTS:(i + 1) * LSTM_TRACE_EVENTS]) for i in range(n)]
+    return int(kind.value), rows
 
 
 def check(status: int, where: str = "lstm") -> None:

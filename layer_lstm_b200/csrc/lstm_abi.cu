@@ -269,11 +269,62 @@ size_t forward_workspace_prefix(const lstm_desc* desc) {
     return l.seq[1] + al((size_t)l.T * l.B * l.D * l.H * l.es);
 }
 
+static_assert(kTraceSteps == LSTM_TRACE_MAX_STEPS && kTraceEvents == LSTM_TRACE_EVENTS,
+              "trace buffer shape differs from the header");
+
+// Per-step timeline of block 0 of the last traced recurrent launch
+// (instrumentation, off unless lstm_trace_enable(1)).
+__device__ unsigned long long g_trace[kTraceSteps * kTraceEvents];
+
+struct TraceState {
+    std::mutex mu;
+    bool on = false;
+    int kind = 0, steps = 0;   // last traced launch
+};
+
+TraceState& trace_state() {
+    static TraceState t;
+    return t;
+}
+
+// Trace buffer for a recurrent launch of `kind` (LSTM_TRACE_*) over `steps`
+// steps, zeroed on the stream; null when tracing is off.
+unsigned long long* trace_for(int kind, int steps, cudaStream_t s) {
+    TraceState& ts = trace_state();
+    std::lock_guard<std::mutex> lk(ts.mu);
+    if (!ts.on) return nullptr;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_trace) != cudaSuccess) return nullptr;
+    if (cudaMemsetAsync(p, 0, sizeof(unsigned long long) * kTraceSteps * kTraceEvents, s) != cudaSuccess)
+        return nullptr;
+    ts.kind = kind;
+    ts.steps = std::min(steps, kTraceSteps);
+    return static_cast<unsigned long long*>(p);
+}
+
 }  // namespace lstm
 
 using namespace lstm;
 
 extern "C" {
+
+lstm_status lstm_trace_enable(int enable) {
+    TraceState& ts = trace_state();
+    std::lock_guard<std::mutex> lk(ts.mu);
+    ts.on = enable != 0;
+    return LSTM_OK;
+}
+
+int lstm_trace_read(unsigned long long* out, int max_steps, int* kind) {
+    TraceState& ts = trace_state();
+    std::lock_guard<std::mutex> lk(ts.mu);
+    if (kind) *kind = ts.kind;
+    if (!out || max_steps <= 0 || ts.kind == 0) return 0;
+    const int n = std::min(max_steps, ts.steps);
+    if (cudaMemcpyFromSymbol(out, g_trace, sizeof(unsigned long long) * (size_t)n * kTraceEvents) != cudaSuccess)
+        return -1;
+    return n;
+}
 
 size_t lstm_workspace_size(const lstm_desc* desc) {
     Layout l;
@@ -466,6 +517,7 @@ lstm_status lstm_forward(const lstm_desc* desc, const void* x, const void* h0, c
             tr.ctr = reinterpret_cast<unsigned*>(P(workspace, l.ctr_tc)) + (size_t)k * D * l.tcr.nbg * 32;
             tr.status = status;
             tr.timeout_ns = timeout_ns();
+            tr.trace = trace_for(LSTM_TRACE_FWD_REC_TC, T, stream);
             LSTM_CUDA(timed(K_FWD_REC_TC, stream, [&] { return launch_tc_rec(tr, stream); }));
             layer_in = hseq_tc;
             continue;
@@ -500,6 +552,7 @@ lstm_status lstm_forward(const lstm_desc* desc, const void* x, const void* h0, c
         f.ctr = reinterpret_cast<unsigned*>(P(workspace, l.ctr_f)) + (size_t)k * D * l.nbg_ctr;
         f.status = status;
         f.timeout_ns = timeout_ns();
+        f.trace = trace_for(LSTM_TRACE_FWD_REC_FFMA, T, stream);
         LSTM_CUDA(timed(K_FWD_REC_FFMA, stream, [&] { return launch_fwd_rec(f, stream); }));
         layer_in = hseq;
     }
@@ -602,6 +655,7 @@ lstm_status lstm_backward(const lstm_desc* desc, const void* x, const void* h0, 
         b.ctr = reinterpret_cast<unsigned*>(P(workspace, l.ctr_b)) + (size_t)k * D * l.bwd.nbg;
         b.status = status;
         b.timeout_ns = timeout_ns();
+        b.trace = trace_for(LSTM_TRACE_BWD_REC_FFMA, T, stream);
         LSTM_CUDA(timed(K_BWD_REC_FFMA, stream, [&] { return launch_bwd_rec(b, stream); }));
 
         if (desc->bias) {

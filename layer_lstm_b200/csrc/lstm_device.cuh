@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "lstm_internal.h"
+
 namespace lstm {
 
 // Kernel-side status codes written to the workspace status word; the values
@@ -63,6 +65,12 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
+}
+
+// Per-step timeline (instrumentation): the calling thread stamps event e of
+// step s when tracing is on (trace non-null) and `who` holds.
+__device__ __forceinline__ void trace_mark(unsigned long long* trace, bool who, int s, int e) {
+    if (trace != nullptr && who && s < kTraceSteps) trace[(size_t)s * kTraceEvents + e] = globaltimer_ns();
 }
 
 // Block-wide arrival on a counter: every thread's prior global writes are

@@ -10,6 +10,12 @@ namespace lstm {
 
 enum class DType : int { F32 = 0, BF16 = 1 };
 
+// Per-step timeline of block 0 of a recurrent kernel (instrumentation):
+// trace[s * kTraceEvents + e] = %globaltimer (ns) when event e of step s
+// happened; a null trace pointer records nothing.
+constexpr int kTraceSteps = 512;
+constexpr int kTraceEvents = 16;
+
 inline size_t dtype_size(DType t) { return t == DType::F32 ? 4 : 2; }
 
 // ---------------------------------------------------------------- GEMM
@@ -125,6 +131,7 @@ struct FwdRecArgs {
     unsigned* ctr;              // [D*nbg] arrival counters, zero on entry
     int* status;
     uint64_t timeout_ns;
+    unsigned long long* trace;  // [kTraceSteps][kTraceEvents] or null
 };
 cudaError_t launch_fwd_rec(const FwdRecArgs& a, cudaStream_t s);
 RecPlan plan_fwd_rec(int H, int B, int D, DType dt, int num_sms, size_t smem_max);
@@ -152,6 +159,7 @@ struct TcRecArgs {
     unsigned* ctr;              // [D][nbg] group counters, 32 words apart, zeroed
     int* status;
     uint64_t timeout_ns;
+    unsigned long long* trace;  // [kTraceSteps][kTraceEvents] or null
 };
 cudaError_t launch_tc_rec(const TcRecArgs& a, cudaStream_t s);
 
@@ -172,6 +180,7 @@ struct BwdRecArgs {
     unsigned* ctr;
     int* status;
     uint64_t timeout_ns;
+    unsigned long long* trace;  // [kTraceSteps][kTraceEvents] or null
 };
 cudaError_t launch_bwd_rec(const BwdRecArgs& a, cudaStream_t s);
 RecPlan plan_bwd_rec(int H, int B, int D, int num_sms, size_t smem_max);

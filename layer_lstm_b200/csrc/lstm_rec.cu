@@ -213,6 +213,7 @@ __global__ void __launch_bounds__(kRecThreads, 1) fwd_rec_kernel(FwdRecArgs a) {
                       ((reinterpret_cast<uintptr_t>(hT) & 15) == 0);
     uint32_t hphase = 0;
     const int np0 = nU * min(Bs, nB);
+    const bool tr0 = blockIdx.x == 0 && tid == 0;   // the traced thread
     auto store_red = [&](int ks, int r0, int n0, float (&acc)[4][4]) {
         float* rp = red + ((size_t)ks * R + r0) * Bs + n0;
 #pragma unroll
@@ -237,9 +238,11 @@ __global__ void __launch_bounds__(kRecThreads, 1) fwd_rec_kernel(FwdRecArgs a) {
                     a.gx + ((size_t)t * B + b0 + bl) * (size_t)(D * G) + (size_t)d * G + 4 * (u0 + ul));
             }
         }
+        trace_mark(a.trace, tr0, s, 0);
         if (s > 0 && p.nu > 1) {
             if (!block_wait_geq(ctr, (unsigned)(p.nu * s), a.status, a.timeout_ns)) return;
         }
+        trace_mark(a.trace, tr0, s, 1);
         for (int bs0 = 0; bs0 < nB; bs0 += Bs) {
             const int nb = min(Bs, nB - bs0);
             if (s == 0) {
@@ -265,8 +268,10 @@ __global__ void __launch_bounds__(kRecThreads, 1) fwd_rec_kernel(FwdRecArgs a) {
                 copy_tile(hs, Hp, Bs, hT_grp + ((size_t)d * T + tp) * hT_tstride + bs0, (size_t)p.Bg, H, nb);
             }
             __syncthreads();
+            if (bs0 == 0) trace_mark(a.trace, tr0, s, 2);
             block_mm(Ws, R, hs, Bs, R, Bs, Hp, KS, store_red);
             __syncthreads();
+            if (bs0 == 0) trace_mark(a.trace, tr0, s, 3);
             for (int i = tid, q = 0; i < nU * nb; i += nth, ++q) {
                 const int bl = i % nb, ul = i / nb;
                 const int b = b0 + bs0 + bl, u = u0 + ul;
@@ -308,10 +313,12 @@ __global__ void __launch_bounds__(kRecThreads, 1) fwd_rec_kernel(FwdRecArgs a) {
             }
             __syncthreads();
         }
+        trace_mark(a.trace, tr0, s, 4);
         if (p.nu > 1 && s + 1 < T) {
             if (bulk) tc::fence_proxy_async_global();   // h_t is read by bulk copies
             block_arrive(ctr);
         }
+        trace_mark(a.trace, tr0, s, 5);
     }
 }
 
@@ -421,6 +428,7 @@ __global__ void __launch_bounds__(kRecThreads, 1) bwd_rec_kernel(BwdRecArgs a) {
 
     const int nb0 = min(Bs, nB);
     const int np0 = nU * nb0;
+    const bool tr0 = blockIdx.x == 0 && tid == 0;   // the traced thread
     for (int s = 0; s < T; ++s) {
         const int t = d == 0 ? T - 1 - s : s;
         BwdPre pre[2];
@@ -429,10 +437,13 @@ __global__ void __launch_bounds__(kRecThreads, 1) bwd_rec_kernel(BwdRecArgs a) {
             const int i = tid + q * nth;
             if (i < np0) pre[q] = bwd_fetch(a, d, t, b0 + i % nb0, j0 + i / nb0);
         }
+        trace_mark(a.trace, tr0, s, 0);
         if (s > 0) {
             if (p.nu > 1 && !block_wait_geq(ctr, (unsigned)(p.nu * s), a.status, a.timeout_ns)) return;
+            trace_mark(a.trace, tr0, s, 1);
             gather((s - 1) & 1);
         }
+        trace_mark(a.trace, tr0, s, 2);
         for (int bs0 = 0; bs0 < nB; bs0 += Bs) {
             const int nb = min(Bs, nB - bs0);
             for (int i = tid, q = 0; i < U * Bs; i += nth, ++q) {
@@ -472,6 +483,7 @@ __global__ void __launch_bounds__(kRecThreads, 1) bwd_rec_kernel(BwdRecArgs a) {
                 dba[(size_t)3 * U * Bg] += da_o;
             }
             __syncthreads();
+            if (bs0 == 0) trace_mark(a.trace, tr0, s, 3);
             // partial dh_{t-1}[b][0..Hp) from this block's 4U gate rows
             float* Pw = Pblk(s & 1, j) + (size_t)bs0 * Hp;
             auto store_p = [&](int, int r0, int n0, float (&acc)[4][4]) {
@@ -485,8 +497,10 @@ __global__ void __launch_bounds__(kRecThreads, 1) bwd_rec_kernel(BwdRecArgs a) {
             block_mm(Wr, Hp, daT, Bs, Hp, Bs, R4, 1, store_p);
             __syncthreads();
         }
+        trace_mark(a.trace, tr0, s, 4);
         if (p.nu > 1) block_arrive(ctr);
         else __syncthreads();
+        trace_mark(a.trace, tr0, s, 5);
     }
     if (T > 0) {
         if (p.nu > 1 && !block_wait_geq(ctr, (unsigned)(p.nu * T), a.status, a.timeout_ns)) return;

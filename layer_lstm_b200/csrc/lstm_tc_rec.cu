@@ -66,6 +66,7 @@ struct TcRecParams {
     unsigned* ctr;            // [D][nbg] group counters, kCtrStride apart
     int* status;
     uint64_t timeout_ns;
+    unsigned long long* trace;   // per-step timeline of block 0, or null
 };
 
 // Branch-free choice among four registers by a lane-dependent index k in
@@ -271,6 +272,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const bool tr0 = blockIdx.x == 0 && lane == 0;             // traced lane of warps 0 and 1
+    const bool tr2 = blockIdx.x == 0 && warp == 2 && lane == 0;   // traced epilogue thread
     const int cl = blockIdx.x >> 1;                    // cluster index; rank == blockIdx.x & 1
     const int j = cl % a.nu;
     const int bg = (cl / a.nu) % a.nbg;
@@ -355,6 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!ctr_wait(ctr, (unsigned)(2 * a.nu * s), abort_flag, a.status, a.timeout_ns)) break;
                     tc::fence_proxy_async_global();
                 }
+                trace_mark(a.trace, tr0, s, 0);
                 const int row0 = (d * (T + 1) + s) * B + b0;
                 for (int i = 0; i < nch; ++i) {
                     const int c = rot + i < nch ? rot + i : rot + i - nch;
@@ -367,6 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc::tma_load_2d(sH + st * hstage, &tmH, 64 * (c_beg + c), row0, &full[st]);
                     ++issued;
                 }
+                trace_mark(a.trace, tr0, s, 1);
             }
             if (*abort_flag) {
                 for (int idx = issued > S ? issued - S : 0; idx < issued; ++idx)
@@ -382,6 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int s = 0; s < T && ok; ++s) {
                 if (!tc::mbar_wait(d_ready, s & 1, abort_flag, a.status, a.timeout_ns)) break;
                 tc::tc_fence_after();
+                trace_mark(a.trace, tr0, s, 2);
                 for (int i = 0; i < nch; ++i) {
                     const int idx = s * nch + i, st = idx % S, rnd = idx / S;
                     if (!tc::mbar_wait(&full[st], rnd & 1, abort_flag, a.status, a.timeout_ns)) {
@@ -390,6 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     tc::tc_fence_after();
                     const int c = rot + i < nch ? rot + i : rot + i - nch;
+                    if (i == 0) trace_mark(a.trace, tr0, s, 9);
                     const uint32_t b_base = tc::smem_u32(sH + st * hstage);
 #pragma unroll
                     for (int jj = 0; jj < 4; ++jj) {
@@ -407,6 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (!ok) break;
                 tc::mma_commit(mma_done);
+                trace_mark(a.trace, tr0, s, 3);
             }
             if (*abort_flag && last >= 0) drain_wait(&empty[last % S], (last / S) & 1);
         }
@@ -441,6 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool ok = tc::mbar_wait(mma_done, s & 1, abort_flag, a.status, a.timeout_ns);
             if (named_bar_or(1, kEpi, !ok)) break;   // every epilogue thread leaves together
             tc::tc_fence_after();
+            trace_mark(a.trace, tr2, s, 4);
             // 1) this block's partial sums of the partner's columns -> partner,
             //    two 16-column chunks at a time
 #pragma unroll
@@ -464,9 +473,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             mbar_arrive_remote(recv_bar_remote);
+            trace_mark(a.trace, tr2, s, 5);
             // 2) the partner's partial sums of the own columns
             const bool got = mbar_wait_cluster(recv_full, s & 1, abort_flag, a.status, a.timeout_ns);
             if (named_bar_or(1, kEpi, !got)) break;
+            trace_mark(a.trace, tr2, s, 6);
             // 3) gates, cell update and h for the own columns, two chunks at a time
 #pragma unroll
             for (int k0 = 0; k0 < kCcPerHalf; k0 += 2) {
@@ -524,6 +535,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
+            trace_mark(a.trace, tr2, s, 7);
             // 4) h_t of the own columns to global memory in 16-byte pieces
             //    (32 units of a column are 64 contiguous bytes), publish it
             //    to the group, then hand the accumulator Gx[t+1]
@@ -556,9 +568,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __threadfence();
                 atomicAdd(ctr, 1u);
             }
-            if (s + 1 < T)
+            trace_mark(a.trace, tr2, s, 8);
+            if (s + 1 < T) {
                 preload_gx(a.gx, d == 0 ? s + 1 : T - 2 - s, B, ldgx, prow0 + r, b0, own0, pcol0, ncc, nB, half, trow,
                            d_ready);
+                trace_mark(a.trace, tr2, s + 1, 10);
+            }
         }
     }
     tc::tc_fence_before();
@@ -644,6 +659,7 @@ cudaError_t launch_tc_rec(const TcRecArgs& a, cudaStream_t s) {
     prm.out_vec = (reinterpret_cast<uintptr_t>(a.out) & 15) == 0;
     prm.h_n = static_cast<bf16*>(a.h_n); prm.c_n = a.c_n;
     prm.wpk = static_cast<const bf16*>(a.wpk);
+    prm.trace = a.trace;
     prm.ctr = a.ctr; prm.status = a.status; prm.timeout_ns = a.timeout_ns;
     cudaError_t e = cudaFuncSetAttribute(tc_rec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
     if (e != cudaSuccess) return e;
