@@ -38,16 +38,23 @@ __device__ __forceinline__ size_t align16(size_t x) { return (x + 15) & ~size_t(
 inline size_t align16h(size_t x) { return (x + 15) & ~size_t(15); }
 
 // C[r][n] = sum_k A[k*lda + r] * X[k*ldx + n] for r < R, n < N, k < K, with
-// R, N, K multiples of 4.  Each thread computes a 4 x 4 tile over one of KS
-// K-slices and hands it to st(ks, r0, n0, acc).  Lanes of a warp cover an
-// 8 x 4 block of tiles of the same K-slice, so every shared-memory load of a
-// warp touches at most 128 contiguous bytes of A and of X.
-template <typename AT, typename XT, typename St>
+// R and K multiples of 4 and N a multiple of TN (4 or 8).  Each thread
+// computes a 4 x TN register tile over one of KS K-slices and hands it to
+// st(ks, r0, n0, acc).  Lanes of a warp cover a wr x wn block of tiles of
+// the same K-slice (wn tile columns, at most 128 contiguous bytes of X per
+// load; wr = 32 / wn tile rows, contiguous in A), so shared-memory loads of
+// a warp touch few wavefronts and no lane is idle while tiles remain.
+template <int TN>
+__host__ __device__ constexpr int tile_cols_wn(int nNT) {
+    return nNT >= 128 / (4 * TN) ? 128 / (4 * TN) : (nNT >= 4 ? 4 : (nNT >= 2 ? 2 : 1));
+}
+
+template <int TN, typename AT, typename XT, typename St>
 __device__ __forceinline__ void block_mm(const AT* __restrict__ A, int lda, const XT* __restrict__ X,
                                          int ldx, int R, int N, int K, int KS, St&& st) {
-    const int nRT = R >> 2, nNT = N >> 2;
-    const int wr = nRT >= 8 ? 8 : (nRT >= 4 ? 4 : (nRT >= 2 ? 2 : 1));
-    const int wn = 32 / wr;
+    const int nRT = R >> 2, nNT = N / TN;
+    const int wn = tile_cols_wn<TN>(nNT);
+    const int wr = 32 / wn;
     const int nRB = (nRT + wr - 1) / wr, nNB = (nNT + wn - 1) / wn;
     const int nblk = nRB * nNB;
     const int KL = (((K >> 2) + KS - 1) / KS) << 2;
@@ -59,29 +66,35 @@ __device__ __forceinline__ void block_mm(const AT* __restrict__ A, int lda, cons
         const int nt = (blk / nRB) * wn + lane / wr;
         if (rt >= nRT || nt >= nNT) continue;
         const int k0 = ks * KL, k1 = min(K, k0 + KL);
-        float acc[4][4];
+        float acc[4][TN];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+            for (int j = 0; j < TN; ++j) acc[i][j] = 0.f;
         const AT* ap = A + rt * 4;
-        const XT* xp = X + nt * 4;
+        const XT* xp = X + nt * TN;
 #pragma unroll 2
         for (int k = k0; k < k1; k += 4) {
-            float a[4][4], x[4][4];
+            float a[4][4], x[4][TN];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 load4(ap + (size_t)(k + q) * lda, a[q]);
-                load4(xp + (size_t)(k + q) * ldx, x[q]);
+#pragma unroll
+                for (int h = 0; h < TN; h += 4) {
+                    float t4[4];
+                    load4(xp + (size_t)(k + q) * ldx + h, t4);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) x[q][h + e] = t4[e];
+                }
             }
 #pragma unroll
             for (int q = 0; q < 4; ++q)
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[q][i], x[q][j], acc[i][j]);
+                    for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(a[q][i], x[q][j], acc[i][j]);
         }
-        st(ks, rt * 4, nt * 4, acc);
+        st(ks, rt * 4, nt * TN, acc);
     }
 }
 
@@ -146,8 +159,11 @@ __device__ __forceinline__ void copy_tile(T* __restrict__ dst, int nrows, int nc
 
 constexpr int kRecThreads = 256;   // threads per recurrent block
 
+// Column-tile width of the block_mm calls on an N-column operand.
+__host__ __device__ constexpr int rec_tn(int N) { return N % 8 == 0 ? 8 : 4; }
+
 inline int pick_ks(int R, int N, int K) {
-    const int nT = (R / 4) * (N / 4);
+    const int nT = (R / 4) * (N / rec_tn(N));
     int ks = 1;
     while (nT * ks * 2 <= kRecThreads && K / (ks * 2) >= 16) ks *= 2;
     return ks;
@@ -214,12 +230,15 @@ __global__ void __launch_bounds__(kRecThreads, 1) fwd_rec_kernel(FwdRecArgs a) {
     uint32_t hphase = 0;
     const int np0 = nU * min(Bs, nB);
     const bool tr0 = blockIdx.x == 0 && tid == 0;   // the traced thread
-    auto store_red = [&](int ks, int r0, int n0, float (&acc)[4][4]) {
+    auto store_red = [&](int ks, int r0, int n0, auto& acc) {
+        constexpr int tn = sizeof(acc[0]) / sizeof(float);
         float* rp = red + ((size_t)ks * R + r0) * Bs + n0;
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-            *reinterpret_cast<float4*>(rp + (size_t)i * Bs) =
-                make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+#pragma unroll
+            for (int h = 0; h < tn; h += 4)
+                *reinterpret_cast<float4*>(rp + (size_t)i * Bs + h) =
+                    make_float4(acc[i][h], acc[i][h + 1], acc[i][h + 2], acc[i][h + 3]);
     };
     for (int s = 0; s < T; ++s) {
         const int t = d == 0 ? s : T - 1 - s;
@@ -269,7 +288,10 @@ __global__ void __launch_bounds__(kRecThreads, 1) fwd_rec_kernel(FwdRecArgs a) {
             }
             __syncthreads();
             if (bs0 == 0) trace_mark(a.trace, tr0, s, 2);
-            block_mm(Ws, R, hs, Bs, R, Bs, Hp, KS, store_red);
+            if (rec_tn(Bs) == 8)
+                block_mm<8>(Ws, R, hs, Bs, R, Bs, Hp, KS, store_red);
+            else
+                block_mm<4>(Ws, R, hs, Bs, R, Bs, Hp, KS, store_red);
             __syncthreads();
             if (bs0 == 0) trace_mark(a.trace, tr0, s, 3);
             for (int i = tid, q = 0; i < nU * nb; i += nth, ++q) {
@@ -486,15 +508,19 @@ __global__ void __launch_bounds__(kRecThreads, 1) bwd_rec_kernel(BwdRecArgs a) {
             if (bs0 == 0) trace_mark(a.trace, tr0, s, 3);
             // partial dh_{t-1}[b][0..Hp) from this block's 4U gate rows
             float* Pw = Pblk(s & 1, j) + (size_t)bs0 * Hp;
-            auto store_p = [&](int, int r0, int n0, float (&acc)[4][4]) {
+            auto store_p = [&](int, int r0, int n0, auto& acc) {
+                constexpr int tn = sizeof(acc[0]) / sizeof(float);
 #pragma unroll
-                for (int jn = 0; jn < 4; ++jn) {
+                for (int jn = 0; jn < tn; ++jn) {
                     if (n0 + jn < nb)
                         *reinterpret_cast<float4*>(Pw + (size_t)(n0 + jn) * Hp + r0) =
                             make_float4(acc[0][jn], acc[1][jn], acc[2][jn], acc[3][jn]);
                 }
             };
-            block_mm(Wr, Hp, daT, Bs, Hp, Bs, R4, 1, store_p);
+            if (rec_tn(Bs) == 8)
+                block_mm<8>(Wr, Hp, daT, Bs, Hp, Bs, R4, 1, store_p);
+            else
+                block_mm<4>(Wr, Hp, daT, Bs, Hp, Bs, R4, 1, store_p);
             __syncthreads();
         }
         trace_mark(a.trace, tr0, s, 4);
