@@ -129,8 +129,11 @@ lstm_status lstm_forward(const lstm_desc* desc, const void* x, const void* h0, c
  *   dw_ih, dw_hh, db_ih, db_hh: host arrays of L*D device pointers to float32
  *     gradients, OVERWRITTEN (not accumulated); db arrays ignored if !bias.
  *     db_ih and db_hh receive the same values (the biases enter as a sum).
- * Only desc->dtype == LSTM_F32 is implemented; bf16 returns
- * LSTM_ERR_UNSUPPORTED.
+ * Both dtypes compute in float32.  For LSTM_BF16, x, h0, weights, grad_out,
+ * grad_hn and the saved layer outputs are widened to float32 copies in the
+ * workspace, and dx and dh0 are rounded to bf16 (nearest even) at the end;
+ * the weight and bias gradients stay float32.  LSTM_ERR_UNSUPPORTED only
+ * when no recurrent plan fits the device.
  */
 lstm_status lstm_backward(const lstm_desc* desc, const void* x, const void* h0, const float* c0,
                           const void* const* w_ih, const void* const* w_hh,

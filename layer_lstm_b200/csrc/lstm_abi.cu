@@ -152,6 +152,8 @@ struct Layout {
     // workspace offsets
     size_t status, ctr_f, ctr_b, ctr_tc, ctr_end, wih[32], bias[32], whh_f, whh_b, gx, hT, seq[2], dG, dseq[2], xt,
         dbpart, P, dGT, bop, wcatT, hx, whh_tc, bias_dummy, total;
+    // bf16 backward: float32 staging of what it reads and writes
+    size_t s_x, s_h0, s_gout, s_ghn, s_hs[2], s_dx, s_dh0, s_wih[32];
     // reserve offsets
     size_t act[32], cst[32], hseq[32], rtotal;   // per layer: [D][T][B][G], [D][T][B][H], [T][B][D*H]
 };
@@ -192,7 +194,7 @@ bool make_layout(const lstm_desc* d, Layout& l) {
     const int Bp = l.B > 0 ? l.B : 1;
     l.fwd = plan_fwd_rec(l.H, Bp, l.D, l.dt, dev.sms, smem_max);
     if (l.fwd.ctas == 0) return false;
-    l.bwd = plan_bwd_rec(l.H, Bp, l.D, dev.sms, smem_max);
+    l.bwd = plan_bwd_rec(l.H, Bp, l.D, l.dt, dev.sms, smem_max);
     l.bwd_ok = l.bwd.ctas > 0;
     l.tcr = l.dt == DType::BF16 ? plan_tc_rec(l.H, Bp, l.D, dev.sms, smem_max) : TcRecPlan{};
     const size_t TB = (size_t)l.T * l.B;
@@ -211,7 +213,7 @@ bool make_layout(const lstm_desc* d, Layout& l) {
     }
     l.whh_f = o; o += al((size_t)l.D * l.fwd.nu * ((l.H + 3) & ~3) * 4 * l.fwd.U * l.es);
     const size_t Hp = (size_t)((l.H + 3) & ~3);
-    l.whh_b = o; o += al(l.bwd_ok ? (size_t)l.D * l.bwd.nu * 4 * l.bwd.U * Hp * 4 : 0);
+    l.whh_b = o; o += al(l.bwd_ok ? (size_t)l.D * l.bwd.nu * 4 * l.bwd.U * Hp * l.es : 0);
     l.gx = o; o += al(TB * l.D * l.G * 4);
     l.hT = o; o += al((size_t)l.T * l.D * l.fwd.nbg * l.fwd.Bg * l.H * l.es);   // [D][T][nbg][H][Bg]
     l.seq[0] = o; o += al(TB * l.D * l.H * l.es);
@@ -223,19 +225,30 @@ bool make_layout(const lstm_desc* d, Layout& l) {
     } else {
         l.hx = l.whh_tc = l.bias_dummy = 0;
     }
+    // backward (float32 arithmetic for both dtypes)
     const size_t maxin = (size_t)(l.I > l.D * l.H ? l.I : l.D * l.H);
-    if (l.dt == DType::F32) {
-        l.dG = o; o += al(TB * l.D * l.G * 4);
-        l.dseq[0] = o; o += al(TB * maxin * 4);
-        l.dseq[1] = o; o += al(TB * maxin * 4);
-        l.xt = o; o += al(TB * l.I * 4);
-        l.dbpart = o; o += al((size_t)l.D * (l.bwd_ok ? l.bwd.nbg : 1) * l.G * 4);
-        l.P = o; o += al(l.bwd_ok ? (size_t)2 * l.D * l.bwd.nbg * l.bwd.nu * l.bwd.Bg * Hp * 4 : 0);
-        l.dGT = o; o += al(TB * l.D * l.G * 4);
-        l.bop = o; o += al((size_t)l.D * (maxin + l.H) * TB * 4);
-        l.wcatT = o; o += al(maxin * l.D * l.G * 4);
-    } else {
-        l.dG = l.dseq[0] = l.dseq[1] = l.xt = l.dbpart = l.P = l.dGT = l.bop = l.wcatT = 0;
+    l.dG = o; o += al(TB * l.D * l.G * 4);
+    l.dseq[0] = o; o += al(TB * maxin * 4);
+    l.dseq[1] = o; o += al(TB * maxin * 4);
+    l.xt = o; o += al(TB * l.I * 4);
+    l.dbpart = o; o += al((size_t)l.D * (l.bwd_ok ? l.bwd.nbg : 1) * l.G * 4);
+    l.P = o; o += al(l.bwd_ok ? (size_t)2 * l.D * l.bwd.nbg * l.bwd.nu * l.bwd.Bg * Hp * 4 : 0);
+    l.dGT = o; o += al(TB * l.D * l.G * 4);
+    l.bop = o; o += al((size_t)l.D * (maxin + l.H) * TB * 4);
+    l.wcatT = o; o += al(maxin * l.D * l.G * 4);
+    if (l.dt == DType::BF16) {
+        const size_t states = (size_t)l.L * l.D * l.B * l.H;
+        l.s_x = o; o += al(TB * l.I * 4);
+        l.s_h0 = o; o += al(states * 4);
+        l.s_gout = o; o += al(TB * l.D * l.H * 4);
+        l.s_ghn = o; o += al(states * 4);
+        l.s_hs[0] = o; o += al(TB * l.D * l.H * 4);
+        l.s_hs[1] = o; o += al(TB * l.D * l.H * 4);
+        l.s_dx = o; o += al(TB * l.I * 4);
+        l.s_dh0 = o; o += al(states * 4);
+        for (int k = 0; k < l.L; ++k) {
+            l.s_wih[k] = o; o += al((size_t)l.D * l.G * in_size(l, k) * 4);
+        }
     }
     l.total = o;
     size_t r = 0;
@@ -580,7 +593,6 @@ lstm_status lstm_backward(const lstm_desc* desc, const void* x, const void* h0, 
     if (!workspace) return LSTM_ERR_INVALID_ARG;
     if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return LSTM_ERR_INVALID_ARG;
     if (reserve && reinterpret_cast<uintptr_t>(reserve) % 256 != 0) return LSTM_ERR_INVALID_ARG;
-    if (desc->dtype != LSTM_F32) return LSTM_ERR_UNSUPPORTED;
     Layout l;
     if (!make_layout(desc, l)) return LSTM_ERR_UNSUPPORTED;
     if (!l.bwd_ok) return LSTM_ERR_UNSUPPORTED;
@@ -608,25 +620,63 @@ lstm_status lstm_backward(const lstm_desc* desc, const void* x, const void* h0, 
     if (B == 0) return LSTM_OK;
     if (T == 0) {
         const size_t n = (size_t)L * state;
-        if (grad_hn) LSTM_CUDA(cudaMemcpyAsync(dh0, grad_hn, n * 4, cudaMemcpyDeviceToDevice, stream));
-        else LSTM_CUDA(cudaMemsetAsync(dh0, 0, n * 4, stream));
+        if (grad_hn) LSTM_CUDA(cudaMemcpyAsync(dh0, grad_hn, n * l.es, cudaMemcpyDeviceToDevice, stream));
+        else LSTM_CUDA(cudaMemsetAsync(dh0, 0, n * l.es, stream));
         if (grad_cn) LSTM_CUDA(cudaMemcpyAsync(dc0, grad_cn, n * 4, cudaMemcpyDeviceToDevice, stream));
         else LSTM_CUDA(cudaMemsetAsync(dc0, 0, n * 4, stream));
         return LSTM_OK;
     }
     int* status = reinterpret_cast<int*>(P(workspace, l.status));
     float* dG = reinterpret_cast<float*>(P(workspace, l.dG));
+    // Everything below computes in float32.  A bf16 problem reads float32
+    // copies of its bf16 inputs (x, h0, weights, grad_out, grad_hn and the
+    // saved layer outputs) and writes dx and dh0 through float32 staging.
+    const bool bf = l.dt == DType::BF16;
+    auto stage = [&](const void* src, size_t off, size_t n) -> const float* {
+        if (!src) return nullptr;
+        if (!bf) return static_cast<const float*>(src);
+        float* dst = reinterpret_cast<float*>(P(workspace, off));
+        const cudaError_t e = launch_convert(src, DType::BF16, dst, DType::F32, (long long)n, stream);
+        return e == cudaSuccess ? dst : nullptr;
+    };
+    const size_t BTs = (size_t)B * T;
+    const float* xf = stage(x, l.s_x, BTs * l.I);
+    const float* h0f = stage(h0, l.s_h0, (size_t)L * state);
+    const float* goutf = stage(grad_out, l.s_gout, BTs * D * H);
+    const float* ghnf = stage(grad_hn, l.s_ghn, (size_t)L * state);
+    if (!xf || !goutf || (h0 && !h0f) || (grad_hn && !ghnf)) return LSTM_ERR_CUDA;
+    std::vector<const float*> wihf(L * D);   // W_hh stays in its own type (resident rows)
+    for (int k = 0; k < L; ++k)
+        for (int d = 0; d < D; ++d) {
+            const int i = k * D + d;
+            const size_t nih = (size_t)G * in_size(l, k);
+            wihf[i] = stage(w_ih[i], bf ? l.s_wih[k] + (size_t)d * nih * 4 : 0, nih);
+            if (!wihf[i]) return LSTM_ERR_CUDA;
+        }
+    // float32 output sequence of layer k, saved by the forward in the reserve
+    auto layer_out = [&](int k) -> const float* {
+        const void* src = static_cast<const char*>(reserve) + l.hseq[k];
+        return bf ? reinterpret_cast<const float*>(P(workspace, l.s_hs[k & 1])) : static_cast<const float*>(src);
+    };
+    auto stage_layer_out = [&](int k) -> bool {
+        if (!bf) return true;
+        return launch_convert(static_cast<const char*>(reserve) + l.hseq[k], DType::BF16, P(workspace, l.s_hs[k & 1]),
+                              DType::F32, (long long)(BTs * D * H), stream) == cudaSuccess;
+    };
+    if (!stage_layer_out(L - 1)) return LSTM_ERR_CUDA;
+    float* dh0f = bf ? reinterpret_cast<float*>(P(workspace, l.s_dh0)) : static_cast<float*>(dh0);
+    float* dxf = bf ? reinterpret_cast<float*>(P(workspace, l.s_dx)) : static_cast<float*>(dx);
     // time-major copy of x for the layer-0 weight gradient
-    const float* x_tm = static_cast<const float*>(x);
+    const float* x_tm = xf;
     if (desc->batch_first) {
         SeqCopyArgs sc{};
         sc.T = T; sc.B = B; sc.W = l.I; sc.dt = DType::F32;
-        sc.src = x; sc.s_st = l.I; sc.s_sb = (long long)T * l.I;
+        sc.src = xf; sc.s_st = l.I; sc.s_sb = (long long)T * l.I;
         sc.dst = P(workspace, l.xt); sc.d_st = (long long)B * l.I; sc.d_sb = l.I;
         LSTM_CUDA(timed(K_COPY, stream, [&] { return launch_seq_copy(sc, stream); }));
         x_tm = reinterpret_cast<const float*>(P(workspace, l.xt));
     }
-    const float* dy = static_cast<const float*>(grad_out);
+    const float* dy = goutf;
     long long dy_st = desc->batch_first ? (long long)D * H : (long long)B * D * H;
     long long dy_sb = desc->batch_first ? (long long)T * D * H : (long long)D * H;
     int cur = 0;
@@ -634,22 +684,25 @@ lstm_status lstm_backward(const lstm_desc* desc, const void* x, const void* h0, 
         const int in = in_size(l, k);
         PackHhBwdArgs pb{};
         pb.H = H; pb.D = D; pb.nu = l.bwd.nu; pb.U = l.bwd.U;
-        for (int d = 0; d < D; ++d) pb.w[d] = static_cast<const float*>(w_hh[k * D + d]);
-        pb.out = reinterpret_cast<float*>(P(workspace, l.whh_b));
+        pb.dt = l.dt;
+        for (int d = 0; d < D; ++d) pb.w[d] = w_hh[k * D + d];
+        if (k > 0 && !stage_layer_out(k - 1)) return LSTM_ERR_CUDA;
+        pb.out = P(workspace, l.whh_b);
         LSTM_CUDA(timed(K_PACK, stream, [&] { return launch_pack_hh_rows(pb, stream); }));
 
         BwdRecArgs b{};
         b.H = H; b.B = B; b.T = T; b.D = D; b.p = l.bwd;
-        b.wr = reinterpret_cast<const float*>(P(workspace, l.whh_b));
+        b.wr = P(workspace, l.whh_b);
+        b.wdt = l.dt;
         b.P = reinterpret_cast<float*>(P(workspace, l.P));
         b.act = reinterpret_cast<const float*>(static_cast<const char*>(reserve) + l.act[k]);
         b.cst = reinterpret_cast<const float*>(static_cast<const char*>(reserve) + l.cst[k]);
         b.c0 = c0 ? c0 + (size_t)k * state : nullptr;
         b.dy = dy; b.dy_st = dy_st; b.dy_sb = dy_sb;
-        b.grad_hn = grad_hn ? static_cast<const float*>(grad_hn) + (size_t)k * state : nullptr;
+        b.grad_hn = ghnf ? ghnf + (size_t)k * state : nullptr;
         b.grad_cn = grad_cn ? grad_cn + (size_t)k * state : nullptr;
         b.dG = dG;
-        b.dh0 = static_cast<float*>(dh0) + (size_t)k * state;
+        b.dh0 = dh0f + (size_t)k * state;
         b.dc0 = dc0 + (size_t)k * state;
         b.dbpart = reinterpret_cast<float*>(P(workspace, l.dbpart));
         b.ctr = reinterpret_cast<unsigned*>(P(workspace, l.ctr_b)) + (size_t)k * D * l.bwd.nbg;
@@ -664,12 +717,11 @@ lstm_status lstm_backward(const lstm_desc* desc, const void* x, const void* h0, 
             for (int d = 0; d < D; ++d) { db.db_ih[d] = db_ih[k * D + d]; db.db_hh[d] = db_hh[k * D + d]; }
             LSTM_CUDA(timed(K_DB, stream, [&] { return launch_db_reduce(db, stream); }));
         }
-        const float* layer_in = k == 0 ? x_tm
-                                       : reinterpret_cast<const float*>(static_cast<const char*>(reserve) + l.hseq[k - 1]);
-        const float* hs = reinterpret_cast<const float*>(static_cast<const char*>(reserve) + l.hseq[k]);
+        const float* layer_in = k == 0 ? x_tm : layer_out(k - 1);
+        const float* hs = layer_out(k);
         const long long ldg = (long long)D * G, ldh = (long long)D * H;
         const long long BTl = (long long)B * T;
-        float* din = k == 0 ? static_cast<float*>(dx) : reinterpret_cast<float*>(P(workspace, l.dseq[cur]));
+        float* din = k == 0 ? dxf : reinterpret_cast<float*>(P(workspace, l.dseq[cur]));
         // Tensor-core weight phase: dW = dG^T [In | H_prev] per direction over
         // K = B*T (one GEMM writes dW_ih and dW_hh), dIn = dG [W_ih_0; W_ih_1].
         float* dGT = reinterpret_cast<float*>(P(workspace, l.dGT));
@@ -698,10 +750,10 @@ lstm_status lstm_backward(const lstm_desc* desc, const void* x, const void* h0, 
                 TransposeArgs ti{};
                 ti.M = (int)BTl; ti.C = in; ti.mode = 0;
                 if (k == 0) {
-                    ti.src = static_cast<const float*>(x); ti.lds = in;
+                    ti.src = xf; ti.lds = in;
                     ti.bt_remap = desc->batch_first; ti.T = T; ti.B = B;
                 } else {
-                    ti.src = reinterpret_cast<const float*>(static_cast<const char*>(reserve) + l.hseq[k - 1]);
+                    ti.src = layer_out(k - 1);
                     ti.lds = in;
                 }
                 ti.dst = bo; ti.ldd = BTl;
@@ -709,7 +761,7 @@ lstm_status lstm_backward(const lstm_desc* desc, const void* x, const void* h0, 
                 TransposeArgs th{};
                 th.M = (int)BTl; th.C = H; th.mode = 1;
                 th.src = hs + (size_t)d * H; th.lds = ldh; th.T = T; th.B = B; th.dir = d;
-                th.h0 = h0 ? static_cast<const float*>(h0) + ((size_t)k * D + d) * B * H : nullptr;
+                th.h0 = h0f ? h0f + ((size_t)k * D + d) * B * H : nullptr;
                 th.dst = bo + (size_t)in * BTl; th.ldd = BTl;
                 LSTM_CUDA(timed(K_TRANSPOSE, stream, [&] { return launch_transpose(th, stream); }));
                 TcGemmArgs twd = tw;
@@ -720,7 +772,7 @@ lstm_status lstm_backward(const lstm_desc* desc, const void* x, const void* h0, 
                 LSTM_CUDA(timed(K_DW_TC, stream, [&] { return launch_tc_gemm(twd, stream); }));
                 TransposeArgs tww{};
                 tww.M = G; tww.C = in; tww.mode = 0;
-                tww.src = static_cast<const float*>(w_ih[k * D + d]); tww.lds = in;
+                tww.src = wihf[k * D + d]; tww.lds = in;
                 tww.dst = wcatT + (size_t)d * G; tww.ldd = (long long)D * G;
                 LSTM_CUDA(timed(K_TRANSPOSE, stream, [&] { return launch_transpose(tww, stream); }));
             }
@@ -752,11 +804,11 @@ lstm_status lstm_backward(const lstm_desc* desc, const void* x, const void* h0, 
                 } else {
                     LSTM_CUDA(cudaMemsetAsync(dw_hh[k * D + d], 0, (size_t)G * H * 4, stream));
                 }
-                if (h0) {
+                if (h0f) {
                     GemmArgs g0 = gh;
                     g0.K = B;
                     g0.A = dG + (d == 0 ? 0 : (size_t)(T - 1) * B * ldg) + (size_t)d * G;
-                    g0.B = static_cast<const float*>(h0) + ((size_t)k * D + d) * B * H;
+                    g0.B = h0f + ((size_t)k * D + d) * B * H;
                     g0.sBk = H;
                     g0.accumulate = 1;
                     LSTM_CUDA(timed(K_DW_SIMT, stream, [&] { return launch_gemm(g0, stream); }));
@@ -767,7 +819,7 @@ lstm_status lstm_backward(const lstm_desc* desc, const void* x, const void* h0, 
                 GemmArgs g{};
                 g.M = B * T; g.N = in; g.K = G;
                 g.A = dG + (size_t)d * G; g.ta = DType::F32; g.sAm = ldg; g.sAk = 1;
-                g.B = w_ih[k * D + d]; g.tb = DType::F32; g.sBk = in; g.sBn = 1;
+                g.B = wihf[k * D + d]; g.tb = DType::F32; g.sBk = in; g.sBn = 1;
                 g.C = din; g.tc = DType::F32; g.ldc = in;
                 g.accumulate = d > 0;
                 if (k == 0 && desc->batch_first) { g.remap_T = -T; g.remap_B = B; }
@@ -780,6 +832,10 @@ lstm_status lstm_backward(const lstm_desc* desc, const void* x, const void* h0, 
             dy_sb = in;
             cur ^= 1;
         }
+    }
+    if (bf) {
+        LSTM_CUDA(launch_convert(dxf, DType::F32, dx, DType::BF16, (long long)(BTs * l.I), stream));
+        LSTM_CUDA(launch_convert(dh0f, DType::F32, dh0, DType::BF16, (long long)(L * state), stream));
     }
     (void)status;
     return LSTM_OK;

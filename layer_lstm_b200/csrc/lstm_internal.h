@@ -103,8 +103,9 @@ cudaError_t launch_pack_hh_fwd(const PackHhFwdArgs& a, cudaStream_t s);
 // W_hh[q*H + u][:], zero padded.
 struct PackHhBwdArgs {
     int H, D, nu, U;
-    const float* w[2];
-    float* out;
+    DType dt;                   // type of w and out (kept: bf16 weights stay bf16)
+    const void* w[2];
+    void* out;
 };
 cudaError_t launch_pack_hh_rows(const PackHhBwdArgs& a, cudaStream_t s);
 
@@ -166,7 +167,8 @@ cudaError_t launch_tc_rec(const TcRecArgs& a, cudaStream_t s);
 struct BwdRecArgs {
     int H, B, T, D;
     RecPlan p;
-    const float* wr;            // [D][nu*4U][Hp] W_hh rows, packed order 4u+q
+    const void* wr;             // [D][nu*4U][Hp] W_hh rows, packed order 4u+q, type wdt
+    DType wdt;
     const float* act;           // [D][T][B][G] packed
     const float* cst;           // [D][T][B][H]
     const float* c0;            // [D][B][H] or null
@@ -183,7 +185,7 @@ struct BwdRecArgs {
     unsigned long long* trace;  // [kTraceSteps][kTraceEvents] or null
 };
 cudaError_t launch_bwd_rec(const BwdRecArgs& a, cudaStream_t s);
-RecPlan plan_bwd_rec(int H, int B, int D, int num_sms, size_t smem_max);
+RecPlan plan_bwd_rec(int H, int B, int D, DType wdt, int num_sms, size_t smem_max);
 
 // db[d][r] = sum over groups of dbpart[d][g][r] (fixed order), written to
 // both db_ih[d] and db_hh[d].
@@ -204,5 +206,8 @@ struct SeqCopyArgs {
     DType dt;
 };
 cudaError_t launch_seq_copy(const SeqCopyArgs& a, cudaStream_t s);
+
+// dst[i] = src[i] for i < n, converting between float and bf16 (nearest even).
+cudaError_t launch_convert(const void* src, DType st, void* dst, DType dt, long long n, cudaStream_t s);
 
 }  // namespace lstm

@@ -363,14 +363,17 @@ __device__ __forceinline__ BwdPre bwd_fetch(const BwdRecArgs& a, int d, int t, i
     return r;
 }
 
+// WT: type of the resident W_hh rows (the weights' own type; products and
+// sums are float32 either way).
+template <typename WT>
 __global__ void __launch_bounds__(kRecThreads, 1) bwd_rec_kernel(BwdRecArgs a) {
     extern __shared__ __align__(16) unsigned char smem[];
     const RecPlan& p = a.p;
     const int H = a.H, B = a.B, T = a.T, D = a.D, G = 4 * H;
     const int Hp = (H + 3) & ~3;
     const int U = p.U, R4 = 4 * U, Bs = p.Bs, Bg = p.Bg;
-    float* Wr = reinterpret_cast<float*>(smem);                       // [4U][Hp]
-    size_t off = align16((size_t)R4 * Hp * 4);
+    WT* Wr = reinterpret_cast<WT*>(smem);                             // [4U][Hp]
+    size_t off = align16((size_t)R4 * Hp * sizeof(WT));
     float* daT = reinterpret_cast<float*>(smem + off);                // [4U][Bs]
     off += align16((size_t)R4 * Bs * 4);
     float* dcs = reinterpret_cast<float*>(smem + off);                // [U][Bg]
@@ -388,9 +391,11 @@ __global__ void __launch_bounds__(kRecThreads, 1) bwd_rec_kernel(BwdRecArgs a) {
     const int b0 = bg * Bg, nB = min(Bg, B - b0);
     const int tid = threadIdx.x, nth = blockDim.x;
     {
-        const float4* s4 = reinterpret_cast<const float4*>(a.wr + ((size_t)d * p.nu + j) * R4 * Hp);
-        float4* d4 = reinterpret_cast<float4*>(Wr);
-        for (int i = tid; i < R4 * Hp / 4; i += nth) d4[i] = s4[i];
+        const uint4* s4 = reinterpret_cast<const uint4*>(static_cast<const WT*>(a.wr) +
+                                                         ((size_t)d * p.nu + j) * R4 * Hp);
+        uint4* d4 = reinterpret_cast<uint4*>(Wr);
+        const int n16 = (int)((size_t)R4 * Hp * sizeof(WT) / 16);
+        for (int i = tid; i < n16; i += nth) d4[i] = s4[i];
     }
     for (int i = tid; i < U * Bg; i += nth) {
         const int ul = i / Bg, bl = i % Bg;
@@ -550,8 +555,10 @@ __global__ void __launch_bounds__(kRecThreads, 1) bwd_rec_kernel(BwdRecArgs a) {
 
 // Backward weight rows: out[d][p][k] (p < nu*4U, k < Hp) = W_hh[(p&3)*H + p/4][k],
 // zero outside the matrix.
+template <typename T>
 __global__ void pack_hh_rows_kernel(PackHhBwdArgs a) {
     const int Hp = (a.H + 3) & ~3;
+    T* out = static_cast<T*>(a.out);
     const int Rt = 4 * a.U * a.nu;
     const long long total = (long long)a.D * Rt * Hp;
     for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
@@ -560,7 +567,8 @@ __global__ void pack_hh_rows_kernel(PackHhBwdArgs a) {
         const long long r2 = e / Hp;
         const int pr = (int)(r2 % Rt), d = (int)(r2 / Rt);
         const int u = pr >> 2;
-        a.out[e] = (u < a.H && k < a.H) ? a.w[d][((long long)(pr & 3) * a.H + u) * a.H + k] : 0.f;
+        out[e] = (u < a.H && k < a.H) ? static_cast<const T*>(a.w[d])[((long long)(pr & 3) * a.H + u) * a.H + k]
+                                      : from_f<T>(0.f);
     }
 }
 
@@ -613,8 +621,9 @@ RecPlan plan_fwd_rec(int H, int B, int D, DType dt, int num_sms, size_t smem_max
     return best;
 }
 
-RecPlan plan_bwd_rec(int H, int B, int D, int num_sms, size_t smem_max) {
+RecPlan plan_bwd_rec(int H, int B, int D, DType wdt, int num_sms, size_t smem_max) {
     const int Hp = (H + 3) & ~3;
+    const size_t wes = dtype_size(wdt);
     RecPlan best{};
     double best_cost = 1e300;
     const int Us[] = {4, 8, 16, 32};
@@ -631,7 +640,7 @@ RecPlan plan_bwd_rec(int H, int B, int D, int num_sms, size_t smem_max) {
             bool ok = false;
             for (; Bs >= 4; Bs -= 4) {
                 const int CG = std::max(1, kRecThreads / ((U / 4) * std::min(Bg, kRecThreads)));
-                const size_t smem = align16h((size_t)4 * U * Hp * 4) + align16h((size_t)4 * U * Bs * 4) +
+                const size_t smem = align16h((size_t)4 * U * Hp * wes) + align16h((size_t)4 * U * Bs * 4) +
                                     2 * align16h((size_t)U * Bg * 4) + align16h((size_t)4 * U * Bg * 4) +
                                     align16h((size_t)CG * U * Bg * 4);
                 if (smem <= smem_max) {
@@ -669,7 +678,8 @@ cudaError_t launch_fwd_rec(const FwdRecArgs& a, cudaStream_t s) {
 cudaError_t launch_bwd_rec(const BwdRecArgs& a, cudaStream_t s) {
     BwdRecArgs args = a;
     void* params[] = {&args};
-    const void* fn = reinterpret_cast<const void*>(&bwd_rec_kernel);
+    const void* fn = a.wdt == DType::F32 ? reinterpret_cast<const void*>(&bwd_rec_kernel<float>)
+                                         : reinterpret_cast<const void*>(&bwd_rec_kernel<bf16>);
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)a.p.smem);
     if (e != cudaSuccess) return e;
     return cudaLaunchCooperativeKernel(fn, dim3(a.p.ctas), dim3(a.p.threads), params, a.p.smem, s);
@@ -678,7 +688,10 @@ cudaError_t launch_bwd_rec(const BwdRecArgs& a, cudaStream_t s) {
 cudaError_t launch_pack_hh_rows(const PackHhBwdArgs& a, cudaStream_t s) {
     const long long total = (long long)a.D * 4 * a.U * a.nu * ((a.H + 3) & ~3);
     const long long g = std::min<long long>(std::max<long long>((total + 255) / 256, 1), 148LL * 16);
-    pack_hh_rows_kernel<<<(int)g, 256, 0, s>>>(a);
+    if (a.dt == DType::F32)
+        pack_hh_rows_kernel<float><<<(int)g, 256, 0, s>>>(a);
+    else
+        pack_hh_rows_kernel<bf16><<<(int)g, 256, 0, s>>>(a);
     return cudaGetLastError();
 }
 

@@ -205,7 +205,26 @@ __global__ void seq_copy_kernel(SeqCopyArgs a) {
     }
 }
 
+// dst[i] = src[i] converted (float <-> bf16, round to nearest even)
+template <typename S, typename D>
+__global__ void convert_kernel(const S* __restrict__ src, D* __restrict__ dst, long long n) {
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+         i += (long long)gridDim.x * blockDim.x)
+        dst[i] = from_f<D>(to_f(src[i]));
+}
+
 }  // namespace
+
+cudaError_t launch_convert(const void* src, DType st, void* dst, DType dt, long long n, cudaStream_t s) {
+    if (n <= 0) return cudaSuccess;
+    if (st == DType::BF16 && dt == DType::F32)
+        convert_kernel<<<grid_for(n), 256, 0, s>>>(static_cast<const bf16*>(src), static_cast<float*>(dst), n);
+    else if (st == DType::F32 && dt == DType::BF16)
+        convert_kernel<<<grid_for(n), 256, 0, s>>>(static_cast<const float*>(src), static_cast<bf16*>(dst), n);
+    else
+        return cudaMemcpyAsync(dst, src, (size_t)n * dtype_size(st), cudaMemcpyDeviceToDevice, s);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_db_reduce(const DbArgs& a, cudaStream_t s) {
     const int n = a.D * a.G;

@@ -157,6 +157,8 @@ def make_inputs(wl: Workload, seed: int | None = None, zero_weights: bool = Fals
         if b_ih is not None:
             b_ih = [bf16_round(b) for b in b_ih]
             b_hh = [bf16_round(b) for b in b_hh]
+        if grad_out is not None:
+            grad_out = bf16_round(grad_out)   # the device holds it in bf16
     if not wl.batch_first:
         x = np.ascontiguousarray(x.transpose(1, 0, 2))
         if grad_out is not None:

@@ -103,10 +103,13 @@ def test_workspace_too_small():
     assert st == binding.LSTM_ERR_WORKSPACE
 
 
-def test_bf16_backward_unsupported():
+def test_bf16_backward_checks_workspace():
+    """bf16 backward is implemented (float32 staging in the workspace): an
+    undersized workspace is refused before anything is enqueued."""
     d = binding.make_desc(8, 16, 1, False, True, True, 4, 5, binding.LSTM_BF16)
     one = [256]
+    need = binding.lstm_workspace_size(d)
     st = binding.lstm_backward(d, 256, None, None, one, one, 256, None, None, 256, 256,
                                256, 256, 256, one, one, one, one, stream=0,
-                               ws_bytes=1 << 30, rs_bytes=1 << 30)
-    assert st == binding.LSTM_ERR_UNSUPPORTED
+                               ws_bytes=need - 1, rs_bytes=1 << 30)
+    assert st == binding.LSTM_ERR_WORKSPACE

@@ -2,7 +2,12 @@
 oracle on identical seeded inputs.
 
 Tolerances: float32 path max-abs 1e-5 on out, h_n, c_n and per-tensor
-max-rel 1e-4 on gradients (max|g - o| / max|o|); bf16 path max-abs 2e-2.
+max-rel 1e-4 on gradients (max|g - o| / max|o|); bf16 path max-abs 2e-2 on
+outputs and per-tensor max-rel 1e-2 on gradients.  The bf16 gradient bound is
+derived from the rounding the bf16 path applies and the oracle does not:
+h_t is rounded to bf16 every step of the forward (relative error up to
+2^-9 ~ 2e-3 per step, which the backward's saved sequence inherits) and dx,
+dh0 are returned in bf16 (another 2^-9); 1e-2 is five bf16 half-ulps.
 
 Small cases cover several tiles and ragged tails of every partition (units,
 batch groups, K slices) and the degenerate cases; the five workloads run at
@@ -14,13 +19,14 @@ import pytest
 import torch
 
 import oracle
-from layer_lstm_b200.workloads import WORKLOADS, Workload, make_inputs, select_rows
+from layer_lstm_b200.workloads import WORKLOADS, Workload, bf16_round, make_inputs, select_rows
 
 pytestmark = pytest.mark.gpu
 
 ATOL_F32 = 1e-5
 RTOL_GRAD = 1e-4
 ATOL_BF16 = 2e-2
+RTOL_GRAD_BF16 = 1e-2
 
 
 def _run_gpu(inp, cuda_lib):
@@ -51,19 +57,20 @@ def _relerr(g, o):
 
 def _check_bwd(wl, gpu, ref, rows=None, weights=True):
     bt = 0 if wl.batch_first else 1
+    rtol = RTOL_GRAD if wl.dtype == "f32" else RTOL_GRAD_BF16
     for k in ("dx", "dh0", "dc0"):
         g = gpu[k]
         if rows is not None:
             g = np.take(g, rows, axis=bt if k == "dx" else 1)
         e = _relerr(g, ref[k])
-        assert e <= RTOL_GRAD, f"{k}: max-rel {e:.3e}"
+        assert e <= rtol, f"{k}: max-rel {e:.3e}"
     if not weights:
         return
     keys = ["dw_ih", "dw_hh"] + (["db_ih", "db_hh"] if wl.bias else [])
     for k in keys:
         for i, (g, o) in enumerate(zip(gpu[k], ref[k])):
             e = _relerr(g, o)
-            assert e <= RTOL_GRAD, f"{k}[{i}]: max-rel {e:.3e}"
+            assert e <= rtol, f"{k}[{i}]: max-rel {e:.3e}"
 
 
 SMALL = {
@@ -107,6 +114,18 @@ TRAIN = {
     "B1_T1": SMALL["B1_T1"].replace(train=True),
     "f32_bi_wide": Workload("s", L=1, D=2, I=33, H=64, T=6, B=40, dtype="f32", state_std=0.2,
                             train=True, seed=110),
+    # bf16 BPTT (float32 arithmetic on widened copies; W_hh rows resident in bf16)
+    "bf16_bi_2layer": Workload("s", L=2, D=2, I=64, H=96, T=11, B=9, dtype="bf16", state_std=0.3,
+                               train=True, seed=141),
+    "bf16_uni_ragged": Workload("s", L=1, D=1, I=50, H=130, T=8, B=20, dtype="bf16", state_std=0.3,
+                                train=True, seed=142),
+    "bf16_bi_seqfirst": Workload("s", L=1, D=2, I=64, H=256, T=6, B=40, dtype="bf16",
+                                 batch_first=False, train=True, seed=143),
+    "bf16_long": Workload("s", L=2, D=1, I=32, H=64, T=64, B=8, dtype="bf16", state_std=0.3,
+                          train=True, seed=144),
+    # c3's layer shapes (H = 1024, bidirectional, 2 layers) on a short sequence
+    "bf16_c3_shape": Workload("s", L=2, D=2, I=512, H=1024, T=12, B=8, dtype="bf16", w_k=1 / 32,
+                              train=True, seed=145),
 }
 
 
@@ -118,6 +137,8 @@ def test_backward_small(name, cuda_lib):
     LDBH = (wl.L * wl.D, wl.B, wl.H)
     inp.grad_hn = rng.standard_normal(LDBH).astype(np.float32)
     inp.grad_cn = rng.standard_normal(LDBH).astype(np.float32)
+    if wl.dtype == "bf16":
+        inp.grad_hn = bf16_round(inp.grad_hn)   # the device holds it in bf16
     _, gpu = _run_gpu(inp, cuda_lib)
     ref = oracle.run_inputs(inp, backward=True)
     _check_fwd(wl, gpu, ref)
