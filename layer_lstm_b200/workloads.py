@@ -41,6 +41,7 @@ class Workload:
     bias: bool = True
     batch_first: bool = True
     seed: int = 0
+    varlen: bool = False   # per-row lengths ~ U{0..T} (drawn last), else all rows length T
 
     @property
     def G(self) -> int:
@@ -114,6 +115,7 @@ class Inputs:
     grad_out: np.ndarray | None = None   # same layout as out
     grad_hn: np.ndarray | None = None
     grad_cn: np.ndarray | None = None
+    lengths: np.ndarray | None = None    # (B,) int32 valid steps per row, or None (all T)
 
 
 def make_inputs(wl: Workload, seed: int | None = None, zero_weights: bool = False) -> Inputs:
@@ -163,7 +165,16 @@ def make_inputs(wl: Workload, seed: int | None = None, zero_weights: bool = Fals
         x = np.ascontiguousarray(x.transpose(1, 0, 2))
         if grad_out is not None:
             grad_out = np.ascontiguousarray(grad_out.transpose(1, 0, 2))
-    return Inputs(wl, x, h0, c0, w_ih, w_hh, b_ih, b_hh, grad_out)
+    lengths = None
+    if wl.varlen:
+        # drawn after everything else, so the other arrays match the fixed-length draw;
+        # one row always has the full length and one (if B > 1) is empty
+        lengths = rng.integers(0, T + 1, size=B).astype(np.int32)
+        if B > 0:
+            lengths[0] = T
+        if B > 1:
+            lengths[-1] = 0
+    return Inputs(wl, x, h0, c0, w_ih, w_hh, b_ih, b_hh, grad_out, lengths=lengths)
 
 
 def select_rows(inp: Inputs, rows) -> Inputs:
@@ -180,4 +191,5 @@ def select_rows(inp: Inputs, rows) -> Inputs:
 
     return Inputs(wl, take_seq(inp.x), take_state(inp.h0), take_state(inp.c0),
                   inp.w_ih, inp.w_hh, inp.b_ih, inp.b_hh, take_seq(inp.grad_out),
-                  take_state(inp.grad_hn), take_state(inp.grad_cn))
+                  take_state(inp.grad_hn), take_state(inp.grad_cn),
+                  None if inp.lengths is None else np.ascontiguousarray(inp.lengths[rows]))

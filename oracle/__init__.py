@@ -31,10 +31,11 @@ def _load():
         dp = ctypes.POINTER(ctypes.c_double)
         dpp = ctypes.POINTER(dp)
         i = ctypes.c_int
-        lib.oracle_lstm_forward.argtypes = [i, i, i, i, i, i, i, dp, dp, dp, dpp, dpp, dpp, dpp,
+        ip = ctypes.POINTER(ctypes.c_int)
+        lib.oracle_lstm_forward.argtypes = [i, i, i, i, i, i, i, ip, dp, dp, dp, dpp, dpp, dpp, dpp,
                                             dp, dp, dp]
         lib.oracle_lstm_forward.restype = i
-        lib.oracle_lstm_backward.argtypes = [i, i, i, i, i, i, i, dp, dp, dp, dpp, dpp, dpp, dpp,
+        lib.oracle_lstm_backward.argtypes = [i, i, i, i, i, i, i, ip, dp, dp, dp, dpp, dpp, dpp, dpp,
                                              dp, dp, dp, dp, dp, dp, dp, dp, dp, dpp, dpp, dpp, dpp]
         lib.oracle_lstm_backward.restype = i
         lib.oracle_num_threads.restype = i
@@ -63,6 +64,16 @@ def _ptr(a):
     return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
 
 
+def _lengths(lengths, B):
+    """(keep-alive array, pointer) for per-row lengths; NULL when None."""
+    if lengths is None:
+        return None, ctypes.POINTER(ctypes.c_int)()
+    a = np.ascontiguousarray(lengths, dtype=np.int32)
+    if a.shape != (B,):
+        raise ValueError(f"lengths must have shape ({B},)")
+    return a, a.ctypes.data_as(ctypes.POINTER(ctypes.c_int))
+
+
 def _ptr_array(arrs):
     dp = ctypes.POINTER(ctypes.c_double)
     if arrs is None:
@@ -79,8 +90,9 @@ def _dims(x, h_sz, L, D, batch_first):
 
 
 def lstm_forward(x, w_ih, w_hh, b_ih=None, b_hh=None, h0=None, c0=None,
-                 num_layers=1, bidirectional=False, batch_first=True):
-    """Returns (out, h_n, c_n) as float64 arrays in the same layout as x."""
+                 num_layers=1, bidirectional=False, batch_first=True, lengths=None):
+    """Returns (out, h_n, c_n) as float64 arrays in the same layout as x.
+    lengths: per-row valid steps (variable-length batch) or None."""
     lib = _load()
     L, D = int(num_layers), 2 if bidirectional else 1
     x = _f64(x)
@@ -97,7 +109,8 @@ def lstm_forward(x, w_ih, w_hh, b_ih=None, b_hh=None, h0=None, c0=None,
     out = np.zeros((B, T, D * H))
     h_n = np.zeros((L * D, B, H))
     c_n = np.zeros((L * D, B, H))
-    rc = lib.oracle_lstm_forward(L, D, I, H, B, T, int(bias), _ptr(x), _ptr(h0), _ptr(c0),
+    keep, lp = _lengths(lengths, B)
+    rc = lib.oracle_lstm_forward(L, D, I, H, B, T, int(bias), lp, _ptr(x), _ptr(h0), _ptr(c0),
                                  _ptr_array(w_ih), _ptr_array(w_hh), _ptr_array(b_ih),
                                  _ptr_array(b_hh), _ptr(out), _ptr(h_n), _ptr(c_n))
     if rc != 0:
@@ -109,7 +122,7 @@ def lstm_forward(x, w_ih, w_hh, b_ih=None, b_hh=None, h0=None, c0=None,
 
 def lstm_backward(x, w_ih, w_hh, grad_out, b_ih=None, b_hh=None, h0=None, c0=None,
                   grad_hn=None, grad_cn=None, num_layers=1, bidirectional=False,
-                  batch_first=True):
+                  batch_first=True, lengths=None):
     """Forward + BPTT.  Returns a dict with out, h_n, c_n, dx, dh0, dc0 and the
     per-(layer, direction) lists dw_ih, dw_hh, db_ih, db_hh (float64)."""
     lib = _load()
@@ -138,7 +151,8 @@ def lstm_backward(x, w_ih, w_hh, grad_out, b_ih=None, b_hh=None, h0=None, c0=Non
     dw_hh = [np.zeros((G, H)) for _ in range(L * D)]
     db_ih = [np.zeros(G) for _ in range(L * D)] if bias else None
     db_hh = [np.zeros(G) for _ in range(L * D)] if bias else None
-    rc = lib.oracle_lstm_backward(L, D, I, H, B, T, int(bias), _ptr(x), _ptr(h0), _ptr(c0),
+    keep, lp = _lengths(lengths, B)
+    rc = lib.oracle_lstm_backward(L, D, I, H, B, T, int(bias), lp, _ptr(x), _ptr(h0), _ptr(c0),
                                   _ptr_array(w_ih), _ptr_array(w_hh), _ptr_array(b_ih),
                                   _ptr_array(b_hh), _ptr(grad_out), _ptr(grad_hn), _ptr(grad_cn),
                                   _ptr(out), _ptr(h_n), _ptr(c_n), _ptr(dx), _ptr(dh0), _ptr(dc0),
@@ -157,7 +171,8 @@ def run_inputs(inp, backward=False):
     """Run the oracle on a layer_lstm_b200.workloads.Inputs bundle."""
     wl = inp.wl
     kw = dict(b_ih=inp.b_ih, b_hh=inp.b_hh, h0=inp.h0, c0=inp.c0, num_layers=wl.L,
-              bidirectional=wl.D == 2, batch_first=wl.batch_first)
+              bidirectional=wl.D == 2, batch_first=wl.batch_first,
+              lengths=getattr(inp, "lengths", None))
     if backward:
         return lstm_backward(inp.x, inp.w_ih, inp.w_hh, inp.grad_out, grad_hn=inp.grad_hn,
                              grad_cn=inp.grad_cn, **kw)

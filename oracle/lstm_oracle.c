@@ -44,6 +44,15 @@
  *        dW_ih += da x_t^T,  dW_hh += da h_{t-1}^T,  db_ih = db_hh += da
  *    These are the chain rule applied to the cell equations above.
  *
+ *  - Variable-length batches: "Complete Trace: nn.LSTM", Step 3, lists a
+ *    second overload for packed sequences (per-step batch sizes), and
+ *    "LSTM Forward Computation", Sequence Buckets, pads sequences to a fixed
+ *    length.  Plain reading, with lengths[b] (0 <= lengths[b] <= T) valid
+ *    steps in row b of the padded batch: row b is the ordinary problem on
+ *    its first lengths[b] steps (the reverse direction starts at step
+ *    lengths[b] - 1), its padded outputs are 0, h_n/c_n are its final states,
+ *    the padding receives no gradient and contributes none.
+ *
  * Layout of every array is row-major and batch-first as listed; the Python
  * wrapper converts seq-first data before calling.
  */
@@ -79,7 +88,11 @@ static double sig(double z) { return 1.0 / (1.0 + exp(-z)); }
 /* Problem description shared by the entry points. */
 typedef struct {
     int L, D, I, H, B, T, bias;
+    const int* lengths;   /* [B] valid steps per row, or NULL (all T) */
 } prob;
+
+/* Valid steps of row b. */
+static int row_len(const prob* p, int b) { return p->lengths ? p->lengths[b] : p->T; }
 
 static int in_size(const prob* p, int layer) { return layer == 0 ? p->I : p->D * p->H; }
 
@@ -155,19 +168,21 @@ static int forward_row(const prob* p, int b,
         free(a); free(hprev); free(h); free(c); free(bufA); free(bufB);
         return ORACLE_ERR_NOMEM;
     }
+    const int n = row_len(p, b);   /* this row's steps; positions n..T-1 are padding */
     /* layer-0 input: the x row */
     double* cur = rec ? rec->seq[0] : bufA;
     memcpy(cur, x + (size_t)b * T * p->I, sizeof(double) * (size_t)T * p->I);
     for (int l = 0; l < L; ++l) {
         const int in = in_size(p, l);
         double* nxt = rec ? rec->seq[l + 1] : (cur == bufA ? bufB : bufA);
+        memset(nxt, 0, sizeof(double) * (size_t)T * D * H);   /* padded outputs stay 0 */
         for (int d = 0; d < D; ++d) {
             const int ld = l * D + d;
             for (int u = 0; u < H; ++u) {
                 h[u] = h0 ? h0[((size_t)ld * B + b) * H + u] : 0.0;
                 c[u] = c0 ? c0[((size_t)ld * B + b) * H + u] : 0.0;
             }
-            cell_pass(T, in, H, d == 1, p->bias, cur, w_ih[ld], w_hh[ld],
+            cell_pass(n, in, H, d == 1, p->bias, cur, w_ih[ld], w_hh[ld],
                       p->bias ? b_ih[ld] : NULL, p->bias ? b_hh[ld] : NULL,
                       h, c, nxt + d * H, D * H,
                       rec ? rec->act[ld] : NULL, rec ? rec->hs[ld] : NULL, a, hprev);
@@ -186,21 +201,25 @@ static int forward_row(const prob* p, int b,
 static int check_prob(const prob* p) {
     if (p->L < 1 || (p->D != 1 && p->D != 2) || p->I < 1 || p->H < 1 || p->B < 0 || p->T < 0)
         return ORACLE_ERR_ARG;
+    if (p->lengths)
+        for (int b = 0; b < p->B; ++b)
+            if (p->lengths[b] < 0 || p->lengths[b] > p->T) return ORACLE_ERR_ARG;
     return ORACLE_OK;
 }
 
 /*
  * Forward.  x [B][T][I]; h0, c0 [L*D][B][H] or NULL (zeros); w_ih[l*D+d]
  * [4H][in_l]; w_hh [4H][H]; b_ih, b_hh [4H] (ignored when bias == 0);
- * out [B][T][D*H]; h_n, c_n [L*D][B][H].  Returns 0 on success.
+ * lengths [B] or NULL; out [B][T][D*H]; h_n, c_n [L*D][B][H].  Returns 0 on
+ * success.
  */
-int oracle_lstm_forward(int L, int D, int I, int H, int B, int T, int bias,
+int oracle_lstm_forward(int L, int D, int I, int H, int B, int T, int bias, const int* lengths,
                         const double* x, const double* h0, const double* c0,
                         const double* const* w_ih, const double* const* w_hh,
                         const double* const* b_ih, const double* const* b_hh,
                         double* out, double* h_n, double* c_n)
 {
-    prob p = {L, D, I, H, B, T, bias};
+    prob p = {L, D, I, H, B, T, bias, lengths};
     if (check_prob(&p)) return ORACLE_ERR_ARG;
     int err = 0;
 #pragma omp parallel for schedule(dynamic, 1) reduction(|:err)
@@ -258,6 +277,7 @@ static int backward_row(const prob* p, int b, const row_record* rec,
         free(dy); free(din); free(dh); free(dc); free(dhn);
         return ORACLE_ERR_NOMEM;
     }
+    const int n = row_len(p, b);   /* steps n..T-1 are padding: no gradient in or out */
     memcpy(dy, grad_out + (size_t)b * T * D * H, sizeof(double) * (size_t)T * D * H);
     for (int l = L - 1; l >= 0; --l) {
         const int in = in_size(p, l);
@@ -273,10 +293,10 @@ static int backward_row(const prob* p, int b, const row_record* rec,
                 dc[u] = grad_cn ? grad_cn[((size_t)ld * B + b) * H + u] : 0.0;
             }
             /* walk time opposite to the forward order of this direction */
-            for (int s = T - 1; s >= 0; --s) {
-                const int t = d == 1 ? T - 1 - s : s;
+            for (int s = n - 1; s >= 0; --s) {
+                const int t = d == 1 ? n - 1 - s : s;
                 const int tp = d == 1 ? t + 1 : t - 1;   /* forward-order predecessor */
-                const int has_prev = d == 1 ? (t + 1 < T) : (t >= 1);
+                const int has_prev = d == 1 ? (t + 1 < n) : (t >= 1);
                 const double* at = act + (size_t)t * 5 * H;
                 double* dat = dal + (size_t)t * G;
                 for (int u = 0; u < H; ++u) {
@@ -330,7 +350,7 @@ static int backward_row(const prob* p, int b, const row_record* rec,
  * dw_ih[l*D+d] [4H][in_l], dw_hh [4H][H], db_ih, db_hh [4H] (bias only).
  * The weight gradients are overwritten, not accumulated.
  */
-int oracle_lstm_backward(int L, int D, int I, int H, int B, int T, int bias,
+int oracle_lstm_backward(int L, int D, int I, int H, int B, int T, int bias, const int* lengths,
                          const double* x, const double* h0, const double* c0,
                          const double* const* w_ih, const double* const* w_hh,
                          const double* const* b_ih, const double* const* b_hh,
@@ -340,7 +360,7 @@ int oracle_lstm_backward(int L, int D, int I, int H, int B, int T, int bias,
                          double* const* dw_ih, double* const* dw_hh,
                          double* const* db_ih, double* const* db_hh)
 {
-    prob p = {L, D, I, H, B, T, bias};
+    prob p = {L, D, I, H, B, T, bias, lengths};
     if (check_prob(&p)) return ORACLE_ERR_ARG;
     const int G = 4 * H, LD = L * D;
     row_record* recs = (row_record*)calloc((size_t)B + 1, sizeof(row_record));
@@ -377,13 +397,14 @@ int oracle_lstm_backward(int L, int D, int I, int H, int B, int T, int bias,
                     const double* dal = da[b][ld];
                     const double* seq_in = recs[b].seq[l];
                     const double* hs = recs[b].hs[ld];
-                    for (int t = 0; t < T; ++t) {
+                    const int n = row_len(&p, b);
+                    for (int t = 0; t < n; ++t) {
                         const double g = dal[(size_t)t * G + r];
                         sb += g;
                         const double* xt = seq_in + (size_t)t * in;
                         for (int k = 0; k < in; ++k) wi[k] += g * xt[k];
                         /* h_{t-1} in this direction's order; h0 (or 0) at the start */
-                        const int has_prev = d == 1 ? (t + 1 < T) : (t >= 1);
+                        const int has_prev = d == 1 ? (t + 1 < n) : (t >= 1);
                         if (has_prev) {
                             const double* hp = hs + (size_t)(d == 1 ? t + 1 : t - 1) * H;
                             for (int j = 0; j < H; ++j) wh[j] += g * hp[j];

@@ -308,10 +308,23 @@ def _torch_lstm(inp):
     LDBH = (wl.L * wl.D, wl.B, wl.H)
     h0 = torch.tensor(inp.h0 if inp.h0 is not None else np.zeros(LDBH), dtype=torch.float64, requires_grad=True)
     c0 = torch.tensor(inp.c0 if inp.c0 is not None else np.zeros(LDBH), dtype=torch.float64, requires_grad=True)
-    out, (hn, cn) = m(x, (h0, c0))
+    if inp.lengths is None:
+        out, (hn, cn) = m(x, (h0, c0))
+    else:
+        # packed sequences (the lstm.data overload); padding back with zeros
+        from torch.nn.utils.rnn import pack_padded_sequence, pad_packed_sequence
+        packed = pack_padded_sequence(x, torch.tensor(inp.lengths, dtype=torch.int64),
+                                      batch_first=wl.batch_first, enforce_sorted=False)
+        pout, (hn, cn) = m(packed, (h0, c0))
+        out, _ = pad_packed_sequence(pout, batch_first=wl.batch_first, padding_value=0.0,
+                                     total_length=wl.T)
     res = dict(out=out.detach().numpy(), h_n=hn.detach().numpy(), c_n=cn.detach().numpy())
     if inp.grad_out is not None:
         loss = (out * torch.tensor(inp.grad_out, dtype=torch.float64)).sum()
+        if inp.grad_hn is not None:
+            loss = loss + (hn * torch.tensor(inp.grad_hn, dtype=torch.float64)).sum()
+        if inp.grad_cn is not None:
+            loss = loss + (cn * torch.tensor(inp.grad_cn, dtype=torch.float64)).sum()
         loss.backward()
         res["dx"] = x.grad.numpy()
         res["dh0"] = h0.grad.numpy()
@@ -353,3 +366,65 @@ def test_empty_sequence_returns_initial_state():
     assert r["out"].shape == (2, 0, 8)
     np.testing.assert_array_equal(r["h_n"], inp.h0)
     np.testing.assert_array_equal(r["c_n"], inp.c0)
+
+
+# ------------------------------------------------ variable-length batches
+def _varlen_inputs(seed, lengths, **kw):
+    wl = Workload("vl", dtype="f32", train=True, seed=seed, varlen=True, **kw)
+    inp = make_inputs(wl)
+    inp.lengths = np.asarray(lengths, dtype=np.int32)
+    rng = np.random.default_rng(seed)
+    LDBH = (wl.L * wl.D, wl.B, wl.H)
+    inp.grad_hn = rng.standard_normal(LDBH).astype(np.float32)
+    inp.grad_cn = rng.standard_normal(LDBH).astype(np.float32)
+    return inp
+
+
+@pytest.mark.parametrize("kw,lengths", [
+    (dict(L=1, D=1, I=4, H=5, T=6, B=4, state_std=0.3), [6, 1, 3, 5]),
+    (dict(L=2, D=2, I=3, H=4, T=7, B=3, state_std=0.3), [2, 7, 4]),
+    (dict(L=2, D=2, I=3, H=4, T=5, B=3, state_std=0.2, batch_first=False), [5, 3, 1]),
+], ids=["uni", "bi2", "bi_seqfirst"])
+def test_varlen_matches_torch_packed_float64(kw, lengths):
+    """Per-row lengths against torch's packed-sequence LSTM in float64 (zero
+    padding, final states of each row, gradients through the packing)."""
+    inp = _varlen_inputs(51, lengths, **kw)
+    ref = _torch_lstm(inp)
+    r = oracle.run_inputs(inp, backward=True)
+    for k in ("out", "h_n", "c_n", "dx", "dh0", "dc0"):
+        np.testing.assert_allclose(r[k], ref[k], rtol=0, atol=1e-12, err_msg=k)
+    for ours, theirs in (("dw_ih", "weight_ih"), ("dw_hh", "weight_hh"), ("db_ih", "bias_ih")):
+        for a, b in zip(r[ours], ref[theirs]):
+            np.testing.assert_allclose(a, b, rtol=0, atol=1e-12, err_msg=ours)
+
+
+def test_varlen_row_is_the_truncated_problem():
+    """Row b with n valid steps gives, on its first n steps, exactly the
+    fixed-length problem on x[b, :n]; its padded outputs and input
+    gradients are zero."""
+    inp = _varlen_inputs(52, [5, 2, 4], L=2, D=2, I=3, H=4, T=5, B=3, state_std=0.3)
+    r = oracle.run_inputs(inp, backward=True)
+    for b, n in enumerate(inp.lengths):
+        one = select_rows(inp, [b])
+        one.lengths = None
+        one.wl = one.wl.replace(T=int(n), varlen=False)
+        one.x = np.ascontiguousarray(one.x[:, :n])
+        one.grad_out = np.ascontiguousarray(one.grad_out[:, :n])
+        ref = oracle.run_inputs(one, backward=True)
+        np.testing.assert_array_equal(r["out"][b, :n], ref["out"][0])
+        assert not np.any(r["out"][b, n:]) and not np.any(r["dx"][b, n:])
+        np.testing.assert_array_equal(r["dx"][b, :n], ref["dx"][0])
+        for k in ("h_n", "c_n", "dh0", "dc0"):
+            np.testing.assert_array_equal(r[k][:, b], ref[k][:, 0], err_msg=k)
+
+
+def test_varlen_empty_row_keeps_initial_state():
+    """A row of length 0 runs no step: zero outputs, h_n = h0, c_n = c0, and
+    the state gradients pass straight through (dh0 = grad_hn, dc0 = grad_cn)."""
+    inp = _varlen_inputs(53, [3, 0], L=2, D=2, I=3, H=4, T=3, B=2, state_std=0.5)
+    r = oracle.run_inputs(inp, backward=True)
+    assert not np.any(r["out"][1]) and not np.any(r["dx"][1])
+    np.testing.assert_array_equal(r["h_n"][:, 1], inp.h0[:, 1])
+    np.testing.assert_array_equal(r["c_n"][:, 1], inp.c0[:, 1])
+    np.testing.assert_array_equal(r["dh0"][:, 1], inp.grad_hn[:, 1])
+    np.testing.assert_array_equal(r["dc0"][:, 1], inp.grad_cn[:, 1])
