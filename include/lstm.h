@@ -145,6 +145,34 @@ lstm_status lstm_backward(const lstm_desc* desc, const void* x, const void* h0, 
                           float* const* db_ih, float* const* db_hh, cudaStream_t stream);
 
 /*
+ * Variable-length batches ([trace] Step 3: the packed-sequence overload of
+ * the LSTM op; [mxnet] Sequence Buckets: sequences padded to a fixed
+ * length).  `lengths` is a device array of desc->batch int32 values: row b
+ * of the padded x holds lengths[b] valid steps (values above seq_len act as
+ * seq_len, below 0 as 0); NULL means every row has seq_len steps, which is
+ * lstm_forward / lstm_backward.  Row b is the ordinary problem on its first
+ * lengths[b] steps: the reverse direction starts at step lengths[b] - 1, out
+ * is 0 at padded positions, h_n / c_n hold each row's final states, the
+ * padding of grad_out is ignored and dx is 0 there.  Arguments, buffers and
+ * errors are otherwise those of lstm_forward / lstm_backward; the backward
+ * takes the same lengths as its forward.
+ */
+lstm_status lstm_forward_varlen(const lstm_desc* desc, const int* lengths, const void* x, const void* h0,
+                                const float* c0, const void* const* w_ih, const void* const* w_hh,
+                                const void* const* b_ih, const void* const* b_hh,
+                                void* out, void* h_n, float* c_n,
+                                void* workspace, size_t ws_bytes,
+                                void* reserve, size_t rs_bytes, cudaStream_t stream);
+lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, const void* x, const void* h0,
+                                 const float* c0, const void* const* w_ih, const void* const* w_hh,
+                                 const void* grad_out, const void* grad_hn, const float* grad_cn,
+                                 const void* reserve, size_t rs_bytes,
+                                 void* workspace, size_t ws_bytes,
+                                 void* dx, void* dh0, float* dc0,
+                                 float* const* dw_ih, float* const* dw_hh,
+                                 float* const* db_ih, float* const* db_hh, cudaStream_t stream);
+
+/*
  * Inference forward that allocates nothing and takes no workspace.  The pages
  * have no counterpart: this is an integration aid.  It exists for callers
  * that cannot call cudaMalloc or size a workspace for us, such as a plugin

@@ -23,7 +23,8 @@ LSTM_BF16 = 1
 
 EXPORTED = ("lstm_workspace_size", "lstm_reserve_size", "lstm_forward", "lstm_backward",
             "lstm_query_status", "lstm_status_string", "lstm_timing_enable", "lstm_timing_read",
-            "lstm_timing_reset", "lstm_forward_noalloc", "lstm_trace_enable", "lstm_trace_read")
+            "lstm_timing_reset", "lstm_forward_noalloc", "lstm_trace_enable", "lstm_trace_read",
+            "lstm_forward_varlen", "lstm_backward_varlen")
 LSTM_NOALLOC_SCRATCH_BYTES = 32 << 20
 LSTM_TRACE_MAX_STEPS = 512
 LSTM_TRACE_EVENTS = 16
@@ -88,6 +89,10 @@ def load(build_if_stale: bool = True):
     lib.lstm_backward.argtypes = [dp, vp, vp, vp, vpp, vpp, vp, vp, vp, vp, sz, vp, sz, vp, vp, vp,
                                   vpp, vpp, vpp, vpp, vp]
     lib.lstm_backward.restype = ctypes.c_int
+    lib.lstm_forward_varlen.argtypes = [dp, vp] + list(lib.lstm_forward.argtypes[1:])
+    lib.lstm_forward_varlen.restype = ctypes.c_int
+    lib.lstm_backward_varlen.argtypes = [dp, vp] + list(lib.lstm_backward.argtypes[1:])
+    lib.lstm_backward_varlen.restype = ctypes.c_int
     lib.lstm_query_status.argtypes = [vp, vp]
     lib.lstm_query_status.restype = ctypes.c_int
     lib.lstm_status_string.argtypes = [ctypes.c_int]
@@ -154,25 +159,33 @@ def lstm_reserve_size(desc: lstm_desc) -> int:
 
 
 def lstm_forward(desc, x, h0, c0, w_ih, w_hh, b_ih, b_hh, out, h_n, c_n, workspace,
-                 reserve=None, stream=None, ws_bytes=None, rs_bytes=None) -> int:
+                 reserve=None, stream=None, ws_bytes=None, rs_bytes=None, lengths=None) -> int:
+    """lengths: device int32 tensor of per-row valid steps (lstm_forward_varlen),
+    or None (lstm_forward)."""
     lib = load()
-    return lib.lstm_forward(ctypes.byref(desc), _p(x), _p(h0), _p(c0), _parr(w_ih), _parr(w_hh),
-                            _parr(b_ih), _parr(b_hh), _p(out), _p(h_n), _p(c_n),
-                            _p(workspace), _nbytes(workspace) if ws_bytes is None else ws_bytes,
-                            _p(reserve), _nbytes(reserve) if rs_bytes is None else rs_bytes,
-                            _stream(stream))
+    args = (_p(x), _p(h0), _p(c0), _parr(w_ih), _parr(w_hh),
+            _parr(b_ih), _parr(b_hh), _p(out), _p(h_n), _p(c_n),
+            _p(workspace), _nbytes(workspace) if ws_bytes is None else ws_bytes,
+            _p(reserve), _nbytes(reserve) if rs_bytes is None else rs_bytes,
+            _stream(stream))
+    if lengths is None:
+        return lib.lstm_forward(ctypes.byref(desc), *args)
+    return lib.lstm_forward_varlen(ctypes.byref(desc), _p(lengths), *args)
 
 
 def lstm_backward(desc, x, h0, c0, w_ih, w_hh, grad_out, grad_hn, grad_cn, reserve, workspace,
                   dx, dh0, dc0, dw_ih, dw_hh, db_ih, db_hh, stream=None,
-                  ws_bytes=None, rs_bytes=None) -> int:
+                  ws_bytes=None, rs_bytes=None, lengths=None) -> int:
     lib = load()
-    return lib.lstm_backward(ctypes.byref(desc), _p(x), _p(h0), _p(c0), _parr(w_ih), _parr(w_hh),
-                             _p(grad_out), _p(grad_hn), _p(grad_cn), _p(reserve),
-                             _nbytes(reserve) if rs_bytes is None else rs_bytes,
-                             _p(workspace), _nbytes(workspace) if ws_bytes is None else ws_bytes,
-                             _p(dx), _p(dh0), _p(dc0), _parr(dw_ih), _parr(dw_hh),
-                             _parr(db_ih), _parr(db_hh), _stream(stream))
+    args = (_p(x), _p(h0), _p(c0), _parr(w_ih), _parr(w_hh),
+            _p(grad_out), _p(grad_hn), _p(grad_cn), _p(reserve),
+            _nbytes(reserve) if rs_bytes is None else rs_bytes,
+            _p(workspace), _nbytes(workspace) if ws_bytes is None else ws_bytes,
+            _p(dx), _p(dh0), _p(dc0), _parr(dw_ih), _parr(dw_hh),
+            _parr(db_ih), _parr(db_hh), _stream(stream))
+    if lengths is None:
+        return lib.lstm_backward(ctypes.byref(desc), *args)
+    return lib.lstm_backward_varlen(ctypes.byref(desc), _p(lengths), *args)
 
 
 def lstm_forward_noalloc(desc, x, h0, c0, w_ih, w_hh, b_ih, b_hh, out, h_n, c_n,

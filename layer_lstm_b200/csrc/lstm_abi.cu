@@ -425,6 +425,16 @@ lstm_status lstm_forward(const lstm_desc* desc, const void* x, const void* h0, c
                          void* out, void* h_n, float* c_n,
                          void* workspace, size_t ws_bytes,
                          void* reserve, size_t rs_bytes, cudaStream_t stream) {
+    return lstm_forward_varlen(desc, nullptr, x, h0, c0, w_ih, w_hh, b_ih, b_hh, out, h_n, c_n, workspace,
+                               ws_bytes, reserve, rs_bytes, stream);
+}
+
+lstm_status lstm_forward_varlen(const lstm_desc* desc, const int* lengths, const void* x, const void* h0,
+                                const float* c0, const void* const* w_ih, const void* const* w_hh,
+                                const void* const* b_ih, const void* const* b_hh,
+                                void* out, void* h_n, float* c_n,
+                                void* workspace, size_t ws_bytes,
+                                void* reserve, size_t rs_bytes, cudaStream_t stream) {
     if (!valid_desc(desc)) return LSTM_ERR_INVALID_ARG;
     if (!w_ih || !w_hh) return LSTM_ERR_INVALID_ARG;
     const int LD = desc->num_layers * (desc->bidirectional ? 2 : 1);
@@ -531,6 +541,7 @@ lstm_status lstm_forward(const lstm_desc* desc, const void* x, const void* h0, c
             tr.status = status;
             tr.timeout_ns = timeout_ns();
             tr.trace = trace_for(LSTM_TRACE_FWD_REC_TC, T, stream);
+            tr.len = lengths;
             LSTM_CUDA(timed(K_FWD_REC_TC, stream, [&] { return launch_tc_rec(tr, stream); }));
             layer_in = hseq_tc;
             continue;
@@ -566,6 +577,7 @@ lstm_status lstm_forward(const lstm_desc* desc, const void* x, const void* h0, c
         f.status = status;
         f.timeout_ns = timeout_ns();
         f.trace = trace_for(LSTM_TRACE_FWD_REC_FFMA, T, stream);
+        f.len = lengths;
         LSTM_CUDA(timed(K_FWD_REC_FFMA, stream, [&] { return launch_fwd_rec(f, stream); }));
         layer_in = hseq;
     }
@@ -580,6 +592,18 @@ lstm_status lstm_backward(const lstm_desc* desc, const void* x, const void* h0, 
                           void* dx, void* dh0, float* dc0,
                           float* const* dw_ih, float* const* dw_hh,
                           float* const* db_ih, float* const* db_hh, cudaStream_t stream) {
+    return lstm_backward_varlen(desc, nullptr, x, h0, c0, w_ih, w_hh, grad_out, grad_hn, grad_cn, reserve,
+                                rs_bytes, workspace, ws_bytes, dx, dh0, dc0, dw_ih, dw_hh, db_ih, db_hh, stream);
+}
+
+lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, const void* x, const void* h0,
+                                 const float* c0, const void* const* w_ih, const void* const* w_hh,
+                                 const void* grad_out, const void* grad_hn, const float* grad_cn,
+                                 const void* reserve, size_t rs_bytes,
+                                 void* workspace, size_t ws_bytes,
+                                 void* dx, void* dh0, float* dc0,
+                                 float* const* dw_ih, float* const* dw_hh,
+                                 float* const* db_ih, float* const* db_hh, cudaStream_t stream) {
     if (!valid_desc(desc)) return LSTM_ERR_INVALID_ARG;
     if (!w_ih || !w_hh || !dw_ih || !dw_hh) return LSTM_ERR_INVALID_ARG;
     const int LD = desc->num_layers * (desc->bidirectional ? 2 : 1);
@@ -709,6 +733,7 @@ lstm_status lstm_backward(const lstm_desc* desc, const void* x, const void* h0, 
         b.status = status;
         b.timeout_ns = timeout_ns();
         b.trace = trace_for(LSTM_TRACE_BWD_REC_FFMA, T, stream);
+        b.len = lengths;
         LSTM_CUDA(timed(K_BWD_REC_FFMA, stream, [&] { return launch_bwd_rec(b, stream); }));
 
         if (desc->bias) {

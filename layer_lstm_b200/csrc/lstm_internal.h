@@ -133,6 +133,7 @@ struct FwdRecArgs {
     int* status;
     uint64_t timeout_ns;
     unsigned long long* trace;  // [kTraceSteps][kTraceEvents] or null
+    const int* len;             // [B] valid steps per row, or null (all T)
 };
 cudaError_t launch_fwd_rec(const FwdRecArgs& a, cudaStream_t s);
 RecPlan plan_fwd_rec(int H, int B, int D, DType dt, int num_sms, size_t smem_max);
@@ -161,6 +162,7 @@ struct TcRecArgs {
     int* status;
     uint64_t timeout_ns;
     unsigned long long* trace;  // [kTraceSteps][kTraceEvents] or null
+    const int* len;             // [B] valid steps per row, or null (all T)
 };
 cudaError_t launch_tc_rec(const TcRecArgs& a, cudaStream_t s);
 
@@ -183,6 +185,7 @@ struct BwdRecArgs {
     int* status;
     uint64_t timeout_ns;
     unsigned long long* trace;  // [kTraceSteps][kTraceEvents] or null
+    const int* len;             // [B] valid steps per row, or null (all T)
 };
 cudaError_t launch_bwd_rec(const BwdRecArgs& a, cudaStream_t s);
 RecPlan plan_bwd_rec(int H, int B, int D, DType wdt, int num_sms, size_t smem_max);

@@ -311,21 +311,30 @@ __global__ void __launch_bounds__(kRecThreads, 1) fwd_rec_kernel(FwdRecArgs a) {
                     for (int ks = 0; ks < KS; ++ks) acc += red[((size_t)ks * R + 4 * ul + g) * Bs + bl];
                     pre[g] += acc;
                 }
-                const float ig = sigmoidf_(pre[0]);
-                const float fg = sigmoidf_(pre[1]);
-                const float gg = tanhf(pre[2]);
-                const float og = sigmoidf_(pre[3]);
                 float& cref = cs[ul * p.Bg + bs0 + bl];
-                const float c = fg * cref + ig * gg;
-                cref = c;
-                const float h = og * tanhf(c);
-                const WT hv = from_f<WT>(h);
+                // Padding of a variable-length row: the state stays as it was
+                // (h from the gathered tile), the user output is 0, and the
+                // exchange and the saved sequence carry the frozen h.
+                const bool valid = !a.len || t < a.len[b];
+                float c = cref;
+                WT hv = hs[(size_t)u * Bs + bl];
+                float4 gates = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (valid) {
+                    const float ig = sigmoidf_(pre[0]);
+                    const float fg = sigmoidf_(pre[1]);
+                    const float gg = tanhf(pre[2]);
+                    const float og = sigmoidf_(pre[3]);
+                    c = fg * cref + ig * gg;
+                    cref = c;
+                    hv = from_f<WT>(og * tanhf(c));
+                    gates = make_float4(ig, fg, gg, og);
+                }
                 hT_grp[((size_t)d * T + t) * hT_tstride + (size_t)u * p.Bg + bs0 + bl] = hv;
                 if (hseq) hseq[((size_t)t * B + b) * ldseq + (size_t)d * H + u] = hv;
-                if (out) out[(size_t)t * a.out_st + (size_t)b * a.out_sb + (size_t)d * H + u] = hv;
+                if (out)
+                    out[(size_t)t * a.out_st + (size_t)b * a.out_sb + (size_t)d * H + u] = valid ? hv : from_f<WT>(0.f);
                 if (a.act) {
-                    *reinterpret_cast<float4*>(a.act + (((size_t)d * T + t) * B + b) * G + 4 * u) =
-                        make_float4(ig, fg, gg, og);
+                    *reinterpret_cast<float4*>(a.act + (((size_t)d * T + t) * B + b) * G + 4 * u) = gates;
                     a.cst[(((size_t)d * T + t) * B + b) * H + u] = c;
                 }
                 if (s == T - 1) {
@@ -382,6 +391,9 @@ __global__ void __launch_bounds__(kRecThreads, 1) bwd_rec_kernel(BwdRecArgs a) {
     off += align16((size_t)U * Bg * 4);
     float* dbacc = reinterpret_cast<float*>(smem + off);              // [4][U][Bg]
     off += align16((size_t)4 * U * Bg * 4);
+    // dh that padding of a variable-length row hands on unchanged (h_t = h_{t-1})
+    float* dpass = reinterpret_cast<float*>(smem + off);              // [U][Bg]
+    off += align16((size_t)U * Bg * 4);
     float* gpart = reinterpret_cast<float*>(smem + off);              // [CG][U][Bg]
 
     const int j = blockIdx.x % p.nu;
@@ -409,6 +421,7 @@ __global__ void __launch_bounds__(kRecThreads, 1) bwd_rec_kernel(BwdRecArgs a) {
         dhs[i] = dh;
     }
     for (int i = tid; i < 4 * U * Bg; i += nth) dbacc[i] = 0.f;
+    for (int i = tid; i < U * Bg; i += nth) dpass[i] = 0.f;
     __syncthreads();
     if (nB <= 0) return;
 
@@ -448,7 +461,7 @@ __global__ void __launch_bounds__(kRecThreads, 1) bwd_rec_kernel(BwdRecArgs a) {
             const int ul = i / nB, bl = i % nB;
             float s = 0.f;
             for (int cg = 0; cg < CG; ++cg) s += gpart[((size_t)cg * U + ul) * Bg + bl];
-            dhs[ul * Bg + bl] = s;
+            dhs[ul * Bg + bl] = s + dpass[ul * Bg + bl];
         }
         __syncthreads();
     };
@@ -482,6 +495,18 @@ __global__ void __launch_bounds__(kRecThreads, 1) bwd_rec_kernel(BwdRecArgs a) {
                     continue;
                 }
                 const int b = b0 + bs0 + bl, jj = j0 + ul;
+                float* dgp = a.dG + ((size_t)t * B + b) * ldg + (size_t)d * G + jj;
+                if (a.len && t >= a.len[b]) {
+                    // padding of a variable-length row: the state was held, so
+                    // no gate gradient; dc and dh pass on unchanged (the output
+                    // there is constant 0: grad_out does not enter)
+                    dpass[ul * Bg + bs0 + bl] = dhs[ul * Bg + bs0 + bl];
+                    dgp[0] = 0.f; dgp[H] = 0.f; dgp[2 * H] = 0.f; dgp[3 * H] = 0.f;
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) daT[(4 * ul + g) * Bs + bl] = 0.f;
+                    continue;
+                }
+                dpass[ul * Bg + bs0 + bl] = 0.f;
                 const BwdPre v = (bs0 == 0 && i < np0 && nb == nb0 && Bs == nb0 && q < 2)
                                      ? pre[q] : bwd_fetch(a, d, t, b, jj);
                 const float ig = v.act.x, fg = v.act.y, gg = v.act.z, og = v.act.w;
@@ -494,7 +519,6 @@ __global__ void __launch_bounds__(kRecThreads, 1) bwd_rec_kernel(BwdRecArgs a) {
                 const float da_g = dc * ig * (1.f - gg * gg);
                 const float da_o = dh * th * og * (1.f - og);
                 dcref = dc * fg;
-                float* dgp = a.dG + ((size_t)t * B + b) * ldg + (size_t)d * G + jj;
                 dgp[0] = da_i;
                 dgp[H] = da_f;
                 dgp[2 * H] = da_g;
@@ -641,7 +665,7 @@ RecPlan plan_bwd_rec(int H, int B, int D, DType wdt, int num_sms, size_t smem_ma
             for (; Bs >= 4; Bs -= 4) {
                 const int CG = std::max(1, kRecThreads / ((U / 4) * std::min(Bg, kRecThreads)));
                 const size_t smem = align16h((size_t)4 * U * Hp * wes) + align16h((size_t)4 * U * Bs * 4) +
-                                    2 * align16h((size_t)U * Bg * 4) + align16h((size_t)4 * U * Bg * 4) +
+                                    3 * align16h((size_t)U * Bg * 4) + align16h((size_t)4 * U * Bg * 4) +
                                     align16h((size_t)CG * U * Bg * 4);
                 if (smem <= smem_max) {
                     pl = RecPlan{nbg, Bg, nu, U, Bs, 1, kRecThreads, smem, ctas};

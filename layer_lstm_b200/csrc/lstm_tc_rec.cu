@@ -67,6 +67,7 @@ struct TcRecParams {
     int* status;
     uint64_t timeout_ns;
     unsigned long long* trace;   // per-step timeline of block 0, or null
+    const int* len;              // [B] valid steps per row, or null (all T)
 };
 
 // Branch-free choice among four registers by a lane-dependent index k in
@@ -518,11 +519,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int lc = 16 * cc + 4 * gq + i;   // column within the own half
                         const int col = own0 + lc;
                         if (col >= nB) continue;
-                        const float ig = sigmoid_fast(pi), fg = sigmoid_fast(pf), gg = tanh_fast(pgg);
-                        const float og = sigmoid_fast(po);
-                        const float c = fg * creg[k][i] + ig * gg;
-                        creg[k][i] = c;
-                        const bf16 hv = __float2bfloat16_rn(og * tanh_fast(c));
+                        const int bb = b0 + col;
+                        float c = creg[k][i];
+                        bf16 hv;
+                        if (!a.len || t < a.len[bb]) {
+                            const float ig = sigmoid_fast(pi), fg = sigmoid_fast(pf), gg = tanh_fast(pgg);
+                            const float og = sigmoid_fast(po);
+                            c = fg * c + ig * gg;
+                            creg[k][i] = c;
+                            hv = __float2bfloat16_rn(og * tanh_fast(c));
+                        } else {
+                            // padding of a variable-length row: the state stays
+                            hv = __ldcg(a.hx + ((size_t)(d * (T + 1) + s) * B + bb) * H + u);
+                        }
                         // unit octet q of column lc, stored at octet q ^ gq
                         // ((lc >> 2) & 3 == gq): the four columns of a warp's
                         // store fall in different banks
@@ -550,7 +559,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     *reinterpret_cast<uint4*>(hxo + (size_t)b * H + 8 * oct) = val;
                     const size_t uo = (size_t)d * H + 32 * j + 8 * oct;
                     if (a.hseq) *reinterpret_cast<uint4*>(a.hseq + ((size_t)t * B + b) * ldseq + uo) = val;
-                    if (a.out) {
+                    if (a.out && a.len && t >= a.len[b]) {   // padding: the user output is 0
+                        bf16* dst = a.out + (size_t)t * a.out_st + (size_t)b * a.out_sb + uo;
+#pragma unroll
+                        for (int x = 0; x < 8; ++x) dst[x] = __float2bfloat16_rn(0.f);
+                    } else if (a.out) {
                         bf16* dst = a.out + (size_t)t * a.out_st + (size_t)b * a.out_sb + uo;
                         if (a.out_vec) {
                             *reinterpret_cast<uint4*>(dst) = val;
@@ -660,6 +673,7 @@ cudaError_t launch_tc_rec(const TcRecArgs& a, cudaStream_t s) {
     prm.h_n = static_cast<bf16*>(a.h_n); prm.c_n = a.c_n;
     prm.wpk = static_cast<const bf16*>(a.wpk);
     prm.trace = a.trace;
+    prm.len = a.len;
     prm.ctr = a.ctr; prm.status = a.status; prm.timeout_ns = a.timeout_ns;
     cudaError_t e = cudaFuncSetAttribute(tc_rec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
     if (e != cudaSuccess) return e;

@@ -39,6 +39,9 @@ class DeviceProblem:
             return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device=device, dtype=dtype)
 
         self.desc = desc_for(wl)
+        self.lengths = None
+        if getattr(inp, "lengths", None) is not None:
+            self.lengths = torch.from_numpy(np.ascontiguousarray(inp.lengths, dtype=np.int32)).to(device)
         self.x = dev(inp.x)
         self.h0 = dev(inp.h0)
         self.c0 = dev(inp.c0, torch.float32)
@@ -74,14 +77,14 @@ class DeviceProblem:
     def forward(self, stream=None) -> int:
         return binding.lstm_forward(self.desc, self.x, self.h0, self.c0, self.w_ih, self.w_hh,
                                     self.b_ih, self.b_hh, self.out, self.h_n, self.c_n,
-                                    self.workspace, self.reserve, stream)
+                                    self.workspace, self.reserve, stream, lengths=self.lengths)
 
     def backward(self, stream=None) -> int:
         return binding.lstm_backward(self.desc, self.x, self.h0, self.c0, self.w_ih, self.w_hh,
                                      self.grad_out, self.grad_hn, self.grad_cn, self.reserve,
                                      self.workspace, self.dx, self.dh0, self.dc0, self.dw_ih,
                                      self.dw_hh, self.db_ih if self.wl.bias else None,
-                                     self.db_hh if self.wl.bias else None, stream)
+                                     self.db_hh if self.wl.bias else None, stream, lengths=self.lengths)
 
     def step(self, stream=None) -> None:
         binding.check(self.forward(stream), "lstm_forward")
