@@ -42,6 +42,8 @@ class Workload:
     batch_first: bool = True
     seed: int = 0
     varlen: bool = False   # per-row lengths ~ U{0..T} (drawn last), else all rows length T
+    dropout: float = 0.0   # inter-layer dropout probability of the training forward
+    dropout_seed: int = 0  # key word 0 of its Philox4x64-10 stream
 
     @property
     def G(self) -> int:

@@ -35,13 +35,28 @@ def _load():
         lib.oracle_lstm_forward.argtypes = [i, i, i, i, i, i, i, ip, dp, dp, dp, dpp, dpp, dpp, dpp,
                                             dp, dp, dp]
         lib.oracle_lstm_forward.restype = i
-        lib.oracle_lstm_backward.argtypes = [i, i, i, i, i, i, i, ip, dp, dp, dp, dpp, dpp, dpp, dpp,
+        u64 = ctypes.c_uint64
+        lib.oracle_lstm_backward.argtypes = [i, i, i, i, i, i, i, ip, ctypes.c_double, u64,
+                                             dp, dp, dp, dpp, dpp, dpp, dpp,
                                              dp, dp, dp, dp, dp, dp, dp, dp, dp, dpp, dpp, dpp, dpp]
         lib.oracle_lstm_backward.restype = i
         lib.oracle_num_threads.restype = i
+        u64p = ctypes.POINTER(ctypes.c_uint64)
+        lib.oracle_philox4x64_10.argtypes = [u64p, u64p, u64p]
+        lib.oracle_philox4x64_10.restype = None
         lib.oracle_set_num_threads.argtypes = [i]
         _lib = lib
     return _lib
+
+
+def philox4x64_10(ctr, key):
+    """The oracle's Philox4x64-10 block: 4 counter words, 2 key words -> 4 words."""
+    lib = _load()
+    c = (ctypes.c_uint64 * 4)(*[int(v) for v in ctr])
+    k = (ctypes.c_uint64 * 2)(*[int(v) for v in key])
+    o = (ctypes.c_uint64 * 4)()
+    lib.oracle_philox4x64_10(c, k, o)
+    return [int(v) for v in o]
 
 
 def num_threads() -> int:
@@ -122,7 +137,7 @@ def lstm_forward(x, w_ih, w_hh, b_ih=None, b_hh=None, h0=None, c0=None,
 
 def lstm_backward(x, w_ih, w_hh, grad_out, b_ih=None, b_hh=None, h0=None, c0=None,
                   grad_hn=None, grad_cn=None, num_layers=1, bidirectional=False,
-                  batch_first=True, lengths=None):
+                  batch_first=True, lengths=None, dropout=0.0, dropout_seed=0):
     """Forward + BPTT.  Returns a dict with out, h_n, c_n, dx, dh0, dc0 and the
     per-(layer, direction) lists dw_ih, dw_hh, db_ih, db_hh (float64)."""
     lib = _load()
@@ -152,7 +167,8 @@ def lstm_backward(x, w_ih, w_hh, grad_out, b_ih=None, b_hh=None, h0=None, c0=Non
     db_ih = [np.zeros(G) for _ in range(L * D)] if bias else None
     db_hh = [np.zeros(G) for _ in range(L * D)] if bias else None
     keep, lp = _lengths(lengths, B)
-    rc = lib.oracle_lstm_backward(L, D, I, H, B, T, int(bias), lp, _ptr(x), _ptr(h0), _ptr(c0),
+    rc = lib.oracle_lstm_backward(L, D, I, H, B, T, int(bias), lp, float(dropout), int(dropout_seed),
+                                  _ptr(x), _ptr(h0), _ptr(c0),
                                   _ptr_array(w_ih), _ptr_array(w_hh), _ptr_array(b_ih),
                                   _ptr_array(b_hh), _ptr(grad_out), _ptr(grad_hn), _ptr(grad_cn),
                                   _ptr(out), _ptr(h_n), _ptr(c_n), _ptr(dx), _ptr(dh0), _ptr(dc0),
@@ -175,6 +191,7 @@ def run_inputs(inp, backward=False):
               lengths=getattr(inp, "lengths", None))
     if backward:
         return lstm_backward(inp.x, inp.w_ih, inp.w_hh, inp.grad_out, grad_hn=inp.grad_hn,
-                             grad_cn=inp.grad_cn, **kw)
+                             grad_cn=inp.grad_cn, dropout=getattr(wl, "dropout", 0.0),
+                             dropout_seed=getattr(wl, "dropout_seed", 0), **kw)
     out, h_n, c_n = lstm_forward(inp.x, inp.w_ih, inp.w_hh, **kw)
     return dict(out=out, h_n=h_n, c_n=c_n)

@@ -52,11 +52,23 @@
  *    its first lengths[b] steps (the reverse direction starts at step
  *    lengths[b] - 1), its padded outputs are 0, h_n/c_n are its final states,
  *    the padding receives no gradient and contributes none.
+ *  - Inter-layer dropout in training ("Complete Trace: nn.LSTM", the dropout
+ *    argument of the LSTM op): with probability p each element of the output
+ *    of layers 0..L-2 is zeroed before it enters the next layer, survivors
+ *    are scaled by 1/(1-p); the last layer's output is not dropped.  The
+ *    pages fix no random stream, so this build fixes one: for boundary l,
+ *    element e = (t*B + b)*(D*H) + k of the time-major output sequence is kept
+ *    iff (w >> 11) >= ceil(p * 2^53), where w is word e mod 4 of
+ *    Philox4x64-10 (Salmon, Moraes, Dror, Shaw 2011, "Parallel random
+ *    numbers: as easy as 1, 2, 3") with key (seed, l) and counter
+ *    (floor(e/4), 0, 0, 0).  An integer decision, so every implementation
+ *    takes the same one.
  *
  * Layout of every array is row-major and batch-first as listed; the Python
  * wrapper converts seq-first data before calling.
  */
 #include <math.h>
+#include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
 #ifdef _OPENMP
@@ -85,11 +97,66 @@ void oracle_set_num_threads(int n) {
 
 static double sig(double z) { return 1.0 / (1.0 + exp(-z)); }
 
+/* ---------------------------------------------------------------- Philox
+ * Philox4x64-10 as defined by Salmon et al. (2011): ten rounds of
+ *   (R0, R1, R2, R3) -> (hi(M1*R2) ^ R1 ^ K0, lo(M1*R2), hi(M0*R0) ^ R3 ^ K1, lo(M0*R0))
+ * with the key bumped by the Weyl constants after every round. */
+static void mul_hilo64(uint64_t a, uint64_t b, uint64_t* hi, uint64_t* lo) {
+    const unsigned __int128 p = (unsigned __int128)a * b;
+    *hi = (uint64_t)(p >> 64);
+    *lo = (uint64_t)p;
+}
+
+void oracle_philox4x64_10(const uint64_t* ctr, const uint64_t* key, uint64_t* out) {
+    const uint64_t M0 = 0xD2E7470EE14C6C93ULL, M1 = 0xCA5A826395121157ULL;
+    const uint64_t W0 = 0x9E3779B97F4A7C15ULL, W1 = 0xBB67AE8584CAA73BULL;
+    uint64_t c0 = ctr[0], c1 = ctr[1], c2 = ctr[2], c3 = ctr[3], k0 = key[0], k1 = key[1];
+    for (int r = 0; r < 10; ++r) {
+        uint64_t hi0, lo0, hi1, lo1;
+        mul_hilo64(M0, c0, &hi0, &lo0);
+        mul_hilo64(M1, c2, &hi1, &lo1);
+        c0 = hi1 ^ c1 ^ k0;
+        c1 = lo1;
+        c2 = hi0 ^ c3 ^ k1;
+        c3 = lo0;
+        k0 += W0;
+        k1 += W1;
+    }
+    out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
+}
+
+/* Dropout decision for element e of boundary l (see the header comment). */
+static int dropout_keep(uint64_t seed, int l, uint64_t e, uint64_t thresh) {
+    const uint64_t ctr[4] = {e >> 2, 0, 0, 0};
+    const uint64_t key[2] = {seed, (uint64_t)l};
+    uint64_t w[4];
+    oracle_philox4x64_10(ctr, key, w);
+    return (w[e & 3] >> 11) >= thresh;
+}
+
 /* Problem description shared by the entry points. */
 typedef struct {
     int L, D, I, H, B, T, bias;
     const int* lengths;   /* [B] valid steps per row, or NULL (all T) */
+    double dropout;       /* inter-layer dropout probability (training), 0 = none */
+    uint64_t seed;
 } prob;
+
+static uint64_t dropout_thresh(double p) { return (uint64_t)ceil(p * 9007199254740992.0); /* p * 2^53 */ }
+
+/* Row b's output sequence of layer l ([T][D*H]) as the next layer's input:
+ * multiplied by the dropout mask over 1-p (training, l < L-1, p > 0). */
+static void apply_dropout(const prob* p, int l, int b, double* seq) {
+    if (!(p->dropout > 0.0) || l >= p->L - 1) return;
+    const int DH = p->D * p->H;
+    const uint64_t th = dropout_thresh(p->dropout);
+    const double scale = 1.0 / (1.0 - p->dropout);
+    for (int t = 0; t < p->T; ++t)
+        for (int k = 0; k < DH; ++k) {
+            const uint64_t e = ((uint64_t)t * p->B + b) * DH + k;
+            seq[(size_t)t * DH + k] *= dropout_keep(p->seed, l, e, th) ? scale : 0.0;
+        }
+}
 
 /* Valid steps of row b. */
 static int row_len(const prob* p, int b) { return p->lengths ? p->lengths[b] : p->T; }
@@ -191,6 +258,7 @@ static int forward_row(const prob* p, int b,
                 if (c_n) c_n[((size_t)ld * B + b) * H + u] = c[u];
             }
         }
+        apply_dropout(p, l, b, nxt);   /* what the next layer reads */
         cur = nxt;
     }
     if (out) memcpy(out + (size_t)b * T * D * H, cur, sizeof(double) * (size_t)T * D * H);
@@ -219,7 +287,7 @@ int oracle_lstm_forward(int L, int D, int I, int H, int B, int T, int bias, cons
                         const double* const* b_ih, const double* const* b_hh,
                         double* out, double* h_n, double* c_n)
 {
-    prob p = {L, D, I, H, B, T, bias, lengths};
+    prob p = {L, D, I, H, B, T, bias, lengths, 0.0, 0};
     if (check_prob(&p)) return ORACLE_ERR_ARG;
     int err = 0;
 #pragma omp parallel for schedule(dynamic, 1) reduction(|:err)
@@ -336,7 +404,10 @@ static int backward_row(const prob* p, int b, const row_record* rec,
                 dc0[((size_t)ld * B + b) * H + u] = dc[u];
             }
         }
-        if (l > 0) memcpy(dy, din, sizeof(double) * (size_t)T * in);
+        if (l > 0) {
+            memcpy(dy, din, sizeof(double) * (size_t)T * in);
+            apply_dropout(p, l - 1, b, dy);   /* the same mask carries the gradient back */
+        }
         else memcpy(dx + (size_t)b * T * p->I, din, sizeof(double) * (size_t)T * p->I);
     }
     free(dy); free(din); free(dh); free(dc); free(dhn);
@@ -348,10 +419,11 @@ static int backward_row(const prob* p, int b, const row_record* rec,
  * [B][T][D*H] and grad_hn, grad_cn [L*D][B][H] (NULL = zeros).  Outputs:
  * out, h_n, c_n (may be NULL), dx [B][T][I], dh0, dc0 [L*D][B][H],
  * dw_ih[l*D+d] [4H][in_l], dw_hh [4H][H], db_ih, db_hh [4H] (bias only).
- * The weight gradients are overwritten, not accumulated.
+ * The weight gradients are overwritten, not accumulated.  dropout in [0, 1)
+ * and seed select the inter-layer dropout of the training forward.
  */
 int oracle_lstm_backward(int L, int D, int I, int H, int B, int T, int bias, const int* lengths,
-                         const double* x, const double* h0, const double* c0,
+                         double dropout, uint64_t seed, const double* x, const double* h0, const double* c0,
                          const double* const* w_ih, const double* const* w_hh,
                          const double* const* b_ih, const double* const* b_hh,
                          const double* grad_out, const double* grad_hn, const double* grad_cn,
@@ -360,8 +432,9 @@ int oracle_lstm_backward(int L, int D, int I, int H, int B, int T, int bias, con
                          double* const* dw_ih, double* const* dw_hh,
                          double* const* db_ih, double* const* db_hh)
 {
-    prob p = {L, D, I, H, B, T, bias, lengths};
+    prob p = {L, D, I, H, B, T, bias, lengths, dropout, seed};
     if (check_prob(&p)) return ORACLE_ERR_ARG;
+    if (!(dropout >= 0.0 && dropout < 1.0)) return ORACLE_ERR_ARG;
     const int G = 4 * H, LD = L * D;
     row_record* recs = (row_record*)calloc((size_t)B + 1, sizeof(row_record));
     double*** da = (double***)calloc((size_t)B + 1, sizeof(double**));

@@ -428,3 +428,72 @@ def test_varlen_empty_row_keeps_initial_state():
     np.testing.assert_array_equal(r["c_n"][:, 1], inp.c0[:, 1])
     np.testing.assert_array_equal(r["dh0"][:, 1], inp.grad_hn[:, 1])
     np.testing.assert_array_equal(r["dc0"][:, 1], inp.grad_cn[:, 1])
+
+
+# ------------------------------------------------ inter-layer dropout (training)
+def test_philox_matches_numpy():
+    """The oracle's Philox4x64-10 against numpy's independent implementation
+    of the same published generator (numpy advances its counter by one
+    before the first block it returns)."""
+    for ctr, key in [([1, 0, 0, 0], [0, 0]), ([2, 0, 0, 0], [0x1234, 5]),
+                     ([7, 3, 0, 9], [2 ** 64 - 1, 17]), ([2 ** 40 + 5, 0, 0, 0], [99, 0])]:
+        bg = np.random.Philox(key=np.array(key, dtype=np.uint64),
+                              counter=np.array([ctr[0] - 1] + ctr[1:], dtype=np.uint64))
+        want = [int(v) for v in bg.random_raw(4)]
+        assert oracle.philox4x64_10(ctr, key) == want, (ctr, key)
+
+
+def _numpy_keep_mask(seed, layer, T, B, DH, p):
+    """keep[t, b, k] from numpy's Philox: word e mod 4 of the block at counter
+    floor(e/4), key (seed, layer), compared as integers with ceil(p * 2^53)."""
+    n = T * B * DH
+    nblk = (n + 3) // 4
+    bg = np.random.Philox(key=np.array([seed, layer], dtype=np.uint64),
+                          counter=np.array([2 ** 64 - 1, 2 ** 64 - 1, 2 ** 64 - 1, 2 ** 64 - 1],
+                                           dtype=np.uint64))   # +1 wraps to counter 0
+    words = bg.random_raw(4 * nblk)[:n]
+    thresh = math.ceil(p * 2.0 ** 53)
+    return ((words >> np.uint64(11)) >= np.uint64(thresh)).reshape(T, B, DH)
+
+
+@pytest.mark.parametrize("D", [1, 2])
+def test_dropout_equals_chained_layers_with_an_independent_mask(D):
+    """A 2-layer training run with inter-layer dropout p equals: layer 0 run
+    alone, its output multiplied by a mask drawn with numpy's Philox over
+    (1 - p), layer 1 run alone on that; gradients likewise chained through
+    the same mask."""
+    p, seed = 0.35, 0xC0FFEE
+    wl = Workload("dr", L=2, D=D, I=3, H=4, T=5, B=3, dtype="f32", state_std=0.3, train=True,
+                  seed=61, dropout=p, dropout_seed=seed)
+    inp = make_inputs(wl)
+    rng = np.random.default_rng(61)
+    inp.grad_hn = rng.standard_normal((2 * D, 3, 4)).astype(np.float32)
+    r = oracle.run_inputs(inp, backward=True)
+    keep = _numpy_keep_mask(seed, 0, wl.T, wl.B, D * wl.H, p).transpose(1, 0, 2)   # [B][T][DH]
+    m = keep / (1.0 - p)
+    s0, s1 = slice(0, D), slice(D, 2 * D)
+    kw0 = dict(b_ih=inp.b_ih[s0], b_hh=inp.b_hh[s0], h0=inp.h0[s0], c0=inp.c0[s0], bidirectional=D == 2)
+    kw1 = dict(b_ih=inp.b_ih[s1], b_hh=inp.b_hh[s1], h0=inp.h0[s1], c0=inp.c0[s1], bidirectional=D == 2)
+    out0, _, _ = oracle.lstm_forward(inp.x, inp.w_ih[s0], inp.w_hh[s0], **kw0)
+    r1 = oracle.lstm_backward(out0 * m, inp.w_ih[s1], inp.w_hh[s1], inp.grad_out,
+                              grad_hn=inp.grad_hn[s1], **kw1)
+    r0 = oracle.lstm_backward(inp.x, inp.w_ih[s0], inp.w_hh[s0], r1["dx"] * m,
+                              grad_hn=inp.grad_hn[s0], **kw0)
+    assert 0 < keep.mean() < 1
+    np.testing.assert_allclose(r["out"], r1["out"], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(r["h_n"], np.concatenate([r0["h_n"], r1["h_n"]]), rtol=0, atol=1e-13)
+    np.testing.assert_allclose(r["dx"], r0["dx"], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(r["dh0"], np.concatenate([r0["dh0"], r1["dh0"]]), rtol=0, atol=1e-13)
+    for k in ("dw_ih", "dw_hh", "db_ih"):
+        for a, b in zip(r[k], r0[k] + r1[k]):
+            np.testing.assert_allclose(a, b, rtol=0, atol=1e-13, err_msg=k)
+
+
+def test_dropout_zero_is_no_dropout():
+    wl = Workload("dr0", L=2, D=2, I=3, H=4, T=4, B=2, dtype="f32", state_std=0.3, train=True, seed=62)
+    inp = make_inputs(wl)
+    a = oracle.run_inputs(inp, backward=True)
+    inp.wl = wl.replace(dropout=0.0, dropout_seed=123)
+    b = oracle.run_inputs(inp, backward=True)
+    for k in ("out", "dx", "dh0"):
+        np.testing.assert_array_equal(a[k], b[k])
