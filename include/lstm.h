@@ -89,6 +89,16 @@ typedef struct {
     int batch;          /* B >= 0 */
     int seq_len;        /* T >= 0; T == 0 gives h_n = h0, c_n = c0 */
     lstm_dtype dtype;
+    /* Inter-layer dropout of the training forward ([trace] Step 3: the
+     * dropout argument of the LSTM op), 0 <= dropout < 1; 0 = none.  Applied
+     * only when lstm_forward gets a reserve, to the outputs of layers
+     * 0..L-2 before they enter the next layer; the backward replays the
+     * same mask.  Element e = (t*B + b)*(D*H) + k of layer l's time-major
+     * output is kept iff (w >> 11) >= ceil(dropout * 2^53), w = word e mod 4
+     * of Philox4x64-10 (Salmon et al. 2011) with key (dropout_seed, l) and
+     * counter (e / 4, 0, 0, 0); kept elements are scaled by 1/(1-dropout). */
+    float dropout;
+    unsigned long long dropout_seed;
 } lstm_desc;
 
 /* Workspace bytes needed by lstm_forward and lstm_backward for this

@@ -42,13 +42,16 @@ class lstm_desc(ctypes.Structure):
     _fields_ = [("input_size", ctypes.c_int), ("hidden_size", ctypes.c_int),
                 ("num_layers", ctypes.c_int), ("bidirectional", ctypes.c_int),
                 ("bias", ctypes.c_int), ("batch_first", ctypes.c_int),
-                ("batch", ctypes.c_int), ("seq_len", ctypes.c_int), ("dtype", ctypes.c_int)]
+                ("batch", ctypes.c_int), ("seq_len", ctypes.c_int), ("dtype", ctypes.c_int),
+                ("dropout", ctypes.c_float), ("dropout_seed", ctypes.c_ulonglong)]
 
 
 def make_desc(input_size, hidden_size, num_layers=1, bidirectional=False, bias=True,
-              batch_first=True, batch=1, seq_len=1, dtype=LSTM_F32) -> lstm_desc:
+              batch_first=True, batch=1, seq_len=1, dtype=LSTM_F32, dropout=0.0,
+              dropout_seed=0) -> lstm_desc:
     return lstm_desc(int(input_size), int(hidden_size), int(num_layers), int(bool(bidirectional)),
-                     int(bool(bias)), int(bool(batch_first)), int(batch), int(seq_len), int(dtype))
+                     int(bool(bias)), int(bool(batch_first)), int(batch), int(seq_len), int(dtype),
+                     float(dropout), int(dropout_seed))
 
 
 _lib = None

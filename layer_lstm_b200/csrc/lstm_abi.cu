@@ -15,6 +15,7 @@
 
 #include <algorithm>
 #include <mutex>
+#include <cmath>
 #include <vector>
 
 #include "../../include/lstm.h"
@@ -64,12 +65,23 @@ uint64_t timeout_ns() {
 // CUDA cores.
 enum Kind {
     K_PACK = 0, K_PROJ_TC, K_PROJ_SIMT, K_FWD_REC_TC, K_FWD_REC_FFMA, K_BWD_REC_FFMA, K_DW_TC, K_DW_SIMT,
-    K_DX_TC, K_DX_SIMT, K_DB, K_COPY, K_TRANSPOSE, K_COUNT
+    K_DX_TC, K_DX_SIMT, K_DB, K_COPY, K_TRANSPOSE, K_DROPOUT, K_COUNT
 };
 const char* const kKindNames[K_COUNT] = {"pack",       "proj_gemm_tc", "proj_gemm_simt", "fwd_rec_tc",
                                          "fwd_rec_ffma", "bwd_rec_ffma", "dw_gemm_tc",   "dw_gemm_simt",
                                          "dx_gemm_tc", "dx_gemm_simt", "db_reduce",    "seq_copy",
-                                         "transpose"};
+                                         "transpose",  "dropout"};
+
+// Dropout launch for boundary `layer` over n time-major elements.
+DropoutArgs dropout_args(const lstm_desc* d, int layer, const void* src, void* dst, DType dt, long long n) {
+    DropoutArgs a{};
+    const double p = d->dropout;
+    a.n = n; a.src = src; a.dst = dst; a.dt = dt;
+    a.seed = d->dropout_seed; a.layer = layer;
+    a.thresh = (unsigned long long)ceil(p * 9007199254740992.0);   // p * 2^53
+    a.scale = (float)(1.0 / (1.0 - p));
+    return a;
+}
 
 struct Timing {
     std::mutex mu;
@@ -156,6 +168,8 @@ struct Layout {
     size_t s_x, s_h0, s_gout, s_ghn, s_hs[2], s_dx, s_dh0, s_wih[32];
     // reserve offsets
     size_t act[32], cst[32], hseq[32], rtotal;   // per layer: [D][T][B][G], [D][T][B][H], [T][B][D*H]
+    size_t hdrop[32];   // layers 0..L-2 with dropout: the next layer's input, [T][B][D*H]
+    float dropout;
 };
 
 int in_size(const Layout& l, int layer) { return layer == 0 ? l.I : l.D * l.H; }
@@ -167,6 +181,7 @@ bool valid_desc(const lstm_desc* d) {
     if (d->bidirectional != 0 && d->bidirectional != 1) return false;
     if (d->batch < 0 || d->seq_len < 0) return false;
     if (d->dtype != LSTM_F32 && d->dtype != LSTM_BF16) return false;
+    if (!(d->dropout >= 0.f && d->dropout < 1.f)) return false;   // also rejects NaN
     // sizes addressed with 32-bit loop counters inside kernels
     const long long H = d->hidden_size, I = d->input_size;
     if (H > (1 << 16) || I > (1 << 20)) return false;
@@ -256,6 +271,11 @@ bool make_layout(const lstm_desc* d, Layout& l) {
         l.act[k] = r; r += al((size_t)l.D * TB * l.G * 4);
         l.cst[k] = r; r += al((size_t)l.D * TB * l.H * 4);
         l.hseq[k] = r; r += al(TB * l.D * l.H * l.es);
+    }
+    l.dropout = d->dropout;
+    for (int k = 0; k < l.L; ++k) {
+        const bool dropped = l.dropout > 0.f && k < l.L - 1;
+        l.hdrop[k] = r; r += al(dropped ? TB * l.D * l.H * l.es : 0);
     }
     l.rtotal = r;
     return true;
@@ -580,6 +600,12 @@ lstm_status lstm_forward_varlen(const lstm_desc* desc, const int* lengths, const
         f.len = lengths;
         LSTM_CUDA(timed(K_FWD_REC_FFMA, stream, [&] { return launch_fwd_rec(f, stream); }));
         layer_in = hseq;
+        if (reserve && l.dropout > 0.f && k < L - 1) {
+            void* dropped = P(reserve, l.hdrop[k]);
+            const DropoutArgs da = dropout_args(desc, k, hseq, dropped, l.dt, (long long)B * T * D * H);
+            LSTM_CUDA(timed(K_DROPOUT, stream, [&] { return launch_dropout(da, stream); }));
+            layer_in = dropped;
+        }
     }
     return LSTM_OK;
 }
@@ -677,17 +703,16 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
             wihf[i] = stage(w_ih[i], bf ? l.s_wih[k] + (size_t)d * nih * 4 : 0, nih);
             if (!wihf[i]) return LSTM_ERR_CUDA;
         }
-    // float32 output sequence of layer k, saved by the forward in the reserve
-    auto layer_out = [&](int k) -> const float* {
-        const void* src = static_cast<const char*>(reserve) + l.hseq[k];
-        return bf ? reinterpret_cast<const float*>(P(workspace, l.s_hs[k & 1])) : static_cast<const float*>(src);
+    // A sequence the forward saved in the reserve ([T][B][D*H]) as float32:
+    // itself, or (bf16) its copy in staging slot `slot`.
+    auto saved_seq = [&](size_t roff, int slot) -> const float* {
+        const void* src = static_cast<const char*>(reserve) + roff;
+        if (!bf) return static_cast<const float*>(src);
+        float* dst = reinterpret_cast<float*>(P(workspace, l.s_hs[slot]));
+        return launch_convert(src, DType::BF16, dst, DType::F32, (long long)(BTs * D * H), stream) == cudaSuccess
+                   ? dst : nullptr;
     };
-    auto stage_layer_out = [&](int k) -> bool {
-        if (!bf) return true;
-        return launch_convert(static_cast<const char*>(reserve) + l.hseq[k], DType::BF16, P(workspace, l.s_hs[k & 1]),
-                              DType::F32, (long long)(BTs * D * H), stream) == cudaSuccess;
-    };
-    if (!stage_layer_out(L - 1)) return LSTM_ERR_CUDA;
+    const bool dropped = l.dropout > 0.f;   // layer k > 0 read the dropped output of layer k - 1
     float* dh0f = bf ? reinterpret_cast<float*>(P(workspace, l.s_dh0)) : static_cast<float*>(dh0);
     float* dxf = bf ? reinterpret_cast<float*>(P(workspace, l.s_dx)) : static_cast<float*>(dx);
     // time-major copy of x for the layer-0 weight gradient
@@ -710,7 +735,6 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
         pb.H = H; pb.D = D; pb.nu = l.bwd.nu; pb.U = l.bwd.U;
         pb.dt = l.dt;
         for (int d = 0; d < D; ++d) pb.w[d] = w_hh[k * D + d];
-        if (k > 0 && !stage_layer_out(k - 1)) return LSTM_ERR_CUDA;
         pb.out = P(workspace, l.whh_b);
         LSTM_CUDA(timed(K_PACK, stream, [&] { return launch_pack_hh_rows(pb, stream); }));
 
@@ -742,8 +766,9 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
             for (int d = 0; d < D; ++d) { db.db_ih[d] = db_ih[k * D + d]; db.db_hh[d] = db_hh[k * D + d]; }
             LSTM_CUDA(timed(K_DB, stream, [&] { return launch_db_reduce(db, stream); }));
         }
-        const float* layer_in = k == 0 ? x_tm : layer_out(k - 1);
-        const float* hs = layer_out(k);
+        const float* layer_in = k == 0 ? x_tm : saved_seq(dropped ? l.hdrop[k - 1] : l.hseq[k - 1], 1);
+        const float* hs = saved_seq(l.hseq[k], 0);
+        if (!layer_in || !hs) return LSTM_ERR_CUDA;
         const long long ldg = (long long)D * G, ldh = (long long)D * H;
         const long long BTl = (long long)B * T;
         float* din = k == 0 ? dxf : reinterpret_cast<float*>(P(workspace, l.dseq[cur]));
@@ -778,7 +803,7 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
                     ti.src = xf; ti.lds = in;
                     ti.bt_remap = desc->batch_first; ti.T = T; ti.B = B;
                 } else {
-                    ti.src = layer_out(k - 1);
+                    ti.src = layer_in;
                     ti.lds = in;
                 }
                 ti.dst = bo; ti.ldd = BTl;
@@ -850,6 +875,10 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
                 if (k == 0 && desc->batch_first) { g.remap_T = -T; g.remap_B = B; }
                 LSTM_CUDA(timed(K_DX_SIMT, stream, [&] { return launch_gemm(g, stream); }));
             }
+        }
+        if (k > 0 && dropped) {   // through the dropout mask to layer k - 1's output
+            const DropoutArgs da = dropout_args(desc, k - 1, din, din, DType::F32, (long long)BTl * in);
+            LSTM_CUDA(timed(K_DROPOUT, stream, [&] { return launch_dropout(da, stream); }));
         }
         if (k > 0) {
             dy = din;

@@ -210,6 +210,18 @@ struct SeqCopyArgs {
 };
 cudaError_t launch_seq_copy(const SeqCopyArgs& a, cudaStream_t s);
 
+// Inter-layer dropout: dst[e] = keep(e) ? src[e] * scale : 0 for e < n (src
+// may equal dst), keep(e) = (w >> 11) >= thresh with w word e mod 4 of
+// Philox4x64-10 at key (seed, layer), counter (e / 4, 0, 0, 0).
+struct DropoutArgs {
+    long long n;
+    const void* src; void* dst; DType dt;
+    unsigned long long seed; int layer;
+    unsigned long long thresh;   // ceil(p * 2^53)
+    float scale;                 // 1 / (1 - p)
+};
+cudaError_t launch_dropout(const DropoutArgs& a, cudaStream_t s);
+
 // dst[i] = src[i] for i < n, converting between float and bf16 (nearest even).
 cudaError_t launch_convert(const void* src, DType st, void* dst, DType dt, long long n, cudaStream_t s);
 

@@ -205,6 +205,44 @@ __global__ void seq_copy_kernel(SeqCopyArgs a) {
     }
 }
 
+// Philox4x64-10, Salmon, Moraes, Dror, Shaw (2011), "Parallel random numbers:
+// as easy as 1, 2, 3": ten rounds of
+//   (R0, R1, R2, R3) -> (hi(M1 R2) ^ R1 ^ K0, lo(M1 R2), hi(M0 R0) ^ R3 ^ K1, lo(M0 R0))
+// with the key advanced by the Weyl constants after each round.
+__device__ __forceinline__ void philox4x64_10(uint64_t c[4], uint64_t k0, uint64_t k1) {
+    const uint64_t M0 = 0xD2E7470EE14C6C93ull, M1 = 0xCA5A826395121157ull;
+    const uint64_t W0 = 0x9E3779B97F4A7C15ull, W1 = 0xBB67AE8584CAA73Bull;
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        const uint64_t hi0 = __umul64hi(M0, c[0]), lo0 = M0 * c[0];
+        const uint64_t hi1 = __umul64hi(M1, c[2]), lo1 = M1 * c[2];
+        const uint64_t n0 = hi1 ^ c[1] ^ k0, n2 = hi0 ^ c[3] ^ k1;
+        c[0] = n0; c[1] = lo1; c[2] = n2; c[3] = lo0;
+        k0 += W0;
+        k1 += W1;
+    }
+}
+
+// One Philox block per thread iteration: four consecutive elements.
+template <typename T>
+__global__ void dropout_kernel(DropoutArgs a) {
+    const T* src = static_cast<const T*>(a.src);
+    T* dst = static_cast<T*>(a.dst);
+    const long long nblk = (a.n + 3) / 4;
+    for (long long q = blockIdx.x * (long long)blockDim.x + threadIdx.x; q < nblk;
+         q += (long long)gridDim.x * blockDim.x) {
+        uint64_t w[4] = {(uint64_t)q, 0, 0, 0};
+        philox4x64_10(w, a.seed, (uint64_t)a.layer);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const long long e = 4 * q + j;
+            if (e >= a.n) break;
+            const bool keep = (w[j] >> 11) >= a.thresh;
+            dst[e] = from_f<T>(keep ? to_f(src[e]) * a.scale : 0.f);
+        }
+    }
+}
+
 // dst[i] = src[i] converted (float <-> bf16, round to nearest even)
 template <typename S, typename D>
 __global__ void convert_kernel(const S* __restrict__ src, D* __restrict__ dst, long long n) {
@@ -223,6 +261,16 @@ cudaError_t launch_convert(const void* src, DType st, void* dst, DType dt, long 
         convert_kernel<<<grid_for(n), 256, 0, s>>>(static_cast<const float*>(src), static_cast<bf16*>(dst), n);
     else
         return cudaMemcpyAsync(dst, src, (size_t)n * dtype_size(st), cudaMemcpyDeviceToDevice, s);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dropout(const DropoutArgs& a, cudaStream_t s) {
+    if (a.n <= 0) return cudaSuccess;
+    const long long nblk = (a.n + 3) / 4;
+    if (a.dt == DType::F32)
+        dropout_kernel<float><<<grid_for(nblk), 256, 0, s>>>(a);
+    else
+        dropout_kernel<bf16><<<grid_for(nblk), 256, 0, s>>>(a);
     return cudaGetLastError();
 }
 

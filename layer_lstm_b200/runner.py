@@ -18,7 +18,8 @@ def torch_dtype(wl: Workload):
 
 def desc_for(wl: Workload) -> binding.lstm_desc:
     return binding.make_desc(wl.I, wl.H, wl.L, wl.D == 2, wl.bias, wl.batch_first, wl.B, wl.T,
-                             binding.LSTM_F32 if wl.dtype == "f32" else binding.LSTM_BF16)
+                             binding.LSTM_F32 if wl.dtype == "f32" else binding.LSTM_BF16,
+                             wl.dropout, wl.dropout_seed)
 
 
 class DeviceProblem:

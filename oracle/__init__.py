@@ -191,7 +191,8 @@ def run_inputs(inp, backward=False):
               lengths=getattr(inp, "lengths", None))
     if backward:
         return lstm_backward(inp.x, inp.w_ih, inp.w_hh, inp.grad_out, grad_hn=inp.grad_hn,
-                             grad_cn=inp.grad_cn, dropout=getattr(wl, "dropout", 0.0),
+                             # the library's descriptor holds the probability as a float32
+                             grad_cn=inp.grad_cn, dropout=float(np.float32(getattr(wl, "dropout", 0.0))),
                              dropout_seed=getattr(wl, "dropout_seed", 0), **kw)
     out, h_n, c_n = lstm_forward(inp.x, inp.w_ih, inp.w_hh, **kw)
     return dict(out=out, h_n=h_n, c_n=c_n)

@@ -462,7 +462,7 @@ def test_dropout_equals_chained_layers_with_an_independent_mask(D):
     alone, its output multiplied by a mask drawn with numpy's Philox over
     (1 - p), layer 1 run alone on that; gradients likewise chained through
     the same mask."""
-    p, seed = 0.35, 0xC0FFEE
+    p, seed = float(np.float32(0.35)), 0xC0FFEE   # the descriptor carries p as a float32
     wl = Workload("dr", L=2, D=D, I=3, H=4, T=5, B=3, dtype="f32", state_std=0.3, train=True,
                   seed=61, dropout=p, dropout_seed=seed)
     inp = make_inputs(wl)

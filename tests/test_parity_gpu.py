@@ -123,6 +123,13 @@ TRAIN = {
                                  batch_first=False, train=True, seed=143),
     "bf16_long": Workload("s", L=2, D=1, I=32, H=64, T=64, B=8, dtype="bf16", state_std=0.3,
                           train=True, seed=144),
+    # inter-layer dropout (Philox4x64-10 mask; identical decisions on both sides)
+    "f32_dropout_3layer": Workload("s", L=3, D=1, I=20, H=40, T=7, B=9, dtype="f32", state_std=0.3,
+                                   train=True, dropout=0.3, dropout_seed=77, seed=151),
+    "f32_dropout_bi": Workload("s", L=2, D=2, I=16, H=36, T=6, B=10, dtype="f32", state_std=0.3,
+                               train=True, dropout=0.5, dropout_seed=2 ** 63 + 5, seed=152),
+    "bf16_dropout_varlen": Workload("s", L=2, D=2, I=32, H=64, T=8, B=12, dtype="bf16", state_std=0.3,
+                                    train=True, dropout=0.25, dropout_seed=9, varlen=True, seed=153),
     # c3's layer shapes (H = 1024, bidirectional, 2 layers) on a short sequence
     "bf16_c3_shape": Workload("s", L=2, D=2, I=512, H=1024, T=12, B=8, dtype="bf16", w_k=1 / 32,
                               train=True, seed=145),
