@@ -49,6 +49,17 @@ __host__ __device__ constexpr int tile_cols_wn(int nNT) {
     return nNT >= 128 / (4 * TN) ? 128 / (4 * TN) : (nNT >= 4 ? 4 : (nNT >= 2 ? 2 : 1));
 }
 
+// c0 += a * b0, c1 += a * b1 as one packed instruction (two IEEE fused
+// multiply-adds, each rounded exactly as fmaf).
+__device__ __forceinline__ void ffma2(float& c0, float& c1, float a, float b0, float b1) {
+    asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+        "mov.b64 ra, {%2, %2};\n\tmov.b64 rb, {%3, %4};\n\tmov.b64 rc, {%0, %1};\n\t"
+        "fma.rn.f32x2 rc, ra, rb, rc;\n\t"
+        "mov.b64 {%0, %1}, rc;\n\t}"
+        : "+f"(c0), "+f"(c1)
+        : "f"(a), "f"(b0), "f"(b1));
+}
+
 template <int TN, typename AT, typename XT, typename St>
 __device__ __forceinline__ void block_mm(const AT* __restrict__ A, int lda, const XT* __restrict__ X,
                                          int ldx, int R, int N, int K, int KS, St&& st) {
@@ -92,7 +103,7 @@ __device__ __forceinline__ void block_mm(const AT* __restrict__ A, int lda, cons
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
 #pragma unroll
-                    for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(a[q][i], x[q][j], acc[i][j]);
+                    for (int j = 0; j < TN; j += 2) ffma2(acc[i][j], acc[i][j + 1], a[q][i], x[q][j], x[q][j + 1]);
         }
         st(ks, rt * 4, nt * TN, acc);
     }
