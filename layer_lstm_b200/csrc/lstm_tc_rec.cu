@@ -14,9 +14,9 @@
 // the MMAs of its half only, so the serial chain of MMA instructions per step
 // is half as long as with one block per slice.  Each block owns half of the N
 // columns: it sends its partial sums of the partner's columns into the
-// partner's shared memory (distributed shared memory stores, then a remote
-// mbarrier arrive), adds the partner's partial sums of its own columns, and
-// updates c and h there.  One step:
+// partner's shared memory (asynchronous distributed-shared-memory stores that
+// complete on the partner's mbarrier), adds the partner's partial sums of its
+// own columns, and updates c and h there.  One step:
 //   warp 0:     wait for the group's h_{t-1}, TMA this block's K chunks of it
 //               (N rows x 64 k each) through a ring of shared-memory stages
 //   warp 1:     once the accumulator holds Gx[t] in the own columns and zero
@@ -128,15 +128,13 @@ __device__ __forceinline__ uint32_t map_rank(uint32_t saddr, uint32_t rank) {
     return r;
 }
 
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
-    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+// Asynchronous 16-byte store into another block of the cluster; its bytes
+// count against the transaction count of that block's mbarrier remote_bar,
+// so the storing thread does not wait for it to land.
+__device__ __forceinline__ void st_async_v4(uint32_t addr, float a, float b, float c, float d, uint32_t remote_bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
+                 ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d), "r"(remote_bar)
                  : "memory");
-}
-
-// Arrive on an mbarrier of another block of the cluster, releasing this
-// thread's earlier distributed-shared-memory stores at cluster scope.
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t remote_bar) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
@@ -298,7 +296,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mbar_init(d_ready, kEpi);
         tc::mbar_init(mma_done, 1);
         tc::mbar_init(w_full, 1);
-        tc::mbar_init(recv_full, kEpi);               // one arrive per epilogue thread of the partner
+        tc::mbar_init(recv_full, 1);                  // armed each step with the partner's bytes
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
@@ -442,6 +440,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         preload_gx(a.gx, d == 0 ? 0 : T - 1, B, ldgx, prow0 + r, b0, own0, pcol0, ncc, nB, half, trow, d_ready);
         for (int s = 0; s < T; ++s) {
             const int t = d == 0 ? s : T - 1 - s;
+            // this step's phase of recv_full completes when the partner's
+            // partial sums of the own columns (NH x 128 floats) have landed;
+            // the previous phase completed before this thread left step s-1
+            if (e == 0) tc::mbar_arrive_expect_tx(recv_full, (uint32_t)(NH * kRows * 4));
             // Gx[t_next] of the own columns into L2 while the MMAs run
             if (s + 1 < T && e < NH && own0 + e < nB) {
                 const int tn = d == 0 ? s + 1 : T - 2 - s;
@@ -469,11 +471,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (cc >= ncc) break;
 #pragma unroll
                     for (int m = 0; m < 4; ++m)
-                        st_cluster_v4(recv_remote + (uint32_t)(((4 * cc + m) * kRows + r) * 16), pv[kk][4 * m],
-                                      pv[kk][4 * m + 1], pv[kk][4 * m + 2], pv[kk][4 * m + 3]);
+                        st_async_v4(recv_remote + (uint32_t)(((4 * cc + m) * kRows + r) * 16), pv[kk][4 * m],
+                                    pv[kk][4 * m + 1], pv[kk][4 * m + 2], pv[kk][4 * m + 3], recv_bar_remote);
                 }
             }
-            mbar_arrive_remote(recv_bar_remote);
             trace_mark(a.trace, tr2, s, 5);
             // 2) the partner's partial sums of the own columns
             const bool got = mbar_wait_cluster(recv_full, s & 1, abort_flag, a.status, a.timeout_ns);
