@@ -75,12 +75,15 @@ __device__ __forceinline__ void trace_mark(unsigned long long* trace, bool who, 
 
 // Block-wide arrival on a counter: every thread's prior global writes are
 // made visible at GPU scope before the count moves.
+// *ctr += v with release semantics at GPU scope: everything the block wrote
+// before the preceding barrier is visible to whoever acquires the new value.
+__device__ __forceinline__ void red_release_add(unsigned* ctr, unsigned v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(ctr), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ void block_arrive(unsigned* ctr) {
     __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        atomicAdd(ctr, 1u);
-    }
+    if (threadIdx.x == 0) red_release_add(ctr, 1u);
 }
 
 // Block-wide bounded wait until *ctr >= target.  Returns false (for every
@@ -105,8 +108,7 @@ __device__ __forceinline__ bool block_wait_geq(const unsigned* ctr, unsigned tar
                 }
             }
         }
-        __threadfence();
-        ok_s = ok;
+        ok_s = ok;   // the acquire loads above order what follows
     }
     __syncthreads();
     return ok_s != 0;

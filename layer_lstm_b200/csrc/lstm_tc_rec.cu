@@ -579,8 +579,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::fence_proxy_async_global();
             tc::named_bar_sync(1, kEpi);
             if (warp == 2 && lane == 0) {
-                __threadfence();
-                atomicAdd(ctr, 1u);
+                red_release_add(ctr, 1u);
             }
             trace_mark(a.trace, tr2, s, 8);
             if (s + 1 < T) {
