@@ -120,7 +120,9 @@ size_t lstm_reserve_size(const lstm_desc* desc);
  *     256-byte aligned.
  *   reserve/rs_bytes: NULL for inference; otherwise at least
  *     lstm_reserve_size bytes, filled for lstm_backward.
- * Enqueued on `stream`; returns before the GPU finishes.
+ * Enqueued on `stream`; returns before the GPU finishes.  Only
+ * stream-ordered work is enqueued (no host synchronisation), so a call may be
+ * captured into a CUDA graph and replayed.
  */
 lstm_status lstm_forward(const lstm_desc* desc, const void* x, const void* h0, const float* c0,
                          const void* const* w_ih, const void* const* w_hh,
