@@ -51,6 +51,118 @@ def parse_args():
     return ap.parse_args()
 
 
+def _io_tensors(wl, prob):
+    """(inputs a user copies in per step, results read back per step)."""
+    h_in = {"x": prob.x, "h0": prob.h0, "c0": prob.c0}
+    if wl.train:
+        h_in["grad_out"] = prob.grad_out
+    h_in = {k: v for k, v in h_in.items() if v is not None}
+    outs = [prob.out, prob.h_n, prob.c_n]
+    if wl.train:
+        outs += [prob.dx, prob.dh0, prob.dc0] + prob.dw_ih + prob.dw_hh + \
+            (prob.db_ih + prob.db_hh if wl.bias else [])
+    return h_in, outs
+
+
+def measure_e2e(args, wl, inp, prob, step, flush, stream, rank, world, local):
+    """Same metric through the public API with host buffers: every step copies
+    its inputs from pinned host memory and reads its results back.  One GPU:
+    two problem instances alternate, so step i+1's input copy and step i's
+    result copy (copy streams) overlap step i+1's / step i's compute; the time
+    is the device span of all steps (L2 flushes included).  Several ranks: the
+    copies and the step run back to back on the compute stream, timed per
+    step, max over ranks."""
+    import torch
+    import torch.distributed as dist
+    from layer_lstm_b200 import binding
+    from layer_lstm_b200.runner import DeviceProblem
+    h_in, outs = _io_tensors(wl, prob)
+    host_in = {k: v.detach().cpu().pin_memory() for k, v in h_in.items()}
+    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+    d2h = sum(o.numel() * o.element_size() for o in outs)
+    tokens = wl.B * wl.T * world * args.steps
+    if world > 1:
+        host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+
+        def e2e_step():
+            for k, v in host_in.items():
+                h_in[k].copy_(v, non_blocking=True)
+            step()
+            for ho, o in zip(host_out, outs):
+                ho.copy_(o, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        dist.barrier()
+        for i in range(args.steps):
+            flush.zero_()
+            ev[i][0].record(stream)
+            e2e_step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        t = torch.tensor([sum(a.elapsed_time(b) for a, b in ev)], device=prob.x.device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return {"value": tokens / (float(t.item()) / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "overlap": False}
+
+    probs = [prob, DeviceProblem(inp, device=f"cuda:{local}")]
+    io = [_io_tensors(wl, p) for p in probs]
+    host_out = [[torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs] for _ in probs]
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def pipeline(n, t0=None, t1=None):
+        in_done = [torch.cuda.Event() for _ in range(n)]
+        comp_done = [torch.cuda.Event() for _ in range(n)]
+        out_done = [torch.cuda.Event() for _ in range(n)]
+        gate = torch.cuda.Event()
+        if t0 is not None:
+            t0.record(stream)
+        gate.record(stream)
+
+        def copy_in(i):
+            with torch.cuda.stream(s_in):
+                s_in.wait_event(gate if i < 2 else comp_done[i - 2])   # after the start / its buffers' last reader
+                for name, v in host_in.items():
+                    io[i % 2][0][name].copy_(v, non_blocking=True)
+                in_done[i].record(s_in)
+
+        copy_in(0)
+        for i in range(n):
+            k = i % 2
+            if i + 1 < n:
+                copy_in(i + 1)
+            flush.zero_()
+            stream.wait_event(in_done[i])
+            if i >= 2:
+                stream.wait_event(out_done[i - 2])   # results last written to these buffers are read
+            probs[k].step(stream)
+            comp_done[i].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(comp_done[i])
+                for ho, o in zip(host_out[k], io[k][1]):
+                    ho.copy_(o, non_blocking=True)
+                out_done[i].record(s_out)
+        for i in range(max(0, n - 2), n):
+            stream.wait_event(out_done[i])
+        if t1 is not None:
+            t1.record(stream)
+
+    pipeline(2)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    pipeline(args.steps, t0, t1)
+    torch.cuda.synchronize()
+    for p in probs:
+        st = p.status(stream)
+        if st != binding.LSTM_OK:
+            raise binding.LstmError(st, "e2e steps")
+    return {"value": tokens / (t0.elapsed_time(t1) / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "overlap": True}
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -338,45 +450,7 @@ def run_ours(args):
     # ------------------------------------------------------ end to end (host)
     e2e = None
     if not args.no_e2e:
-        h_in = {"x": prob.x, "h0": prob.h0, "c0": prob.c0}
-        if wl.train:
-            h_in["grad_out"] = prob.grad_out
-        h_in = {k: v for k, v in h_in.items() if v is not None}
-        outs = [prob.out, prob.h_n, prob.c_n]
-        if wl.train:
-            outs += [prob.dx, prob.dh0, prob.dc0] + prob.dw_ih + prob.dw_hh + \
-                (prob.db_ih + prob.db_hh if wl.bias else [])
-        host_in = {k: v.detach().cpu().pin_memory() for k, v in h_in.items()}
-        host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
-        h2d = sum(v.numel() * v.element_size() for v in host_in.values())
-        d2h = sum(o.numel() * o.element_size() for o in outs)
-
-        def e2e_step():
-            for k, v in host_in.items():
-                h_in[k].copy_(v, non_blocking=True)
-            step()
-            for ho, o in zip(host_out, outs):
-                ho.copy_(o, non_blocking=True)
-
-        for _ in range(2):
-            e2e_step()
-        torch.cuda.synchronize()
-        ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps)]
-        if world > 1:
-            dist.barrier()
-        for i in range(args.steps):
-            flush.zero_()
-            ev2[i][0].record(stream)
-            e2e_step()
-            ev2[i][1].record(stream)
-        torch.cuda.synchronize()
-        e_ms = sum(a.elapsed_time(b) for a, b in ev2)
-        te = torch.tensor([e_ms], device=prob.x.device, dtype=torch.float64)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e = {"value": tokens / (float(te.item()) / 1e3), "unit": "tokens/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        e2e = measure_e2e(args, wl, inp, prob, step, flush, stream, rank, world, local)
 
     # ------------------------------------------------------------- roofline
     peaks = load_peaks()
