@@ -51,12 +51,6 @@ __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
     return v;
 }
 
-__device__ __forceinline__ unsigned ld_relaxed(const unsigned* p) {
-    unsigned v;
-    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
 __device__ __forceinline__ int ld_volatile(const int* p) {
     return *reinterpret_cast<const volatile int*>(p);
 }
