@@ -6,7 +6,9 @@
 // layer-input gradient dX = dG W_ih.
 //
 // C[M x N] = A[M x K] * B[N x K]^T with both operands K-major in global
-// memory.  A persistent grid (one CTA per SM) walks the 128 x BN output tiles;
+// memory.  A persistent grid (one CTA per SM) walks the BM x BN output tiles
+// (bf16 with M >= 1024: 256 x 256, two M = 128 MMAs per K step, so each
+// operand byte fetched from L2 feeds twice the products of a 128-row tile);
 // warp 0 issues TMA tile loads into a ring of shared-memory stages, warp 1
 // (one thread) issues tcgen05.mma into one of two TMEM accumulators, warps
 // 4-7 drain the other accumulator through registers to global memory while
@@ -27,23 +29,36 @@
 namespace lstm {
 namespace {
 
+// MH: 128-row halves of the tile (one M = 128 MMA each per K step); NACC:
+// accumulator sets in tensor memory (2: a tile's epilogue overlaps the next
+// tile's MMAs); epilogue warps 4 .. 4 + 4*MH - 1.
 template <int KIND> struct Cfg;
-template <> struct Cfg<0> {   // bf16
-    static constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4, FMT = 1;
+template <> struct Cfg<0> {   // bf16, 128 x 256 tiles (small M)
+    static constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4, FMT = 1, MH = 1, NACC = 2;
     static constexpr int A_BYTES = BM * 128, B_BYTES = BN * 128;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 };
 template <> struct Cfg<1> {   // 3xTF32
-    static constexpr int BM = 128, BN = 128, BK = 32, STAGES = 3, FMT = 2;
+    static constexpr int BM = 128, BN = 128, BK = 32, STAGES = 3, FMT = 2, MH = 1, NACC = 2;
     static constexpr int A_BYTES = BM * 128, B_BYTES = BN * 128;
     static constexpr int STAGE_BYTES = 2 * (A_BYTES + B_BYTES);   // hi tiles, then lo tiles
 };
+template <> struct Cfg<2> {   // bf16, 256 x 256 tiles: a third less operand traffic from L2
+    static constexpr int BM = 256, BN = 256, BK = 64, STAGES = 3, FMT = 1, MH = 2, NACC = 1;
+    static constexpr int A_BYTES = BM * 128, B_BYTES = BN * 128;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+};
 
-constexpr int kStageFloats = 4 * 32 * 33;   // epilogue staging: one 32 x 33 block per epilogue warp
+template <int KIND>
+constexpr int epi_warps() { return 4 * Cfg<KIND>::MH; }
+template <int KIND>
+constexpr int threads_of() { return 128 + 32 * epi_warps<KIND>(); }
+template <int KIND>
+constexpr int stage_floats() { return epi_warps<KIND>() * 32 * 33; }   // one 32 x 33 block per epilogue warp
 
 template <int KIND>
 constexpr size_t smem_bytes() {
-    return (size_t)Cfg<KIND>::STAGES * Cfg<KIND>::STAGE_BYTES + (size_t)kStageFloats * 4 + 1024 + 256;
+    return (size_t)Cfg<KIND>::STAGES * Cfg<KIND>::STAGE_BYTES + (size_t)stage_floats<KIND>() * 4 + 1024 + 256;
 }
 
 struct TcEpi {
@@ -96,14 +111,14 @@ __device__ __forceinline__ TileCoord tile_coord(const TcEpi& e, int t) {
 // of BN tensor-memory columns alternate between tiles, so the epilogue of
 // one tile overlaps the loads and MMAs of the next.
 template <int KIND>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(threads_of<KIND>(), 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, TcEpi e) {
     using Cf = Cfg<KIND>;
-    constexpr int S = Cf::STAGES, BM = Cf::BM, BN = Cf::BN, BK = Cf::BK;
+    constexpr int S = Cf::STAGES, BN = Cf::BN, BK = Cf::BK;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
     float* stage_out = reinterpret_cast<float*>(smem + S * Cf::STAGE_BYTES);
-    uint64_t* full = reinterpret_cast<uint64_t*>(stage_out + kStageFloats);
+    uint64_t* full = reinterpret_cast<uint64_t*>(stage_out + stage_floats<KIND>());
     uint64_t* lofull = full + S;
     uint64_t* empty = lofull + S;
     uint64_t* tmem_full = empty + S;       // [2]
@@ -122,13 +137,13 @@ __global__ void __launch_bounds__(256, 1)
         }
         for (int b = 0; b < 2; ++b) {
             tc::mbar_init(&tmem_full[b], 1);
-            tc::mbar_init(&tmem_empty[b], 4);   // one arrive per epilogue warp
+            tc::mbar_init(&tmem_empty[b], epi_warps<KIND>());   // one arrive per epilogue warp
         }
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
     if (warp == 1) {
-        tc::tmem_alloc(tmem_slot, 2 * BN);
+        tc::tmem_alloc(tmem_slot, Cf::NACC * Cf::MH * BN);
         tc::tmem_relinquish();
     }
     tc::tc_fence_before();
@@ -163,16 +178,17 @@ __global__ void __launch_bounds__(256, 1)
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            constexpr uint32_t idesc = tc::instr_desc(Cf::FMT, BM, BN);
+            constexpr uint32_t idesc = tc::instr_desc(Cf::FMT, 128, BN);
             int it = 0, last = -1, i = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++i) {
                 const TileCoord c = tile_coord<KIND>(e, t);
-                const int ab = i & 1;
-                // the epilogue has drained this accumulator (tile i - 2)
-                if (!tc::mbar_wait(&tmem_empty[ab], ((i >> 1) & 1) ^ 1, abort_flag, e.status, e.timeout_ns)) break;
+                const int ab = i % Cf::NACC;
+                // the epilogue has drained this accumulator set (tile i - NACC)
+                if (!tc::mbar_wait(&tmem_empty[ab], ((i / Cf::NACC) & 1) ^ 1, abort_flag, e.status, e.timeout_ns))
+                    break;
                 tc::tc_fence_after();
-                const uint32_t acc_t = tmem + (uint32_t)(ab * BN);
+                const uint32_t acc_t = tmem + (uint32_t)(ab * Cf::MH * BN);
                 for (int kt = 0; kt < c.nk; ++kt, ++it) {
                     const int s = it % S, r = it / S;
                     uint64_t* ready = KIND == 1 ? &lofull[s] : &full[s];
@@ -189,8 +205,12 @@ __global__ void __launch_bounds__(256, 1)
                         const uint64_t ad = tc::smem_desc_sw128(a_base + j * 32);
                         const uint64_t bd = tc::smem_desc_sw128(b_base + j * 32);
                         const uint32_t acc = (kt | j) != 0;
-                        if (KIND == 0) {
-                            tc::mma_bf16(acc_t, ad, bd, idesc, acc);
+                        if (KIND != 1) {
+#pragma unroll
+                            for (int h = 0; h < Cf::MH; ++h)   // rows [128h, 128h + 128) of the tile
+                                tc::mma_bf16(acc_t + (uint32_t)(h * BN), tc::smem_desc_sw128(a_base + h * 16384 + j * 32),
+                                             bd, idesc, acc);
+                            (void)ad;
                         } else {
                             const uint32_t lo_off = Cf::A_BYTES + Cf::B_BYTES;
                             const uint64_t adl = tc::smem_desc_sw128(a_base + lo_off + j * 32);
@@ -243,21 +263,24 @@ __global__ void __launch_bounds__(256, 1)
         // Epilogue: each warp drains its 32 accumulator rows in 32 x 32
         // blocks staged through its own shared-memory block, so each global
         // store instruction writes one contiguous 128-byte row segment.
-        const int q = warp & 3;
-        float* stg = stage_out + q * (32 * 33);
+        const int q = warp & 3;               // tensor-memory lane quarter
+        const int h = (warp - 4) >> 2;        // 128-row half of the tile
+        float* stg = stage_out + (warp - 4) * (32 * 33);
         int i = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++i) {
             const TileCoord c = tile_coord<KIND>(e, t);
-            const int ab = i & 1;
-            const bool ok = tc::mbar_wait(&tmem_full[ab], (i >> 1) & 1, abort_flag, e.status, e.timeout_ns);
+            const int ab = i % Cf::NACC;
+            const bool ok = tc::mbar_wait(&tmem_full[ab], (i / Cf::NACC) & 1, abort_flag, e.status, e.timeout_ns);
             if (!ok) break;
             tc::tc_fence_after();
-            const uint32_t acc_t = tmem + (uint32_t)(ab * BN) + ((uint32_t)(q * 32) << 16);
+            const uint32_t acc_t =
+                tmem + (uint32_t)(ab * Cf::MH * BN + h * BN) + ((uint32_t)(q * 32) << 16);
             // Output row of accumulator row (q*32 + lane), computed once per
             // tile and broadcast inside the row loop.
-            const int mrow = c.m0 + q * 32 + lane;
+            const int rbase = c.m0 + h * 128 + q * 32;
+            const int mrow = rbase + lane;
             const long long my_row = e.ws ? (long long)mrow : out_row(e, mrow);
-            const int rows_here = min(32, e.M - (c.m0 + q * 32));
+            const int rows_here = min(32, e.M - rbase);
             for (int cc = 0; cc < BN; cc += 32) {
                 float v[16], w[16];
                 tc::tmem_ld16(acc_t + (uint32_t)cc, v);
@@ -309,7 +332,7 @@ __global__ void __launch_bounds__(256, 1)
     __syncthreads();
     if (warp == 1) {
         tc::tc_fence_after();
-        tc::tmem_dealloc(tmem, 2 * BN);
+        tc::tmem_dealloc(tmem, Cf::NACC * Cf::MH * BN);
     }
 }
 
@@ -388,7 +411,7 @@ cudaError_t launch_kind(const TcGemmArgs& g, cudaStream_t s) {
     e.splits = splits;
     const long long ntiles = (long long)e.tiles_n * e.tiles_m * splits;
     const int grid = (int)std::min<long long>(ntiles, g.num_sms > 0 ? g.num_sms : 148);
-    tc_gemm_kernel<KIND><<<grid, 256, smem, s>>>(ta, tb, e);
+    tc_gemm_kernel<KIND><<<grid, threads_of<KIND>(), smem, s>>>(ta, tb, e);
     err = cudaGetLastError();
     if (err != cudaSuccess || splits == 1) return err;
     const long long total = (long long)g.M * g.N;
@@ -412,7 +435,8 @@ bool tc_gemm_supported(const TcGemmArgs& g) {
 int tc_gemm_tile_n(DType dt) { return dt == DType::F32 ? Cfg<1>::BN : Cfg<0>::BN; }
 
 cudaError_t launch_tc_gemm(const TcGemmArgs& g, cudaStream_t s) {
-    return g.dt == DType::F32 ? launch_kind<1>(g, s) : launch_kind<0>(g, s);
+    if (g.dt == DType::F32) return launch_kind<1>(g, s);
+    return g.M >= 4 * Cfg<2>::BM ? launch_kind<2>(g, s) : launch_kind<0>(g, s);
 }
 
 // ---------------------------------------------------------------- transposes
