@@ -163,7 +163,8 @@ struct Layout {
     bool bwd_ok;
     // workspace offsets
     size_t status, ctr_f, ctr_b, ctr_tc, ctr_end, wih[32], bias[32], whh_f, whh_b, gx, hT, seq[2], dG, dseq[2], xt,
-        dbpart, P, dGT, bop, wcatT, hx, whh_tc, bias_dummy, total;
+        dbpart, P, dGT, bop, wcatT, hx, whh_tc, bias_dummy, gemm_ws, total;
+    size_t gemm_ws_floats;
     // bf16 backward: float32 staging of what it reads and writes
     size_t s_x, s_h0, s_gout, s_ghn, s_hs[2], s_dx, s_dh0, s_wih[32];
     // reserve offsets
@@ -173,6 +174,8 @@ struct Layout {
 };
 
 int in_size(const Layout& l, int layer) { return layer == 0 ? l.I : l.D * l.H; }
+
+constexpr int kMaxSplitK = 4;   // K splits the weight-gradient GEMMs may use
 
 bool valid_desc(const lstm_desc* d) {
     if (!d) return false;
@@ -251,6 +254,9 @@ bool make_layout(const lstm_desc* d, Layout& l) {
     l.dGT = o; o += al(TB * l.D * l.G * 4);
     l.bop = o; o += al((size_t)l.D * (maxin + l.H) * TB * 4);
     l.wcatT = o; o += al(maxin * l.D * l.G * 4);
+    // split-K partial sums of the weight-gradient GEMMs (up to 4 splits)
+    l.gemm_ws_floats = (size_t)kMaxSplitK * l.G * (maxin + l.H);
+    l.gemm_ws = o; o += al(l.gemm_ws_floats * 4);
     if (l.dt == DType::BF16) {
         const size_t states = (size_t)l.L * l.D * l.B * l.H;
         l.s_x = o; o += al(TB * l.I * 4);
@@ -782,6 +788,9 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
         tw.A = dGT; tw.lda = BTl; tw.B = bop; tw.ldb = BTl;
         tw.C = dw_ih[k * D]; tw.ldc = in; tw.C1 = dw_hh[k * D]; tw.ldc1 = H; tw.n_split = in;
         tw.status = status; tw.timeout_ns = timeout_ns(); tw.num_sms = device_info().sms;
+        tw.splitk = kMaxSplitK;
+        tw.ws = reinterpret_cast<float*>(P(workspace, l.gemm_ws));
+        tw.ws_floats = (long long)l.gemm_ws_floats;
         TcGemmArgs tx{};
         tx.M = (int)BTl; tx.N = in; tx.K = D * G; tx.dt = DType::F32;
         tx.A = dG; tx.lda = ldg; tx.B = wcatT; tx.ldb = (long long)D * G;

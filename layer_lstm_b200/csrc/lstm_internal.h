@@ -51,8 +51,9 @@ struct TcGemmArgs {
     const float* bias;
     int accumulate;
     int remap_T, remap_B;
-    int splitk;
-    float* ws;
+    int splitk;                 // largest K split to consider (<= 1: none)
+    float* ws;                  // scratch for split-K partial sums, or null
+    long long ws_floats;        // its capacity
     int* status;
     uint64_t timeout_ns;
     int num_sms;                // persistent grid size (SMs of the device)

@@ -43,6 +43,11 @@ template <> struct Cfg<1> {   // 3xTF32
     static constexpr int A_BYTES = BM * 128, B_BYTES = BN * 128;
     static constexpr int STAGE_BYTES = 2 * (A_BYTES + B_BYTES);   // hi tiles, then lo tiles
 };
+template <> struct Cfg<3> {   // 3xTF32, 128 x 256 tiles: half the MMAs per product of Cfg<1>
+    static constexpr int BM = 128, BN = 256, BK = 32, STAGES = 2, FMT = 2, MH = 1, NACC = 2;
+    static constexpr int A_BYTES = BM * 128, B_BYTES = BN * 128;
+    static constexpr int STAGE_BYTES = 2 * (A_BYTES + B_BYTES);   // hi tiles, then lo tiles
+};
 template <> struct Cfg<2> {   // bf16, 256 x 256 tiles: a third less operand traffic from L2
     static constexpr int BM = 256, BN = 256, BK = 64, STAGES = 3, FMT = 1, MH = 2, NACC = 1;
     static constexpr int A_BYTES = BM * 128, B_BYTES = BN * 128;
@@ -115,6 +120,7 @@ __global__ void __launch_bounds__(threads_of<KIND>(), 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, TcEpi e) {
     using Cf = Cfg<KIND>;
     constexpr int S = Cf::STAGES, BN = Cf::BN, BK = Cf::BK;
+    constexpr bool kTf32 = Cf::FMT == 2;   // float32 operands: 3xTF32 with in-place hi/lo split
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
     float* stage_out = reinterpret_cast<float*>(smem + S * Cf::STAGE_BYTES);
@@ -191,7 +197,7 @@ __global__ void __launch_bounds__(threads_of<KIND>(), 1)
                 const uint32_t acc_t = tmem + (uint32_t)(ab * Cf::MH * BN);
                 for (int kt = 0; kt < c.nk; ++kt, ++it) {
                     const int s = it % S, r = it / S;
-                    uint64_t* ready = KIND == 1 ? &lofull[s] : &full[s];
+                    uint64_t* ready = kTf32 ? &lofull[s] : &full[s];
                     if (!tc::mbar_wait(ready, r & 1, abort_flag, e.status, e.timeout_ns)) {
                         ok = false;
                         break;
@@ -205,7 +211,7 @@ __global__ void __launch_bounds__(threads_of<KIND>(), 1)
                         const uint64_t ad = tc::smem_desc_sw128(a_base + j * 32);
                         const uint64_t bd = tc::smem_desc_sw128(b_base + j * 32);
                         const uint32_t acc = (kt | j) != 0;
-                        if (KIND != 1) {
+                        if (!kTf32) {
 #pragma unroll
                             for (int h = 0; h < Cf::MH; ++h)   // rows [128h, 128h + 128) of the tile
                                 tc::mma_bf16(acc_t + (uint32_t)(h * BN), tc::smem_desc_sw128(a_base + h * 16384 + j * 32),
@@ -228,7 +234,7 @@ __global__ void __launch_bounds__(threads_of<KIND>(), 1)
             }
             if (*abort_flag && last >= 0) mbar_drain(&empty[last % S], (last / S) & 1);
         }
-    } else if (KIND == 1 && warp < 4) {
+    } else if (kTf32 && warp < 4) {
         // hi/lo split of each stage (64 threads), in place for hi.
         const int ct = threadIdx.x - 64;
         int it = 0;
@@ -392,8 +398,24 @@ cudaError_t launch_kind(const TcGemmArgs& g, cudaStream_t s) {
     if (!make_map(&tb, g.dt, g.B, g.N, g.K, g.ldb, Cf::BN)) return cudaErrorInvalidValue;
     TcEpi e{};
     e.M = g.M; e.N = g.N; e.K = g.K;
-    const int splits = g.splitk > 1 && g.ws ? g.splitk : 1;
     const int kchunks = (g.K + Cf::BK - 1) / Cf::BK;
+    const int sms = g.num_sms > 0 ? g.num_sms : 148;
+    const long long tiles = (long long)((g.N + Cf::BN - 1) / Cf::BN) * ((g.M + Cf::BM - 1) / Cf::BM);
+    // Split K when the tiles fill the SMs poorly and partial sums fit in
+    // g.ws: the split count (<= g.splitk) with the best last-wave occupancy,
+    // each split keeping at least 16 K chunks.
+    int splits = 1;
+    if (g.ws && g.splitk > 1) {
+        auto occ = [&](long long u) { return (double)u / (double)(((u + sms - 1) / sms) * sms); };
+        double best = occ(tiles);
+        for (int sp = 2; sp <= g.splitk; ++sp) {
+            if (kchunks / sp < 16 || (long long)sp * g.M * g.N > g.ws_floats) break;
+            if (occ(tiles * sp) > best + 0.05) {
+                best = occ(tiles * sp);
+                splits = sp;
+            }
+        }
+    }
     e.k_per_split = ((kchunks + splits - 1) / splits) * Cf::BK;
     e.C = g.C; e.ldc = g.ldc;
     e.C1 = g.C1 ? g.C1 : g.C; e.ldc1 = g.C1 ? g.ldc1 : g.ldc;
@@ -410,7 +432,7 @@ cudaError_t launch_kind(const TcGemmArgs& g, cudaStream_t s) {
     e.tiles_m = (g.M + Cf::BM - 1) / Cf::BM;
     e.splits = splits;
     const long long ntiles = (long long)e.tiles_n * e.tiles_m * splits;
-    const int grid = (int)std::min<long long>(ntiles, g.num_sms > 0 ? g.num_sms : 148);
+    const int grid = (int)std::min<long long>(ntiles, sms);
     tc_gemm_kernel<KIND><<<grid, threads_of<KIND>(), smem, s>>>(ta, tb, e);
     err = cudaGetLastError();
     if (err != cudaSuccess || splits == 1) return err;
@@ -435,7 +457,14 @@ bool tc_gemm_supported(const TcGemmArgs& g) {
 int tc_gemm_tile_n(DType dt) { return dt == DType::F32 ? Cfg<1>::BN : Cfg<0>::BN; }
 
 cudaError_t launch_tc_gemm(const TcGemmArgs& g, cudaStream_t s) {
-    if (g.dt == DType::F32) return launch_kind<1>(g, s);
+    if (g.dt == DType::F32) {
+        // 128 x 256 tiles halve the MMAs per product but halve the tile count:
+        // used when they still fill the SMs or K can be split
+        const long long tiles3 = (long long)((g.M + Cfg<3>::BM - 1) / Cfg<3>::BM) * ((g.N + Cfg<3>::BN - 1) / Cfg<3>::BN);
+        const int sms = g.num_sms > 0 ? g.num_sms : 148;
+        const bool wide = g.N >= Cfg<3>::BN && (tiles3 >= sms || (g.ws && g.splitk > 1));
+        return wide ? launch_kind<3>(g, s) : launch_kind<1>(g, s);
+    }
     return g.M >= 4 * Cfg<2>::BM ? launch_kind<2>(g, s) : launch_kind<0>(g, s);
 }
 
