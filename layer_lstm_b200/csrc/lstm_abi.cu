@@ -86,7 +86,7 @@ DropoutArgs dropout_args(const lstm_desc* d, int layer, const void* src, void* d
 struct Timing {
     std::mutex mu;
     bool on = false;
-    struct Pending { int kind; cudaEvent_t a, b; };
+    struct Pending { int kind; cudaEvent_t a, b; int n; };
     std::vector<Pending> pending;
     std::vector<cudaEvent_t> pool;
     double total_ms[K_COUNT] = {};
@@ -109,8 +109,9 @@ cudaEvent_t take_event(Timing& tm) {
     return e;
 }
 
+// nlaunch: where f leaves the number of kernels it launched (null: one).
 template <typename F>
-cudaError_t timed(int kind, cudaStream_t s, F&& f) {
+cudaError_t timed(int kind, cudaStream_t s, F&& f, const int* nlaunch = nullptr) {
     Timing& tm = timing();
     if (!tm.on) return f();
     std::lock_guard<std::mutex> lk(tm.mu);
@@ -122,7 +123,7 @@ cudaError_t timed(int kind, cudaStream_t s, F&& f) {
     if (e != cudaSuccess) return e;
     e = cudaEventRecord(b, s);
     if (e != cudaSuccess) return e;
-    tm.pending.push_back({kind, a, b});
+    tm.pending.push_back({kind, a, b, nlaunch ? *nlaunch : 1});
     return cudaSuccess;
 }
 
@@ -391,7 +392,7 @@ int lstm_timing_read(lstm_kernel_time* out, int max_entries) {
         float ms = 0.f;
         if (cudaEventSynchronize(p.b) == cudaSuccess && cudaEventElapsedTime(&ms, p.a, p.b) == cudaSuccess) {
             tm.total_ms[p.kind] += ms;
-            tm.launches[p.kind] += 1;
+            tm.launches[p.kind] += p.n;
         } else {
             return -1;
         }
@@ -527,7 +528,8 @@ lstm_status lstm_forward_varlen(const lstm_desc* desc, const int* lengths, const
         tg.bias = g.bias; tg.remap_T = g.remap_T; tg.remap_B = g.remap_B;
         tg.status = status; tg.timeout_ns = timeout_ns(); tg.num_sms = device_info().sms;
         if (tc_gemm_enabled() && tc_gemm_supported(tg)) {
-            LSTM_CUDA(timed(K_PROJ_TC, stream, [&] { return launch_tc_gemm(tg, stream); }));
+            int nl = 1;
+            LSTM_CUDA(timed(K_PROJ_TC, stream, [&] { return launch_tc_gemm(tg, stream, &nl); }, &nl));
         } else {
             LSTM_CUDA(timed(K_PROJ_SIMT, stream, [&] { return launch_gemm(g, stream); }));
         }
@@ -828,14 +830,20 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
                 twd.B = bo;
                 twd.C = dw_ih[k * D + d];
                 twd.C1 = dw_hh[k * D + d];
-                LSTM_CUDA(timed(K_DW_TC, stream, [&] { return launch_tc_gemm(twd, stream); }));
+                {
+                    int nl = 1;
+                    LSTM_CUDA(timed(K_DW_TC, stream, [&] { return launch_tc_gemm(twd, stream, &nl); }, &nl));
+                }
                 TransposeArgs tww{};
                 tww.M = G; tww.C = in; tww.mode = 0;
                 tww.src = wihf[k * D + d]; tww.lds = in;
                 tww.dst = wcatT + (size_t)d * G; tww.ldd = (long long)D * G;
                 LSTM_CUDA(timed(K_TRANSPOSE, stream, [&] { return launch_transpose(tww, stream); }));
             }
-            LSTM_CUDA(timed(K_DX_TC, stream, [&] { return launch_tc_gemm(tx, stream); }));
+            {
+                int nl = 1;
+                LSTM_CUDA(timed(K_DX_TC, stream, [&] { return launch_tc_gemm(tx, stream, &nl); }, &nl));
+            }
         } else {
             for (int d = 0; d < D; ++d) {
                 // dW_ih = sum_t dG_t^T x_t

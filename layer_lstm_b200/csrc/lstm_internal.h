@@ -60,7 +60,8 @@ struct TcGemmArgs {
 };
 bool tc_gemm_supported(const TcGemmArgs& g);
 int tc_gemm_tile_n(DType dt);
-cudaError_t launch_tc_gemm(const TcGemmArgs& g, cudaStream_t s);
+// *nlaunch (if given) = kernels launched: 2 when K was split (GEMM + reduction).
+cudaError_t launch_tc_gemm(const TcGemmArgs& g, cudaStream_t s, int* nlaunch = nullptr);
 
 // dst[c*ldd + m] = src(m, c) for m < M, c < C (float32).
 //  mode 0: src(m, c) = src[row(m)*lds + c], row(m) = m, or with bt_remap the

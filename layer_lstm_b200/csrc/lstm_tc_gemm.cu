@@ -391,7 +391,7 @@ bool make_map(CUtensorMap* map, DType dt, const void* base, long long rows, long
 }
 
 template <int KIND>
-cudaError_t launch_kind(const TcGemmArgs& g, cudaStream_t s) {
+cudaError_t launch_kind(const TcGemmArgs& g, cudaStream_t s, int* nlaunch) {
     using Cf = Cfg<KIND>;
     CUtensorMap ta, tb;
     if (!make_map(&ta, g.dt, g.A, g.M, g.K, g.lda, Cf::BM)) return cudaErrorInvalidValue;
@@ -435,10 +435,12 @@ cudaError_t launch_kind(const TcGemmArgs& g, cudaStream_t s) {
     const int grid = (int)std::min<long long>(ntiles, sms);
     tc_gemm_kernel<KIND><<<grid, threads_of<KIND>(), smem, s>>>(ta, tb, e);
     err = cudaGetLastError();
+    if (nlaunch) *nlaunch = 1;
     if (err != cudaSuccess || splits == 1) return err;
     const long long total = (long long)g.M * g.N;
     const int blocks = (int)std::min<long long>((total + 255) / 256, 148LL * 8);
     splitk_reduce_kernel<<<blocks, 256, 0, s>>>(e, splits);
+    if (nlaunch) *nlaunch = 2;
     return cudaGetLastError();
 }
 
@@ -456,16 +458,16 @@ bool tc_gemm_supported(const TcGemmArgs& g) {
 
 int tc_gemm_tile_n(DType dt) { return dt == DType::F32 ? Cfg<1>::BN : Cfg<0>::BN; }
 
-cudaError_t launch_tc_gemm(const TcGemmArgs& g, cudaStream_t s) {
+cudaError_t launch_tc_gemm(const TcGemmArgs& g, cudaStream_t s, int* nlaunch) {
     if (g.dt == DType::F32) {
         // 128 x 256 tiles halve the MMAs per product but halve the tile count:
         // used when they still fill the SMs or K can be split
         const long long tiles3 = (long long)((g.M + Cfg<3>::BM - 1) / Cfg<3>::BM) * ((g.N + Cfg<3>::BN - 1) / Cfg<3>::BN);
         const int sms = g.num_sms > 0 ? g.num_sms : 148;
         const bool wide = g.N >= Cfg<3>::BN && (tiles3 >= sms || (g.ws && g.splitk > 1));
-        return wide ? launch_kind<3>(g, s) : launch_kind<1>(g, s);
+        return wide ? launch_kind<3>(g, s, nlaunch) : launch_kind<1>(g, s, nlaunch);
     }
-    return g.M >= 4 * Cfg<2>::BM ? launch_kind<2>(g, s) : launch_kind<0>(g, s);
+    return g.M >= 4 * Cfg<2>::BM ? launch_kind<2>(g, s, nlaunch) : launch_kind<0>(g, s, nlaunch);
 }
 
 // ---------------------------------------------------------------- transposes
