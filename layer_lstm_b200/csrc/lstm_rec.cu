@@ -192,9 +192,11 @@ __global__ void __launch_bounds__(kRecThreads, 1) fwd_rec_kernel(FwdRecArgs a) {
     size_t off = align16((size_t)Hp * R * sizeof(WT));
     WT* hs = reinterpret_cast<WT*>(smem + off);                        // [Hp][Bs]
     off += align16((size_t)Hp * Bs * sizeof(WT));
-    float* red = reinterpret_cast<float*>(smem + off);                 // [KS][R][Bs]
+    // K-slice partial sums, column-major per slice so that a thread's 4-row
+    // tile column is one 16-byte store and a unit's 4 gates one 16-byte load
+    float* red = reinterpret_cast<float*>(smem + off);                 // [KS][Bs][R]
     off += align16((size_t)KS * R * Bs * sizeof(float));
-    float* cs = reinterpret_cast<float*>(smem + off);                  // [U][Bg]
+    float* cs = reinterpret_cast<float*>(smem + off);                  // [Bg][U]
     off += align16((size_t)U * p.Bg * sizeof(float));
     uint64_t* hbar = reinterpret_cast<uint64_t*>(smem + ((off + 7) & ~size_t(7)));
 
@@ -218,7 +220,7 @@ __global__ void __launch_bounds__(kRecThreads, 1) fwd_rec_kernel(FwdRecArgs a) {
         for (int i = tid; i < Hp * R / 4; i += nth) d4[i] = s4[i];
     }
     for (int i = tid; i < U * p.Bg; i += nth) {
-        const int ul = i / p.Bg, bl = i % p.Bg;
+        const int ul = i % U, bl = i / U;
         float c = 0.f;
         if (a.c0 && ul < nU && bl < nB) c = a.c0[((size_t)d * B + b0 + bl) * H + u0 + ul];
         cs[i] = c;
@@ -243,27 +245,25 @@ __global__ void __launch_bounds__(kRecThreads, 1) fwd_rec_kernel(FwdRecArgs a) {
     const bool tr0 = blockIdx.x == 0 && tid == 0;   // the traced thread
     auto store_red = [&](int ks, int r0, int n0, auto& acc) {
         constexpr int tn = sizeof(acc[0]) / sizeof(float);
-        float* rp = red + ((size_t)ks * R + r0) * Bs + n0;
+        float* rp = red + ((size_t)ks * Bs + n0) * R + r0;
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int h = 0; h < tn; h += 4)
-                *reinterpret_cast<float4*>(rp + (size_t)i * Bs + h) =
-                    make_float4(acc[i][h], acc[i][h + 1], acc[i][h + 2], acc[i][h + 3]);
+        for (int j = 0; j < tn; ++j)
+            *reinterpret_cast<float4*>(rp + (size_t)j * R) = make_float4(acc[0][j], acc[1][j], acc[2][j], acc[3][j]);
     };
     for (int s = 0; s < T; ++s) {
         const int t = d == 0 ? s : T - 1 - s;
         const int tp = d == 0 ? t - 1 : t + 1;
         // Gx of this thread's first-sub-tile pairs does not depend on other
-        // blocks: fetch it before waiting.  Pair i: row bl = i % nb, unit ul = i / nb.
-        const int nb0 = min(Bs, nB);
+        // blocks: fetch it before waiting.  Pair i: unit ul = i % nU, row
+        // bl = i / nU (units fastest: Gx, outputs and saved state of
+        // consecutive threads are contiguous).
         float4 gxp[2];
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
             const int i = tid + q * nth;
             gxp[q] = make_float4(0.f, 0.f, 0.f, 0.f);
             if (i < np0) {
-                const int bl = i % nb0, ul = i / nb0;
+                const int ul = i % nU, bl = i / nU;
                 gxp[q] = *reinterpret_cast<const float4*>(
                     a.gx + ((size_t)t * B + b0 + bl) * (size_t)(D * G) + (size_t)d * G + 4 * (u0 + ul));
             }
@@ -306,7 +306,7 @@ __global__ void __launch_bounds__(kRecThreads, 1) fwd_rec_kernel(FwdRecArgs a) {
             __syncthreads();
             if (bs0 == 0) trace_mark(a.trace, tr0, s, 3);
             for (int i = tid, q = 0; i < nU * nb; i += nth, ++q) {
-                const int bl = i % nb, ul = i / nb;
+                const int ul = i % nU, bl = i / nU;
                 const int b = b0 + bs0 + bl, u = u0 + ul;
                 float4 gxv;
                 if (bs0 == 0 && q < 2) {
@@ -315,22 +315,23 @@ __global__ void __launch_bounds__(kRecThreads, 1) fwd_rec_kernel(FwdRecArgs a) {
                     gxv = *reinterpret_cast<const float4*>(
                         a.gx + ((size_t)t * B + b) * (size_t)(D * G) + (size_t)d * G + 4 * u);
                 }
-                float pre[4] = {gxv.x, gxv.y, gxv.z, gxv.w};
-#pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    float acc = 0.f;
-                    for (int ks = 0; ks < KS; ++ks) acc += red[((size_t)ks * R + 4 * ul + g) * Bs + bl];
-                    pre[g] += acc;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int ks = 0; ks < KS; ++ks) {
+                    const float4 r4 = *reinterpret_cast<const float4*>(red + ((size_t)ks * Bs + bl) * R + 4 * ul);
+                    acc.x += r4.x; acc.y += r4.y; acc.z += r4.z; acc.w += r4.w;
                 }
-                float& cref = cs[ul * p.Bg + bs0 + bl];
+                const float pre[4] = {gxv.x + acc.x, gxv.y + acc.y, gxv.z + acc.z, gxv.w + acc.w};
+                float& cref = cs[(bs0 + bl) * U + ul];
                 // Padding of a variable-length row: the state stays as it was
                 // (h from the gathered tile), the user output is 0, and the
                 // exchange and the saved sequence carry the frozen h.
                 const bool valid = !a.len || t < a.len[b];
                 float c = cref;
-                WT hv = hs[(size_t)u * Bs + bl];
+                WT hv;
                 float4 gates = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (valid) {
+                if (!valid) {
+                    hv = hs[(size_t)u * Bs + bl];
+                } else {
                     const float ig = sigmoidf_(pre[0]);
                     const float fg = sigmoidf_(pre[1]);
                     const float gg = tanhf(pre[2]);
