@@ -173,6 +173,10 @@ constexpr int kRecThreads = 256;   // threads per recurrent block
 // Column-tile width of the block_mm calls on an N-column operand.
 __host__ __device__ constexpr int rec_tn(int N) { return N % 8 == 0 ? 8 : 4; }
 
+// Row stride of the backward's gate-derivative tile (Bs columns): the
+// padding spreads the unit-fastest stores of its gate-major rows over banks.
+__host__ __device__ constexpr int bwd_lda(int Bs) { return Bs + 4; }
+
 inline int pick_ks(int R, int N, int K) {
     const int nT = (R / 4) * (N / rec_tn(N));
     int ks = 1;
@@ -392,21 +396,24 @@ __global__ void __launch_bounds__(kRecThreads, 1) bwd_rec_kernel(BwdRecArgs a) {
     const RecPlan& p = a.p;
     const int H = a.H, B = a.B, T = a.T, D = a.D, G = 4 * H;
     const int Hp = (H + 3) & ~3;
-    const int U = p.U, R4 = 4 * U, Bs = p.Bs, Bg = p.Bg;
+    const int U = p.U, R4 = 4 * U, Bs = p.Bs, Bg = p.Bg, LdA = bwd_lda(Bs);
+    // Gate rows are gate-major within the block (row g*U + ul is gate g of
+    // unit j0 + ul), and per-(row, unit) state is unit-fastest, so the
+    // gate-gradient threads (units fastest) touch contiguous words.
     WT* Wr = reinterpret_cast<WT*>(smem);                             // [4U][Hp]
     size_t off = align16((size_t)R4 * Hp * sizeof(WT));
-    float* daT = reinterpret_cast<float*>(smem + off);                // [4U][Bs]
-    off += align16((size_t)R4 * Bs * 4);
-    float* dcs = reinterpret_cast<float*>(smem + off);                // [U][Bg]
+    float* daT = reinterpret_cast<float*>(smem + off);                // [4U][LdA]
+    off += align16((size_t)R4 * LdA * 4);
+    float* dcs = reinterpret_cast<float*>(smem + off);                // [Bg][U]
     off += align16((size_t)U * Bg * 4);
-    float* dhs = reinterpret_cast<float*>(smem + off);                // [U][Bg]
+    float* dhs = reinterpret_cast<float*>(smem + off);                // [Bg][U]
     off += align16((size_t)U * Bg * 4);
-    float* dbacc = reinterpret_cast<float*>(smem + off);              // [4][U][Bg]
+    float* dbacc = reinterpret_cast<float*>(smem + off);              // [4][Bg][U]
     off += align16((size_t)4 * U * Bg * 4);
     // dh that padding of a variable-length row hands on unchanged (h_t = h_{t-1})
-    float* dpass = reinterpret_cast<float*>(smem + off);              // [U][Bg]
+    float* dpass = reinterpret_cast<float*>(smem + off);              // [Bg][U]
     off += align16((size_t)U * Bg * 4);
-    float* gpart = reinterpret_cast<float*>(smem + off);              // [CG][U][Bg]
+    float* gpart = reinterpret_cast<float*>(smem + off);              // [CG][Bg][U]
 
     const int j = blockIdx.x % p.nu;
     const int bg = (blockIdx.x / p.nu) % p.nbg;
@@ -422,7 +429,7 @@ __global__ void __launch_bounds__(kRecThreads, 1) bwd_rec_kernel(BwdRecArgs a) {
         for (int i = tid; i < n16; i += nth) d4[i] = s4[i];
     }
     for (int i = tid; i < U * Bg; i += nth) {
-        const int ul = i / Bg, bl = i % Bg;
+        const int ul = i % U, bl = i / U;
         float dc = 0.f, dh = 0.f;
         if (ul < nU && bl < nB) {
             const size_t sidx = ((size_t)d * B + b0 + bl) * H + j0 + ul;
@@ -443,7 +450,7 @@ __global__ void __launch_bounds__(kRecThreads, 1) bwd_rec_kernel(BwdRecArgs a) {
     auto Pblk = [&](int buf, int c) {
         return a.P + ((((size_t)buf * D + d) * p.nbg + bg) * p.nu + c) * (size_t)Bg * Hp;
     };
-    // gather: dhs[ul][bl] = sum_c P[buf][c][bl][j0+ul] (fixed order over c)
+    // gather: dhs[bl][ul] = sum_c P[buf][c][bl][j0+ul] (fixed order over c)
     const int U4 = U >> 2;
     const int CG = std::max(1, nth / (U4 * Bg));   // as sized by plan_bwd_rec
     auto gather = [&](int buf) {
@@ -465,29 +472,30 @@ __global__ void __launch_bounds__(kRecThreads, 1) bwd_rec_kernel(BwdRecArgs a) {
                     sum.x += v[u].x; sum.y += v[u].y; sum.z += v[u].z; sum.w += v[u].w;
                 }
             }
-            float* gp = gpart + ((size_t)cg * U + 4 * ul4) * Bg + bl;
-            gp[0] = sum.x; gp[Bg] = sum.y; gp[2 * Bg] = sum.z; gp[3 * Bg] = sum.w;
+            *reinterpret_cast<float4*>(gpart + ((size_t)cg * Bg + bl) * U + 4 * ul4) = sum;
         }
         __syncthreads();
         for (int i = tid; i < U * nB; i += nth) {
-            const int ul = i / nB, bl = i % nB;
+            const int ul = i % U, bl = i / U;
             float s = 0.f;
-            for (int cg = 0; cg < CG; ++cg) s += gpart[((size_t)cg * U + ul) * Bg + bl];
-            dhs[ul * Bg + bl] = s + dpass[ul * Bg + bl];
+            for (int cg = 0; cg < CG; ++cg) s += gpart[((size_t)cg * Bg + bl) * U + ul];
+            dhs[bl * U + ul] = s + dpass[bl * U + ul];
         }
         __syncthreads();
     };
 
     const int nb0 = min(Bs, nB);
-    const int np0 = nU * nb0;
     const bool tr0 = blockIdx.x == 0 && tid == 0;   // the traced thread
     for (int s = 0; s < T; ++s) {
         const int t = d == 0 ? T - 1 - s : s;
+        // inputs of this thread's first-sub-tile pairs (pair i: unit
+        // ul = i % U, row bl = i / U), fetched before the wait
         BwdPre pre[2];
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
             const int i = tid + q * nth;
-            if (i < np0) pre[q] = bwd_fetch(a, d, t, b0 + i % nb0, j0 + i / nb0);
+            const int ul = i % U, bl = i / U;
+            if (ul < nU && bl < nb0) pre[q] = bwd_fetch(a, d, t, b0 + bl, j0 + ul);
         }
         trace_mark(a.trace, tr0, s, 0);
         if (s > 0) {
@@ -499,31 +507,30 @@ __global__ void __launch_bounds__(kRecThreads, 1) bwd_rec_kernel(BwdRecArgs a) {
         for (int bs0 = 0; bs0 < nB; bs0 += Bs) {
             const int nb = min(Bs, nB - bs0);
             for (int i = tid, q = 0; i < U * Bs; i += nth, ++q) {
-                const int bl = i % Bs, ul = i / Bs;
+                const int ul = i % U, bl = i / U;
                 if (ul >= nU || bl >= nb) {
-                    if (ul < U && bl < Bs)
 #pragma unroll
-                        for (int g = 0; g < 4; ++g) daT[(4 * ul + g) * Bs + bl] = 0.f;
+                    for (int g = 0; g < 4; ++g) daT[(g * U + ul) * LdA + bl] = 0.f;
                     continue;
                 }
                 const int b = b0 + bs0 + bl, jj = j0 + ul;
+                const int sb = (bs0 + bl) * U + ul;   // per-(row, unit) state index
                 float* dgp = a.dG + ((size_t)t * B + b) * ldg + (size_t)d * G + jj;
                 if (a.len && t >= a.len[b]) {
                     // padding of a variable-length row: the state was held, so
                     // no gate gradient; dc and dh pass on unchanged (the output
                     // there is constant 0: grad_out does not enter)
-                    dpass[ul * Bg + bs0 + bl] = dhs[ul * Bg + bs0 + bl];
+                    dpass[sb] = dhs[sb];
                     dgp[0] = 0.f; dgp[H] = 0.f; dgp[2 * H] = 0.f; dgp[3 * H] = 0.f;
 #pragma unroll
-                    for (int g = 0; g < 4; ++g) daT[(4 * ul + g) * Bs + bl] = 0.f;
+                    for (int g = 0; g < 4; ++g) daT[(g * U + ul) * LdA + bl] = 0.f;
                     continue;
                 }
-                dpass[ul * Bg + bs0 + bl] = 0.f;
-                const BwdPre v = (bs0 == 0 && i < np0 && nb == nb0 && Bs == nb0 && q < 2)
-                                     ? pre[q] : bwd_fetch(a, d, t, b, jj);
+                dpass[sb] = 0.f;
+                const BwdPre v = (bs0 == 0 && q < 2) ? pre[q] : bwd_fetch(a, d, t, b, jj);
                 const float ig = v.act.x, fg = v.act.y, gg = v.act.z, og = v.act.w;
-                float& dcref = dcs[ul * Bg + bs0 + bl];
-                const float dh = v.dy + dhs[ul * Bg + bs0 + bl];
+                float& dcref = dcs[sb];
+                const float dh = v.dy + dhs[sb];
                 const float th = tanhf(v.c);
                 const float dc = dcref + dh * og * (1.f - th * th);
                 const float da_i = dc * gg * ig * (1.f - ig);
@@ -535,11 +542,11 @@ __global__ void __launch_bounds__(kRecThreads, 1) bwd_rec_kernel(BwdRecArgs a) {
                 dgp[H] = da_f;
                 dgp[2 * H] = da_g;
                 dgp[3 * H] = da_o;
-                daT[(4 * ul + 0) * Bs + bl] = da_i;
-                daT[(4 * ul + 1) * Bs + bl] = da_f;
-                daT[(4 * ul + 2) * Bs + bl] = da_g;
-                daT[(4 * ul + 3) * Bs + bl] = da_o;
-                float* dba = dbacc + (size_t)ul * Bg + bs0 + bl;
+                daT[(0 * U + ul) * LdA + bl] = da_i;
+                daT[(1 * U + ul) * LdA + bl] = da_f;
+                daT[(2 * U + ul) * LdA + bl] = da_g;
+                daT[(3 * U + ul) * LdA + bl] = da_o;
+                float* dba = dbacc + sb;
                 dba[0] += da_i;
                 dba[(size_t)U * Bg] += da_f;
                 dba[(size_t)2 * U * Bg] += da_g;
@@ -559,9 +566,9 @@ __global__ void __launch_bounds__(kRecThreads, 1) bwd_rec_kernel(BwdRecArgs a) {
                 }
             };
             if (rec_tn(Bs) == 8)
-                block_mm<8>(Wr, Hp, daT, Bs, Hp, Bs, R4, 1, store_p);
+                block_mm<8>(Wr, Hp, daT, LdA, Hp, Bs, R4, 1, store_p);
             else
-                block_mm<4>(Wr, Hp, daT, Bs, Hp, Bs, R4, 1, store_p);
+                block_mm<4>(Wr, Hp, daT, LdA, Hp, Bs, R4, 1, store_p);
             __syncthreads();
         }
         trace_mark(a.trace, tr0, s, 4);
@@ -574,23 +581,24 @@ __global__ void __launch_bounds__(kRecThreads, 1) bwd_rec_kernel(BwdRecArgs a) {
         gather((T - 1) & 1);
     }
     for (int i = tid; i < nU * nB; i += nth) {
-        const int ul = i / nB, bl = i % nB;
+        const int ul = i % nU, bl = i / nU;
         const size_t sidx = ((size_t)d * B + b0 + bl) * H + j0 + ul;
-        a.dh0[sidx] = dhs[ul * Bg + bl];
-        a.dc0[sidx] = dcs[ul * Bg + bl];
+        a.dh0[sidx] = dhs[bl * U + ul];
+        a.dc0[sidx] = dcs[bl * U + ul];
     }
     // bias-gradient partial of this block: sum over its batch rows, fixed order
     for (int i = tid; i < 4 * nU; i += nth) {
         const int q = i / nU, ul = i % nU;
-        const float* row = dbacc + ((size_t)q * U + ul) * Bg;
+        const float* col = dbacc + (size_t)q * Bg * U + ul;
         float sum = 0.f;
-        for (int bl = 0; bl < nB; ++bl) sum += row[bl];
+        for (int bl = 0; bl < nB; ++bl) sum += col[(size_t)bl * U];
         a.dbpart[((size_t)d * p.nbg + bg) * G + (size_t)q * H + j0 + ul] = sum;
     }
 }
 
-// Backward weight rows: out[d][p][k] (p < nu*4U, k < Hp) = W_hh[(p&3)*H + p/4][k],
-// zero outside the matrix.
+// Backward weight rows: out[d][p][k] (p < nu*4U, k < Hp) = W_hh[g*H + u][k]
+// with block j = p / 4U, g = (p % 4U) / U and u = j*U + p % U (gate-major
+// within each block's 4U rows), zero outside the matrix.
 template <typename T>
 __global__ void pack_hh_rows_kernel(PackHhBwdArgs a) {
     const int Hp = (a.H + 3) & ~3;
@@ -602,8 +610,9 @@ __global__ void pack_hh_rows_kernel(PackHhBwdArgs a) {
         const int k = (int)(e % Hp);
         const long long r2 = e / Hp;
         const int pr = (int)(r2 % Rt), d = (int)(r2 / Rt);
-        const int u = pr >> 2;
-        out[e] = (u < a.H && k < a.H) ? static_cast<const T*>(a.w[d])[((long long)(pr & 3) * a.H + u) * a.H + k]
+        const int pl = pr % (4 * a.U);
+        const int g = pl / a.U, u = (pr / (4 * a.U)) * a.U + pl % a.U;
+        out[e] = (u < a.H && k < a.H) ? static_cast<const T*>(a.w[d])[((long long)g * a.H + u) * a.H + k]
                                       : from_f<T>(0.f);
     }
 }
@@ -676,7 +685,7 @@ RecPlan plan_bwd_rec(int H, int B, int D, DType wdt, int num_sms, size_t smem_ma
             bool ok = false;
             for (; Bs >= 4; Bs -= 4) {
                 const int CG = std::max(1, kRecThreads / ((U / 4) * std::min(Bg, kRecThreads)));
-                const size_t smem = align16h((size_t)4 * U * Hp * wes) + align16h((size_t)4 * U * Bs * 4) +
+                const size_t smem = align16h((size_t)4 * U * Hp * wes) + align16h((size_t)4 * U * bwd_lda(Bs) * 4) +
                                     3 * align16h((size_t)U * Bg * 4) + align16h((size_t)4 * U * Bg * 4) +
                                     align16h((size_t)CG * U * Bg * 4);
                 if (smem <= smem_max) {
