@@ -1,9 +1,11 @@
 """Builds liblstm_b200.so (sm_100a) in-tree with nvcc."""
 from __future__ import annotations
 
+import fcntl
 import os
 import subprocess
 import sys
+import time
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
@@ -31,9 +33,28 @@ def _stale() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
+    """Builds the library when its sources are newer (or `force`).
+
+    Processes that call this at the same time (the ranks of a multi-GPU
+    launch, parallel test workers) build one at a time under a file lock; a
+    process that got the lock after another one built finds the library
+    fresh and returns."""
     if not force and not _stale():
         return LIB_PATH
+    requested = time.time()
     os.makedirs(BUILD_DIR, exist_ok=True)
+    with open(os.path.join(BUILD_DIR, ".lock"), "a") as lock:
+        fcntl.flock(lock, fcntl.LOCK_EX)
+        try:
+            # built by another process while this one waited for the lock
+            if not _stale() and (not force or os.path.getmtime(LIB_PATH) >= requested):
+                return LIB_PATH
+            return _compile(verbose)
+        finally:
+            fcntl.flock(lock, fcntl.LOCK_UN)
+
+
+def _compile(verbose: bool) -> str:
     objs = []
     flags = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
              "-I", os.path.join(ROOT, "include")] + ARCH
