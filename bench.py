@@ -318,6 +318,22 @@ def cpu_oracle_rate(wl, rows_target=None, min_seconds=10.0):
     return nrows * wl.T / dt, cores, sample, dt
 
 
+def cpu_oracle_single_thread_rate(wl):
+    """The oracle on one host thread over one batch row of the workload
+    (tokens/s): the single-core figure beside the all-core one."""
+    import oracle
+    threads = oracle.num_threads()
+    sub = select_rows(make_inputs(wl), [0])
+    oracle.set_num_threads(1)
+    try:
+        t0 = time.perf_counter()
+        oracle.run_inputs(sub, backward=wl.train)
+        dt = time.perf_counter() - t0
+    finally:
+        oracle.set_num_threads(threads)
+    return wl.T / dt
+
+
 # ------------------------------------------------------------------ arms
 def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -484,7 +500,9 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, cores, sample, secs = cpu_oracle_rate(wl)
         cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-               "sample": sample, "seconds": round(secs, 2)}
+               "sample": sample, "seconds": round(secs, 2),
+               "single_thread": {"value": cpu_oracle_single_thread_rate(wl), "unit": "tokens/s",
+                                 "cores": 1, "sample": "1 batch row, full T/L/H"}}
 
     if rank == 0:
         line = {

@@ -95,3 +95,11 @@ def test_trace_summary_skips_unrecorded_events():
     got = trace_steps.summarize(kind, rows)
     assert got["group wait"] == 50
     assert "publish" not in got   # events 4 and 5 never stamped
+
+
+def test_single_thread_oracle_rate_restores_thread_count():
+    import oracle
+    before = oracle.num_threads()
+    rate = bench.cpu_oracle_single_thread_rate(WORKLOADS["c1"])
+    assert rate > 0
+    assert oracle.num_threads() == before
