@@ -59,7 +59,6 @@ struct TcGemmArgs {
     int num_sms;                // persistent grid size (SMs of the device)
 };
 bool tc_gemm_supported(const TcGemmArgs& g);
-int tc_gemm_tile_n(DType dt);
 // *nlaunch (if given) = kernels launched: 2 when K was split (GEMM + reduction).
 cudaError_t launch_tc_gemm(const TcGemmArgs& g, cudaStream_t s, int* nlaunch = nullptr);
 

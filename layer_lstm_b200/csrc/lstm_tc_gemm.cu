@@ -456,8 +456,6 @@ bool tc_gemm_supported(const TcGemmArgs& g) {
     return true;
 }
 
-int tc_gemm_tile_n(DType dt) { return dt == DType::F32 ? Cfg<1>::BN : Cfg<0>::BN; }
-
 cudaError_t launch_tc_gemm(const TcGemmArgs& g, cudaStream_t s, int* nlaunch) {
     if (g.dt == DType::F32) {
         // 128 x 256 tiles halve the MMAs per product but halve the tile count:
