@@ -48,7 +48,24 @@ def parse_args():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="c5")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the per-workload lines (c1-c4) added beside the headline")
+    ap.add_argument("--rank-probe", action="store_true", help=argparse.SUPPRESS)
     return ap.parse_args()
+
+
+def relaunch_as_ranks(n):
+    """--gpus N > 1 without a launcher environment: start N ranks of this
+    script with torch.distributed.run on this node (127.0.0.1), one per GPU,
+    and return their exit status."""
+    import socket
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.run(cmd).returncode
 
 
 def _io_tensors(wl, prob):
@@ -160,7 +177,9 @@ def measure_e2e(args, wl, inp, prob, step, flush, stream, rank, world, local):
         if st != binding.LSTM_OK:
             raise binding.LstmError(st, "e2e steps")
     return {"value": tokens / (t0.elapsed_time(t1) / 1e3), "unit": "tokens/s",
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "overlap": True}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "overlap": True,
+            "mode": "pipelined: two problem instances alternate, so each step's input copy and "
+                    "its neighbour's result copy (copy streams) overlap compute; time = device span"}
 
 
 def load_peaks():
@@ -380,11 +399,121 @@ def workload_config(wl, n):
             "l2": "flushed between timed steps (256 MiB write)"}
 
 
+def roofline_of(wl, kern, steps, total_ms, peaks):
+    """Roofline object of the kernel kind with the largest share of the timed
+    steps: achieved = algorithmic work per launch / average launch time (CUDA
+    events recorded by the library around every launch on its stream)."""
+    dom = max(((k, v) for k, v in kern.items() if v[0] > 0 and kind_bound(k)),
+              key=lambda kv: kv[1][1], default=None)
+    if dom is None:
+        return None
+    kind, (launches, kms) = dom
+    unit, work_step = kernel_work(wl, kind)
+    per_launch = work_step * steps / launches
+    avg_s = kms / launches / 1e3
+    bound = kind_bound(kind)
+    if bound == "alu":
+        peak = alu_peak_tflops()
+        peak_note = "derived: 148 SMs x 128 FP32 lanes x 2 flop x 1965 MHz"
+    elif wl.dtype == "bf16":
+        peak = peaks["bf16_tflops"]
+        peak_note = f"{peaks['source']} bf16 burst"
+    else:
+        peak = peaks["bf16_tflops"] * TF32_OVER_BF16 / 3.0
+        peak_note = (f"{peaks['source']} bf16 burst x 1.1/2.25 (tf32) / 3 (3xTF32 products "
+                     "per fp32 product)")
+    achieved = per_launch / avg_s / 1e12
+    return {"bound": bound, "kernel": kind, "achieved": achieved, "peak": peak,
+            "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic_for(kind, wl.name),
+            "peak_source": peak_note, "launches": launches,
+            "avg_launch_ms": kms / launches, "share_of_step": kms / total_ms}
+
+
+def recurrence_target(wl, kern, steps, peaks, sm_mhz):
+    """The recurrence against the bound the method's targets name for it.
+    bf16, B >= 256: dense bf16 tensor peak (large-batch recurrence).  bf16,
+    small batch: reading every on-chip-resident W_hh element once per step,
+    at the aggregate shared-memory rate 148 SMs x 128 B/clk x the SM clock
+    observed during the run (small-batch recurrence).  float32: the FP32 FMA
+    peak."""
+    rec = [(k, v) for k, v in kern.items() if kind_base(k) == "fwd_rec" and v[0] > 0]
+    if not rec:
+        return None
+    kind, (launches, kms) = rec[0]
+    per_step_s = kms / 1e3 / launches / wl.T     # one step of one layer (all directions)
+    flop = 2.0 * wl.B * wl.D * 4 * wl.H * wl.H
+    if wl.dtype == "bf16" and wl.B < 256:
+        clk = sm_mhz or SM_MAX_MHZ
+        peak = SM_COUNT * 128 * clk * 1e6 / 1e9          # GB/s
+        bytes_step = wl.D * 4 * wl.H * wl.H * 2
+        ach = bytes_step / per_step_s / 1e9
+        return {"bound": "smem (W_hh on chip, read once per step)", "kernel": kind,
+                "us_per_step": per_step_s * 1e6, "achieved": ach, "peak": peak, "unit": "GB/s",
+                "frac": ach / peak, "sm_mhz": clk}
+    if wl.dtype == "bf16":
+        ach = flop / per_step_s / 1e12
+        return {"bound": "tensor", "kernel": kind, "us_per_step": per_step_s * 1e6, "achieved": ach,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"]}
+    ach = flop / per_step_s / 1e12
+    return {"bound": "alu", "kernel": kind, "us_per_step": per_step_s * 1e6, "achieved": ach,
+            "peak": alu_peak_tflops(), "unit": "TFLOP/s", "frac": ach / alu_peak_tflops()}
+
+
+def time_steps(step, stream, flush, steps, warmup):
+    """(total ms over `steps` timed steps, per-kind kernel timing): CUDA events
+    on the launching stream around each step, L2 flushed before each."""
+    import torch
+    from layer_lstm_b200 import binding
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    binding.lstm_timing_reset()
+    binding.lstm_timing_enable(True)
+    for i in range(steps):
+        flush.zero_()
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    binding.lstm_timing_enable(False)
+    return sum(a.elapsed_time(b) for a, b in evs), binding.lstm_timing_read()
+
+
+def measure_workloads(names, steps, warmup, local, flush, peaks, sm_mhz):
+    """One line per other workload (the parity-test configurations), timed
+    the same way as the headline: tokens/s, ms per step and the roofline of
+    the dominant kernel, plus the recurrence against its target bound."""
+    import torch
+    from layer_lstm_b200 import binding
+    from layer_lstm_b200.runner import DeviceProblem
+    res = {}
+    stream = torch.cuda.current_stream()
+    for name in names:
+        wl = WORKLOADS[name]
+        prob = DeviceProblem(make_inputs(wl), device=f"cuda:{local}")
+        total_ms, kern = time_steps(lambda: prob.step(stream), stream, flush, steps, warmup)
+        st = prob.status(stream)
+        if st != binding.LSTM_OK:
+            raise binding.LstmError(st, f"workload {name}")
+        res[name] = {
+            "workload": DESCRIPTIONS[name], "ms_per_step": total_ms / steps,
+            "value": wl.B * wl.T * steps / (total_ms / 1e3), "unit": "tokens/s", "steps": steps,
+            "kernels_ms": {k: round(v[1] / steps, 4) for k, v in kern.items() if v[0]},
+            "roofline": roofline_of(wl, kern, steps, total_ms, peaks),
+            "recurrence": recurrence_target(wl, kern, steps, peaks, sm_mhz),
+        }
+        del prob
+        torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
 
-    from layer_lstm_b200 import binding
+    from layer_lstm_b200 import binding, dp
     from layer_lstm_b200.runner import DeviceProblem
 
     world, rank, local = dist_setup(args)
@@ -395,31 +524,17 @@ def run_ours(args):
                                 device_id=torch.device("cuda", local))
     binding.load()
     wl = WORKLOADS[args.workload]
-    inp = make_inputs(wl)
+    inp = dp.rank_inputs(wl, rank)
     prob = DeviceProblem(inp, device=f"cuda:{local}")
-    grads = []
-    if wl.train:
-        grads = prob.dw_ih + prob.dw_hh + (prob.db_ih if wl.bias else [])
-        flat = torch.empty(sum(g.numel() for g in grads), device=prob.x.device, dtype=torch.float32)
-        off = 0
-        views = []
-        for g in grads:
-            v = flat[off:off + g.numel()].view_as(g)
-            off += g.numel()
-            views.append(v)
-        n_ih = len(prob.dw_ih)
-        prob.dw_ih = views[:n_ih]
-        prob.dw_hh = views[n_ih:2 * n_ih]
-        if wl.bias:
-            prob.db_ih = views[2 * n_ih:]
-            prob.db_hh = [torch.empty_like(v) for v in prob.db_ih]
-        grad_flat = flat
     stream = torch.cuda.current_stream()
+    if wl.train:
+        bucket = dp.GradBucket.adopt(prob, wl.bias)
 
-    def step():
-        prob.step(stream)
-        if wl.train and world > 1:
-            dist.all_reduce(grad_flat)
+        def step():
+            dp.train_step(lambda: prob.step(stream), bucket, world)
+    else:
+        def step():
+            prob.step(stream)
 
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=prob.x.device)
     for _ in range(args.warmup):
@@ -430,8 +545,6 @@ def run_ours(args):
         raise binding.LstmError(st, "warm-up")
 
     # ------------------------------------------------ device-resident timing
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
     sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
     if world > 1:
         dist.barrier()
@@ -439,23 +552,13 @@ def run_ours(args):
     if sampler:
         sampler.start()
         time.sleep(0.3)
-    binding.lstm_timing_reset()
-    binding.lstm_timing_enable(True)
-    for i in range(args.steps):
-        flush.zero_()
-        evs[i][0].record(stream)
-        step()
-        evs[i][1].record(stream)
-    torch.cuda.synchronize()
-    binding.lstm_timing_enable(False)
+    total_ms, kern = time_steps(step, stream, flush, args.steps, 0)
     if world > 1:
         dist.barrier()
     clocks = sampler.stop() if sampler else None
     st = prob.status(stream)
     if st != binding.LSTM_OK:
         raise binding.LstmError(st, "timed steps")
-    kern = binding.lstm_timing_read()
-    total_ms = sum(a.elapsed_time(b) for a, b in evs)
     t = torch.tensor([total_ms], device=prob.x.device, dtype=torch.float64)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -468,33 +571,16 @@ def run_ours(args):
     if not args.no_e2e:
         e2e = measure_e2e(args, wl, inp, prob, step, flush, stream, rank, world, local)
 
-    # ------------------------------------------------------------- roofline
     peaks = load_peaks()
-    roof = None
-    dom = max(((k, v) for k, v in kern.items() if v[0] > 0 and kind_bound(k)),
-              key=lambda kv: kv[1][1], default=None)
-    if dom is not None:
-        kind, (launches, kms) = dom
-        unit, work_step = kernel_work(wl, kind)
-        per_launch = work_step * args.steps / launches
-        avg_s = kms / launches / 1e3
-        bound = kind_bound(kind)
-        if bound == "alu":
-            peak = alu_peak_tflops()
-            peak_note = "derived: 148 SMs x 128 FP32 lanes x 2 flop x 1965 MHz"
-        elif wl.dtype == "bf16":
-            peak = peaks["bf16_tflops"]
-            peak_note = f"{peaks['source']} bf16 burst"
-        else:
-            peak = peaks["bf16_tflops"] * 1.1 / 2.25 / 3.0
-            peak_note = (f"{peaks['source']} bf16 burst x 1.1/2.25 (tf32) / 3 (3xTF32 products "
-                         "per fp32 product)")
-        achieved = per_launch / avg_s / 1e12
-        traffic = traffic_for(kind, wl.name)
-        roof = {"bound": bound, "kernel": kind, "achieved": achieved, "peak": peak,
-                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
-                "peak_source": peak_note, "launches": launches,
-                "avg_launch_ms": kms / launches, "share_of_step": kms / total_ms}
+    roof = roofline_of(wl, kern, args.steps, total_ms, peaks)
+    sm_mhz = clocks.get("sm_mhz") if clocks else None
+
+    # ------------------------------------------ the other workloads (1 GPU)
+    others = None
+    if rank == 0 and world == 1 and not args.no_workloads:
+        names = [n for n in ("c1", "c2", "c3", "c4", "c5") if n != wl.name]
+        others = measure_workloads(names, steps=10, warmup=3, local=local, flush=flush, peaks=peaks,
+                                   sm_mhz=sm_mhz)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -505,15 +591,19 @@ def run_ours(args):
                                  "cores": 1, "sample": "1 batch row, full T/L/H"}}
 
     if rank == 0:
+        data = "synthetic (seeded)" if world == 1 else \
+            "synthetic (seeded; weights shared, each rank its own batch)"
         line = {
             "metric": "sequence tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": wl.dtype, "data": "synthetic (seeded; identical batch on every rank)",
+            "dtype": wl.dtype, "data": data,
             "config": workload_config(wl, world), "e2e": e2e,
             "gpu_launches": int(sum(v[0] for v in kern.values())),
             "kernels_ms": {k: round(v[1] / args.steps, 4) for k, v in kern.items() if v[0]},
-            "roofline": roof, "cpu_baseline": cpu, "clocks": clocks,
+            "roofline": roof, "recurrence": recurrence_target(wl, kern, args.steps, peaks, sm_mhz),
+            "cpu_baseline": cpu, "clocks": clocks,
+            "workloads": others,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -522,6 +612,14 @@ def run_ours(args):
 
 def main():
     args = parse_args()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(relaunch_as_ranks(args.gpus))
+    world, rank, _ = dist_setup(args)
+    if world != args.gpus:
+        sys.exit(f"bench.py: --gpus {args.gpus} but the launcher started {world} ranks")
+    if args.rank_probe:
+        print(f"rank-probe {rank} of {world}", flush=True)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

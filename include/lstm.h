@@ -202,9 +202,13 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
  * device, with that device current); make that first call before any stream
  * capture.  Every call shares the one array: calls that may overlap on the
  * GPU (other streams, other host threads) race and must be serialised by the
- * caller.  The status word read by lstm_query_status lives in the array too;
- * lstm_query_status cannot reach it, so a bounded-wait failure surfaces only
- * through the outputs of the call.
+ * caller.  The status word of a call (LSTM_ERR_TIMEOUT after a bounded wait
+ * gave up) lives in the array too; read it with lstm_noalloc_query_status.
+ * Errors: LSTM_ERR_INVALID_ARG for an invalid description or pointer,
+ * LSTM_ERR_UNSUPPORTED when no recurrent plan fits the device,
+ * LSTM_ERR_WORKSPACE as above, LSTM_ERR_CUDA when the array's address cannot
+ * be looked up.  A cudaDeviceReset invalidates the address cached for that
+ * device; do not call this entry point on a device after resetting it.
  */
 #define LSTM_NOALLOC_SCRATCH_BYTES (32u << 20)
 
@@ -212,6 +216,12 @@ lstm_status lstm_forward_noalloc(const lstm_desc* desc, const void* x, const voi
                                  const float* c0, const void* const* w_ih, const void* const* w_hh,
                                  const void* const* b_ih, const void* const* b_hh,
                                  void* out, void* h_n, float* c_n, cudaStream_t stream);
+
+/* Synchronises `stream` and returns the kernel-side status that the last
+ * lstm_forward_noalloc on the current device recorded in the library's
+ * scratch array (LSTM_OK or LSTM_ERR_TIMEOUT), or LSTM_ERR_CUDA if the stream
+ * reports an error.  No counterpart on the pages (see lstm_forward_noalloc). */
+lstm_status lstm_noalloc_query_status(cudaStream_t stream);
 
 /* Synchronises `stream` and returns the kernel-side status recorded in
  * `workspace` by the last call that used it (LSTM_OK or LSTM_ERR_TIMEOUT), or

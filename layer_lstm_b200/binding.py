@@ -24,7 +24,7 @@ LSTM_BF16 = 1
 EXPORTED = ("lstm_workspace_size", "lstm_reserve_size", "lstm_forward", "lstm_backward",
             "lstm_query_status", "lstm_status_string", "lstm_timing_enable", "lstm_timing_read",
             "lstm_timing_reset", "lstm_forward_noalloc", "lstm_trace_enable", "lstm_trace_read",
-            "lstm_forward_varlen", "lstm_backward_varlen")
+            "lstm_forward_varlen", "lstm_backward_varlen", "lstm_noalloc_query_status")
 LSTM_NOALLOC_SCRATCH_BYTES = 32 << 20
 LSTM_TRACE_MAX_STEPS = 512
 LSTM_TRACE_EVENTS = 16
@@ -108,6 +108,8 @@ def load(build_if_stale: bool = True):
     lib.lstm_timing_reset.restype = None
     lib.lstm_forward_noalloc.argtypes = [dp, vp, vp, vp, vpp, vpp, vpp, vpp, vp, vp, vp, vp]
     lib.lstm_forward_noalloc.restype = ctypes.c_int
+    lib.lstm_noalloc_query_status.argtypes = [vp]
+    lib.lstm_noalloc_query_status.restype = ctypes.c_int
     lib.lstm_trace_enable.argtypes = [ctypes.c_int]
     lib.lstm_trace_enable.restype = ctypes.c_int
     lib.lstm_trace_read.argtypes = [ctypes.POINTER(ctypes.c_ulonglong), ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
@@ -197,6 +199,10 @@ def lstm_forward_noalloc(desc, x, h0, c0, w_ih, w_hh, b_ih, b_hh, out, h_n, c_n,
     return lib.lstm_forward_noalloc(ctypes.byref(desc), _p(x), _p(h0), _p(c0), _parr(w_ih),
                                     _parr(w_hh), _parr(b_ih), _parr(b_hh), _p(out), _p(h_n),
                                     _p(c_n), _stream(stream))
+
+
+def lstm_noalloc_query_status(stream=None) -> int:
+    return int(load().lstm_noalloc_query_status(_stream(stream)))
 
 
 def lstm_query_status(workspace, stream=None) -> int:

@@ -297,6 +297,8 @@ inline char* P(void* base, size_t off) { return static_cast<char*>(base) + off; 
 
 }  // namespace
 
+bool desc_is_valid(const lstm_desc* desc) { return valid_desc(desc); }
+
 // Bytes at the start of the workspace that an inference forward
 // (reserve == NULL) reads or writes: the status word, the counters, the
 // packed weights, the projection output and the exchange / layer-output

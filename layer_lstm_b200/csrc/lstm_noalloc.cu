@@ -8,6 +8,7 @@
 
 namespace lstm {
 size_t forward_workspace_prefix(const lstm_desc* desc);   // lstm_abi.cu
+bool desc_is_valid(const lstm_desc* desc);                 // lstm_abi.cu
 }
 
 namespace {
@@ -21,7 +22,9 @@ constexpr int kMaxDevices = 64;
 
 // Device address of g_noalloc_scratch on the current device.  In host code the
 // array's name only stands for the symbol, so the address is looked up once
-// per device (with that device current) and cached.
+// per device (with that device current) and cached.  A cudaDeviceReset
+// unloads the module and invalidates the cached address; callers that reset
+// a device do not use this entry point on it again in the same process.
 void* scratch_on_current_device() {
     static std::mutex mu;
     static void* addr[kMaxDevices] = {};
@@ -43,8 +46,9 @@ extern "C" lstm_status lstm_forward_noalloc(const lstm_desc* desc, const void* x
                                             const void* const* w_hh, const void* const* b_ih,
                                             const void* const* b_hh, void* out, void* h_n, float* c_n,
                                             cudaStream_t stream) {
+    if (!lstm::desc_is_valid(desc)) return LSTM_ERR_INVALID_ARG;
     const size_t need = lstm::forward_workspace_prefix(desc);
-    if (need == 0) return LSTM_ERR_INVALID_ARG;
+    if (need == 0) return LSTM_ERR_UNSUPPORTED;   // valid, but no recurrent plan fits the device
     if (need > (size_t)LSTM_NOALLOC_SCRATCH_BYTES) return LSTM_ERR_WORKSPACE;
     void* scratch = scratch_on_current_device();
     if (!scratch) return LSTM_ERR_CUDA;
@@ -54,4 +58,11 @@ extern "C" lstm_status lstm_forward_noalloc(const lstm_desc* desc, const void* x
     // forward clears its status word and counters at the start of every call.
     return lstm_forward(desc, x, h0, c0, w_ih, w_hh, b_ih, b_hh, out, h_n, c_n, scratch,
                         lstm_workspace_size(desc), nullptr, 0, stream);
+}
+
+extern "C" lstm_status lstm_noalloc_query_status(cudaStream_t stream) {
+    void* scratch = scratch_on_current_device();
+    if (!scratch) return LSTM_ERR_CUDA;
+    // the status word is the first int of the scratch, as in any workspace
+    return lstm_query_status(scratch, stream);
 }

@@ -18,7 +18,7 @@ import os
 
 import numpy as np
 
-from .build import build as _build, LIB_PATH
+from .build import build as _build, build_single as _build_single, LIB_PATH, LIB_PATH_SINGLE
 
 _lib = None
 
@@ -181,6 +181,56 @@ def lstm_backward(x, w_ih, w_hh, grad_out, b_ih=None, b_hh=None, h0=None, c0=Non
         dx = np.ascontiguousarray(dx.transpose(1, 0, 2))
     return dict(out=out, h_n=h_n, c_n=c_n, dx=dx, dh0=dh0, dc0=dc0,
                 dw_ih=dw_ih, dw_hh=dw_hh, db_ih=db_ih, db_hh=db_hh)
+
+
+_lib_single = None
+
+
+def lstm_forward_single(x, w_ih, w_hh, b_ih=None, b_hh=None, h0=None, c0=None, num_layers=1,
+                        bidirectional=False):
+    """The oracle's forward built with every value in float32 (batch-first x);
+    returns (out, h_n, c_n) as float32 arrays.  Used only to compare the
+    double oracle with a float32 rendition of itself."""
+    global _lib_single
+    if _lib_single is None:
+        _build_single()
+        lib = ctypes.CDLL(LIB_PATH_SINGLE)
+        fp = ctypes.POINTER(ctypes.c_float)
+        fpp = ctypes.POINTER(fp)
+        i = ctypes.c_int
+        lib.oracle_lstm_forward.argtypes = [i, i, i, i, i, i, i, ctypes.POINTER(ctypes.c_int), fp, fp, fp,
+                                            fpp, fpp, fpp, fpp, fp, fp, fp]
+        lib.oracle_lstm_forward.restype = i
+        _lib_single = lib
+    fp = ctypes.POINTER(ctypes.c_float)
+
+    def f32(a):
+        return None if a is None else np.ascontiguousarray(a, dtype=np.float32)
+
+    def ptr(a):
+        return fp() if a is None else a.ctypes.data_as(fp)
+
+    def parr(arrs):
+        return ctypes.POINTER(fp)() if arrs is None else (fp * len(arrs))(*[ptr(a) for a in arrs])
+
+    L, D = int(num_layers), 2 if bidirectional else 1
+    x = f32(x)
+    B, T, I = x.shape
+    H = np.asarray(w_hh[0]).shape[1]
+    w_ih = [f32(w) for w in w_ih]
+    w_hh = [f32(w) for w in w_hh]
+    b_ih = [f32(b) for b in b_ih] if b_ih is not None else None
+    b_hh = [f32(b) for b in b_hh] if b_hh is not None else None
+    h0, c0 = f32(h0), f32(c0)
+    out = np.zeros((B, T, D * H), np.float32)
+    h_n = np.zeros((L * D, B, H), np.float32)
+    c_n = np.zeros((L * D, B, H), np.float32)
+    rc = _lib_single.oracle_lstm_forward(L, D, I, H, B, T, int(b_ih is not None), ctypes.POINTER(ctypes.c_int)(),
+                                         ptr(x), ptr(h0), ptr(c0), parr(w_ih), parr(w_hh), parr(b_ih),
+                                         parr(b_hh), ptr(out), ptr(h_n), ptr(c_n))
+    if rc != 0:
+        raise RuntimeError(f"oracle_lstm_forward (single) failed with code {rc}")
+    return out, h_n, c_n
 
 
 def run_inputs(inp, backward=False):

@@ -75,6 +75,16 @@
 #include <omp.h>
 #endif
 
+/* Single-precision build (gcc -DORACLE_SINGLE), used only for the precision
+ * comparison of "LSTM Gate Equations > Comparing with PyTorch" (Out[20]: two
+ * independent float32 renditions of the cell agree to a few 1e-8).  Every
+ * array, state and sum below is then a float; exp/tanh, declared above, are
+ * still evaluated in double and rounded when stored.  The library's tests and
+ * the benchmark use the double build. */
+#ifdef ORACLE_SINGLE
+#define double float
+#endif
+
 #define ORACLE_OK 0
 #define ORACLE_ERR_ARG 1
 #define ORACLE_ERR_NOMEM 2

@@ -103,3 +103,40 @@ def test_single_thread_oracle_rate_restores_thread_count():
     rate = bench.cpu_oracle_single_thread_rate(WORKLOADS["c1"])
     assert rate > 0
     assert oracle.num_threads() == before
+
+
+def test_recurrence_target_small_batch_is_whh_bytes_per_step():
+    """c3 (bf16, B = 32): the target bound is reading the on-chip W_hh of both
+    directions once per step at 148 SMs x 128 B/clk."""
+    wl = WORKLOADS["c3"]
+    steps = 10
+    # 10 steps x 2 layers launches, each T = 256 recurrent steps of 2 us
+    kern = {"fwd_rec_tc": (steps * wl.L, steps * wl.L * wl.T * 2e-3)}
+    r = bench.recurrence_target(wl, kern, steps, bench.load_peaks(), 1965.0)
+    assert r["us_per_step"] == pytest.approx(2.0)
+    whh_bytes = wl.D * (4 * wl.H) * wl.H * 2
+    assert r["achieved"] == pytest.approx(whh_bytes / 2e-6 / 1e9)
+    assert r["peak"] == pytest.approx(148 * 128 * 1965e6 / 1e9)
+    assert r["frac"] == pytest.approx(r["achieved"] / r["peak"])
+
+
+def test_recurrence_target_large_batch_is_tensor_peak():
+    wl = WORKLOADS["c4"]
+    kern = {"fwd_rec_tc": (5, 5 * wl.T * 4e-3), "proj_gemm_tc": (5, 1.0)}
+    peaks = bench.load_peaks()
+    r = bench.recurrence_target(wl, kern, 5, peaks, None)
+    flop = 2.0 * wl.B * 4 * wl.H * wl.H
+    assert r["bound"] == "tensor"
+    assert r["achieved"] == pytest.approx(flop / 4e-6 / 1e12)
+    assert r["frac"] == pytest.approx(r["achieved"] / peaks["bf16_tflops"])
+
+
+def test_roofline_picks_largest_counted_kind():
+    wl = WORKLOADS["c5"]
+    kern = {"fwd_rec_ffma": (4, 3.0), "bwd_rec_ffma": (4, 4.0), "transpose": (40, 9.0),
+            "dw_gemm_tc": (8, 1.0)}
+    r = bench.roofline_of(wl, kern, 2, 10.0, bench.load_peaks())
+    assert r["kernel"] == "bwd_rec_ffma"
+    per_launch = bench.kernel_work(wl, "bwd_rec_ffma")[1] * 2 / 4
+    assert r["achieved"] == pytest.approx(per_launch / 1e-3 / 1e12)
+    assert r["share_of_step"] == pytest.approx(0.4)

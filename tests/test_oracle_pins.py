@@ -497,3 +497,22 @@ def test_dropout_zero_is_no_dropout():
     b = oracle.run_inputs(inp, backward=True)
     for k in ("out", "dx", "dh0"):
         np.testing.assert_array_equal(a[k], b[k])
+
+
+def test_single_precision_build_agrees_at_float32_rounding():
+    """The comparison method of "LSTM Gate Equations > Comparing with
+    PyTorch" (Out[20]): two implementations of the cell in float32 agree to
+    max-abs 3.22e-08 on h and 6.41e-08 on c (input 8 -> hidden 16).  The
+    oracle compiled with every value in float32, against its double build on
+    the first workload (I8 H16 T5 B4, five steps), must agree to that order:
+    above 1e-9 (the single build really rounds) and below 1e-6."""
+    from layer_lstm_b200.workloads import WORKLOADS
+    wl = WORKLOADS["c1"]
+    inp = make_inputs(wl)
+    ref = oracle.run_inputs(inp)
+    out, h_n, c_n = oracle.lstm_forward_single(inp.x, inp.w_ih, inp.w_hh, inp.b_ih, inp.b_hh,
+                                               inp.h0, inp.c0, wl.L, wl.D == 2)
+    err_h = float(np.abs(out.astype(np.float64) - ref["out"]).max())
+    err_c = float(np.abs(c_n.astype(np.float64) - ref["c_n"]).max())
+    for err in (err_h, err_c, float(np.abs(h_n - ref["h_n"]).max())):
+        assert 1e-9 < err < 1e-6, err

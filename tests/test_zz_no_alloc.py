@@ -19,6 +19,7 @@ from layer_lstm_b200.workloads import Workload, make_inputs
 pytestmark = pytest.mark.gpu
 
 ATOL_F32 = 1e-5
+ATOL_BF16 = 2e-2
 
 
 def _noalloc(p):
@@ -41,9 +42,29 @@ def test_noalloc_matches_workspace_forward_twice(cuda_lib):
         ref = p.results()
         st, got = _noalloc(p)
         assert st == binding.LSTM_OK, binding.status_string(st)
+        assert binding.lstm_noalloc_query_status() == binding.LSTM_OK
         for k in ("out", "h_n", "c_n"):
             err = np.abs(got[k] - ref[k]).max()
             assert err <= ATOL_F32, f"{k}: {err:.3e}"
+
+
+def test_noalloc_bf16_tensor_core_plan_twice(cuda_lib):
+    """The bf16 inference forward on a shape that takes the tensor-core
+    recurrence (its scratch prefix ends at other buffers than the float32
+    plan's): two calls in a row against lstm_forward, and the status word of
+    each call read back through lstm_noalloc_query_status."""
+    wl = Workload("nab", L=1, D=2, I=64, H=128, T=10, B=40, dtype="bf16", state_std=0.3, seed=904)
+    for seed in (905, 906):
+        inp = make_inputs(wl, seed=seed)
+        p = DeviceProblem(inp, train=False)
+        binding.check(p.forward(), "lstm_forward")
+        ref = p.results()
+        st, got = _noalloc(p)
+        assert st == binding.LSTM_OK, binding.status_string(st)
+        assert binding.lstm_noalloc_query_status() == binding.LSTM_OK
+        for k in ("out", "h_n", "c_n"):
+            err = np.abs(got[k] - ref[k]).max()
+            assert err <= ATOL_BF16, f"{k}: {err:.3e}"
 
 
 def test_noalloc_rejects_problem_larger_than_scratch(cuda_lib):
