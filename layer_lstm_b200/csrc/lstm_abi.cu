@@ -10,6 +10,7 @@
 // then time-batched GEMMs for dW_ih, dW_hh and the layer-input gradient
 // (weight phase), mirroring the data/weight split described under cuDNN
 // Backward on the same page.
+#include <stdio.h>
 #include <stdlib.h>
 #include <string.h>
 
@@ -46,6 +47,33 @@ DevInfo device_info() {
         cache[dev].ok = true;
     }
     return cache[dev];
+}
+
+// Fault injection for the tests of the bounded waits (off unless set):
+// LSTM_B200_DEBUG_SKIP_ARRIVAL="fwd:<block>:<step>" or "bwd:<block>:<step>"
+// makes that block of every FFMA forward (backward) recurrent launch withhold
+// its arrival of that step, so the blocks of its group give up at their next
+// counter wait (no copy is in flight there) and the call ends with
+// LSTM_ERR_TIMEOUT in the status word.
+struct SkipArrival {
+    int fwd_block = -1, fwd_step = -1, bwd_block = -1, bwd_step = -1;
+};
+
+const SkipArrival& skip_arrival() {
+    static SkipArrival v = [] {
+        SkipArrival r;
+        const char* e = getenv("LSTM_B200_DEBUG_SKIP_ARRIVAL");
+        if (e && *e) {
+            char which[8] = {0};
+            int blk = -1, st = -1;
+            if (sscanf(e, "%3[a-z]:%d:%d", which, &blk, &st) == 3 && blk >= 0 && st >= 0) {
+                if (strcmp(which, "fwd") == 0) { r.fwd_block = blk; r.fwd_step = st; }
+                if (strcmp(which, "bwd") == 0) { r.bwd_block = blk; r.bwd_step = st; }
+            }
+        }
+        return r;
+    }();
+    return v;
 }
 
 uint64_t timeout_ns() {
@@ -608,6 +636,8 @@ lstm_status lstm_forward_varlen(const lstm_desc* desc, const int* lengths, const
         f.timeout_ns = timeout_ns();
         f.trace = trace_for(LSTM_TRACE_FWD_REC_FFMA, T, stream);
         f.len = lengths;
+        f.skip_block = skip_arrival().fwd_block;
+        f.skip_step = skip_arrival().fwd_step;
         LSTM_CUDA(timed(K_FWD_REC_FFMA, stream, [&] { return launch_fwd_rec(f, stream); }));
         layer_in = hseq;
         if (reserve && l.dropout > 0.f && k < L - 1) {
@@ -768,6 +798,8 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
         b.timeout_ns = timeout_ns();
         b.trace = trace_for(LSTM_TRACE_BWD_REC_FFMA, T, stream);
         b.len = lengths;
+        b.skip_block = skip_arrival().bwd_block;
+        b.skip_step = skip_arrival().bwd_step;
         LSTM_CUDA(timed(K_BWD_REC_FFMA, stream, [&] { return launch_bwd_rec(b, stream); }));
 
         if (desc->bias) {

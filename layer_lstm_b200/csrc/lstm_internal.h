@@ -135,6 +135,7 @@ struct FwdRecArgs {
     uint64_t timeout_ns;
     unsigned long long* trace;  // [kTraceSteps][kTraceEvents] or null
     const int* len;             // [B] valid steps per row, or null (all T)
+    int skip_block, skip_step;  // fault injection: that block withholds that step's arrival (-1: none)
 };
 cudaError_t launch_fwd_rec(const FwdRecArgs& a, cudaStream_t s);
 RecPlan plan_fwd_rec(int H, int B, int D, DType dt, int num_sms, size_t smem_max);
@@ -187,6 +188,7 @@ struct BwdRecArgs {
     uint64_t timeout_ns;
     unsigned long long* trace;  // [kTraceSteps][kTraceEvents] or null
     const int* len;             // [B] valid steps per row, or null (all T)
+    int skip_block, skip_step;  // fault injection: that block withholds that step's arrival (-1: none)
 };
 cudaError_t launch_bwd_rec(const BwdRecArgs& a, cudaStream_t s);
 RecPlan plan_bwd_rec(int H, int B, int D, DType wdt, int num_sms, size_t smem_max);

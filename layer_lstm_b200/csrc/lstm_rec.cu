@@ -296,7 +296,14 @@ __global__ void __launch_bounds__(kRecThreads, 1) fwd_rec_kernel(FwdRecArgs a) {
                     tc::bulk_load(hs, hT_grp + ((size_t)d * T + tp) * hT_tstride, (uint32_t)(tile * sizeof(WT)), hbar);
                 }
                 volatile int never = 0;
-                if (!tc::mbar_wait(hbar, hphase, &never, a.status, a.timeout_ns)) return;
+                if (!tc::mbar_wait(hbar, hphase, &never, a.status, a.timeout_ns)) {
+                    // the copy may still be writing into this block's shared
+                    // memory: let it land (bounded) before the block leaves
+                    const uint64_t t0 = globaltimer_ns();
+                    while (!tc::mbar_try_wait(hbar, hphase) && globaltimer_ns() - t0 < 100000000ull) {
+                    }
+                    return;
+                }
                 hphase ^= 1;
             } else {
                 copy_tile(hs, Hp, Bs, hT_grp + ((size_t)d * T + tp) * hT_tstride + bs0, (size_t)p.Bg, H, nb);
@@ -363,7 +370,10 @@ __global__ void __launch_bounds__(kRecThreads, 1) fwd_rec_kernel(FwdRecArgs a) {
         trace_mark(a.trace, tr0, s, 4);
         if (p.nu > 1 && s + 1 < T) {
             if (bulk) tc::fence_proxy_async_global();   // h_t is read by bulk copies
-            block_arrive(ctr);
+            if ((int)blockIdx.x == a.skip_block && s == a.skip_step)
+                __syncthreads();   // fault injection: this step's arrival is withheld
+            else
+                block_arrive(ctr);
         }
         trace_mark(a.trace, tr0, s, 5);
     }
@@ -572,8 +582,8 @@ __global__ void __launch_bounds__(kRecThreads, 1) bwd_rec_kernel(BwdRecArgs a) {
             __syncthreads();
         }
         trace_mark(a.trace, tr0, s, 4);
-        if (p.nu > 1) block_arrive(ctr);
-        else __syncthreads();
+        if (p.nu > 1 && !((int)blockIdx.x == a.skip_block && s == a.skip_step)) block_arrive(ctr);
+        else __syncthreads();   // one block per group, or fault injection (arrival withheld)
         trace_mark(a.trace, tr0, s, 5);
     }
     if (T > 0) {

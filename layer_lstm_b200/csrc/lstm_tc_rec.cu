@@ -98,19 +98,6 @@ __device__ __forceinline__ float tanh_fast(float z) {
 // exponential and a reciprocal
 __device__ __forceinline__ float sigmoid_fast(float z) { return fmaf(0.5f, tanh_fast(0.5f * z), 0.5f); }
 
-__device__ __forceinline__ bool named_bar_or(int id, int n, bool pred) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.or.pred q, %2, %3, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)pred), "r"(id), "r"(n)
-        : "memory");
-    return r != 0;
-}
-
 __device__ __forceinline__ uint32_t cluster_rank() {
     uint32_t r;
     asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
@@ -450,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 prefetch_l2(a.gx + ((size_t)tn * B + b0 + own0 + e) * ldgx + prow0, kRows * 4);
             }
             const bool ok = tc::mbar_wait(mma_done, s & 1, abort_flag, a.status, a.timeout_ns);
-            if (named_bar_or(1, kEpi, !ok)) break;   // every epilogue thread leaves together
+            if (tc::named_bar_or(1, kEpi, !ok)) break;   // every epilogue thread leaves together
             tc::tc_fence_after();
             trace_mark(a.trace, tr2, s, 4);
             // 1) this block's partial sums of the partner's columns -> partner,
@@ -478,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             trace_mark(a.trace, tr2, s, 5);
             // 2) the partner's partial sums of the own columns
             const bool got = mbar_wait_cluster(recv_full, s & 1, abort_flag, a.status, a.timeout_ns);
-            if (named_bar_or(1, kEpi, !got)) break;
+            if (tc::named_bar_or(1, kEpi, !got)) break;
             trace_mark(a.trace, tr2, s, 6);
             // 3) gates, cell update and h for the own columns, two chunks at a time
 #pragma unroll
@@ -682,22 +669,23 @@ cudaError_t launch_tc_rec(const TcRecArgs& a, cudaStream_t s) {
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = p.smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[2];
+    cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    // every block waits on the others of its group: the whole grid must be
-    // resident at once
+    // Every block waits on the others of its group, so the whole grid must be
+    // resident at once: the launch is refused unless the device can hold all
+    // its clusters together.  The launch carries no cooperative attribute
+    // (cluster launches with it failed under the profiler); should the grid
+    // not be co-scheduled all the same, the bounded waits end the call with
+    // LSTM_ERR_TIMEOUT instead of a hang.
     int clusters = 0;
     e = cudaOccupancyMaxActiveClusters(&clusters, tc_rec_kernel, &cfg);
     if (e != cudaSuccess) return e;
     if (2 * clusters < p.ctas) return cudaErrorCooperativeLaunchTooLarge;
-    attr[1].id = cudaLaunchAttributeCooperative;
-    attr[1].val.cooperative = 1;
-    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, tc_rec_kernel, tmH, tmW, prm);
 }
 
