@@ -176,6 +176,51 @@ bool tc_rec_enabled() {
     return v;
 }
 
+// Layer wavefront of the forward ("LSTM Forward Computation", Stack Multiple
+// RNN Cells: layer k+1 consumes the h sequence layer k produces), for
+// unidirectional stacks on the CUDA-core recurrence: the sequence is cut
+// into chunks, layer k runs chunk c on its own stream while layer k+1 runs
+// chunk c-1.  LSTM_B200_WAVEFRONT=1 turns it on, =0 off; unset: off.
+bool wavefront_enabled() {
+    static const bool v = [] {
+        const char* e = getenv("LSTM_B200_WAVEFRONT");
+        return e && strcmp(e, "1") == 0;
+    }();
+    return v;
+}
+
+// Steps per wavefront chunk (at least 2, so that inside one launch every
+// block of a group has read the chunk's initial state before any block
+// writes the final state the next chunk starts from).
+int wavefront_chunk(int T) {
+    static const int v = [] {
+        const char* e = getenv("LSTM_B200_WAVEFRONT_CHUNK");
+        return e && *e ? atoi(e) : 16;
+    }();
+    return std::max(2, std::min(v, T));
+}
+
+// Non-blocking streams of the layer wavefront, created on first use per
+// device and kept for the life of the process.
+constexpr int kAuxStreams = 3;
+
+cudaStream_t aux_stream(int i) {
+    static std::mutex mu;
+    static std::vector<std::vector<cudaStream_t>> pool;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+    std::lock_guard<std::mutex> lk(mu);
+    if ((int)pool.size() <= dev) pool.resize(dev + 1);
+    if (pool[dev].empty()) {
+        for (int k = 0; k < kAuxStreams; ++k) {
+            cudaStream_t s = nullptr;
+            if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+            pool[dev].push_back(s);
+        }
+    }
+    return pool[dev][i % kAuxStreams];
+}
+
 constexpr size_t kAlign = 256;
 inline size_t al(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 
@@ -200,6 +245,13 @@ struct Layout {
     size_t act[32], cst[32], hseq[32], rtotal;   // per layer: [D][T][B][G], [D][T][B][H], [T][B][D*H]
     size_t hdrop[32];   // layers 0..L-2 with dropout: the next layer's input, [T][B][D*H]
     float dropout;
+    // layer wavefront (forward): plan on each layer's share of the SMs, a
+    // second Gx buffer (layers alternate), per-layer exchange buffers and
+    // counters sized for one chunk
+    bool wf;
+    int wf_chunk;
+    RecPlan fwd_wf;
+    size_t gx2, whh_wf, hTw[32], ctr_w, wf_end;
 };
 
 int in_size(const Layout& l, int layer) { return layer == 0 ? l.I : l.D * l.H; }
@@ -265,6 +317,23 @@ bool make_layout(const lstm_desc* d, Layout& l) {
     l.hT = o; o += al((size_t)l.T * l.D * l.fwd.nbg * l.fwd.Bg * l.H * l.es);   // [D][T][nbg][H][Bg]
     l.seq[0] = o; o += al(TB * l.D * l.H * l.es);
     l.seq[1] = o; o += al(TB * l.D * l.H * l.es);
+    l.wf = false;
+    if (wavefront_enabled() && l.D == 1 && l.L >= 2 && l.T >= 2) {
+        l.fwd_wf = plan_fwd_rec(l.H, Bp, 1, l.dt, dev.sms / 2, smem_max);
+        if (l.fwd_wf.ctas > 0) {
+            l.wf = true;
+            l.wf_chunk = wavefront_chunk(l.T);
+            const int maxc = l.wf_chunk + 1;   // a short last chunk joins the one before it
+            l.gx2 = o; o += al(TB * l.G * 4);
+            l.whh_wf = o; o += al((size_t)l.L * l.fwd_wf.nu * Hp * 4 * l.fwd_wf.U * l.es);
+            for (int k = 0; k < l.L; ++k) {
+                l.hTw[k] = o;
+                o += al((size_t)(2 * maxc) * l.fwd_wf.nbg * l.fwd_wf.Bg * l.H * l.es);
+            }
+            l.ctr_w = o; o += al(sizeof(unsigned) * (size_t)l.L * l.fwd_wf.nbg);
+        }
+    }
+    l.wf_end = o;
     if (l.tcr.ok) {
         l.hx = o; o += al((size_t)l.D * (l.T + 1) * l.B * l.H * 2);
         l.whh_tc = o; o += al((size_t)l.D * l.G * l.H * 2);
@@ -336,7 +405,7 @@ size_t forward_workspace_prefix(const lstm_desc* desc) {
     Layout l;
     if (!make_layout(desc, l)) return 0;
     if (l.tcr.ok) return l.bias_dummy + al((size_t)l.D * l.G * 4);
-    return l.seq[1] + al((size_t)l.T * l.B * l.D * l.H * l.es);
+    return l.wf_end;
 }
 
 static_assert(kTraceSteps == LSTM_TRACE_MAX_STEPS && kTraceEvents == LSTM_TRACE_EVENTS,
@@ -539,6 +608,141 @@ lstm_status lstm_forward_varlen(const lstm_desc* desc, const int* lengths, const
         pk.bias_p = reinterpret_cast<float*>(P(workspace, l.bias[k]));
         LSTM_CUDA(timed(K_PACK, stream, [&] { return launch_pack_ih(pk, stream); }));
     }
+    // Input projection of layer k over `rows` (batch, time) rows of layer_in
+    // (time-major rows, or batch-first x of layer 0 when remap) into Gx rows
+    // starting at gx_out; tensor cores where TMA can address the operands.
+    auto project = [&](int k, const void* in_ptr, float* gx_out, long long rows, bool remap,
+                       cudaStream_t st) -> cudaError_t {
+        const int in = in_size(l, k);
+        GemmArgs g{};
+        g.M = (int)rows; g.N = D * G; g.K = in;
+        g.A = in_ptr; g.ta = l.dt; g.sAm = in; g.sAk = 1;
+        g.B = P(workspace, l.wih[k]); g.tb = l.dt; g.sBk = 1; g.sBn = in;
+        g.C = gx_out; g.tc = DType::F32; g.ldc = (long long)D * G;
+        g.bias = reinterpret_cast<const float*>(P(workspace, l.bias[k]));
+        g.accumulate = 0;
+        if (remap) { g.remap_T = T; g.remap_B = B; }
+        TcGemmArgs tg{};
+        tg.M = g.M; tg.N = g.N; tg.K = g.K; tg.dt = l.dt;
+        tg.A = g.A; tg.lda = in; tg.B = g.B; tg.ldb = in;
+        tg.C = gx_out; tg.ldc = g.ldc;
+        tg.bias = g.bias; tg.remap_T = g.remap_T; tg.remap_B = g.remap_B;
+        tg.status = status; tg.timeout_ns = timeout_ns(); tg.num_sms = device_info().sms;
+        if (tc_gemm_enabled() && tc_gemm_supported(tg)) {
+            int nl = 1;
+            return timed(K_PROJ_TC, st, [&] { return launch_tc_gemm(tg, st, &nl); }, &nl);
+        }
+        return timed(K_PROJ_SIMT, st, [&] { return launch_gemm(g, st); });
+    };
+
+    const bool tc_path = l.tcr.ok && !reserve && tc_rec_enabled();
+    if (l.wf && !lengths && !(reserve && l.dropout > 0.f) && !tc_path) {
+        // ------------------------------------------------ layer wavefront
+        // Layer k runs on stream k (the caller's stream for k = 0, a pool
+        // stream otherwise).  Chunk c of layer k > 0 waits for chunk c of
+        // layer k-1, projects that chunk of its input, and runs its
+        // recurrence from the state chunk c-1 left in h_n / c_n, so layer k
+        // works on chunk c while layer k-1 works on chunk c+1.
+        const int C = l.wf_chunk;
+        std::vector<int> t0s;
+        for (int t0 = 0; t0 < T; t0 += C) t0s.push_back(t0);
+        if (t0s.size() > 1 && T - t0s.back() < 2) t0s.pop_back();   // a 1-step tail joins the chunk before
+        const int nch = (int)t0s.size();
+        std::vector<cudaStream_t> sts(L, stream);
+        for (int k = 1; k < L; ++k) {
+            sts[k] = aux_stream((k - 1) % kAuxStreams);
+            if (!sts[k]) return LSTM_ERR_CUDA;
+        }
+        // events: fork, then "layer k finished chunk c"
+        std::vector<cudaEvent_t> ev((size_t)L * nch + 1, nullptr);
+        auto cleanup = [&] {
+            for (cudaEvent_t e : ev)
+                if (e) cudaEventDestroy(e);
+        };
+        for (auto& e : ev) {
+            if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+                e = nullptr;
+                cleanup();
+                return LSTM_ERR_CUDA;
+            }
+        }
+        auto fail = [&] { cleanup(); return LSTM_ERR_CUDA; };
+        // layer 0's projection of the whole sequence, on the caller's stream
+        if (project(0, x, reinterpret_cast<float*>(P(workspace, l.gx)), (long long)B * T, desc->batch_first != 0,
+                    stream) != cudaSuccess)
+            return fail();
+        if (cudaEventRecord(ev[(size_t)L * nch], stream) != cudaSuccess) return fail();
+        for (int k = 1; k < L; ++k)
+            if (cudaStreamWaitEvent(sts[k], ev[(size_t)L * nch], 0) != cudaSuccess) return fail();
+        // packed W_hh of every layer (the layers run at the same time)
+        const RecPlan& pw = l.fwd_wf;
+        const size_t whh_layer = (size_t)pw.nu * ((H + 3) & ~3) * 4 * pw.U * es;
+        for (int k = 0; k < L; ++k) {
+            PackHhFwdArgs ph{};
+            ph.H = H; ph.D = 1; ph.nu = pw.nu; ph.U = pw.U; ph.dt = l.dt;
+            ph.w[0] = w_hh[k];
+            ph.out = P(workspace, l.whh_wf) + (size_t)k * whh_layer;
+            if (timed(K_PACK, sts[k], [&] { return launch_pack_hh_fwd(ph, sts[k]); }) != cudaSuccess) return fail();
+        }
+        // issue in wavefront order: at stage q, layer k handles chunk q - k
+        for (int q = 0; q < nch + L - 1; ++q) {
+            for (int k = 0; k < L; ++k) {
+                const int c = q - k;
+                if (c < 0 || c >= nch) continue;
+                cudaStream_t st = sts[k];
+                const int t0 = t0s[c], t1 = c + 1 < nch ? t0s[c + 1] : T, Tc = t1 - t0;
+                float* gxk = reinterpret_cast<float*>(P(workspace, k % 2 == 0 ? l.gx : l.gx2));
+                if (k > 0) {
+                    if (cudaStreamWaitEvent(st, ev[(size_t)(k - 1) * nch + c], 0) != cudaSuccess) return fail();
+                    const void* below = reserve ? (const void*)P(reserve, l.hseq[k - 1]) : (const void*)P(workspace, l.seq[(k - 1) & 1]);
+                    if (project(k, static_cast<const char*>(below) + (size_t)t0 * B * H * es,
+                                gxk + (size_t)t0 * B * G, (long long)B * Tc, false, st) != cudaSuccess)
+                        return fail();
+                }
+                unsigned* ctr = reinterpret_cast<unsigned*>(P(workspace, l.ctr_w)) + (size_t)k * pw.nbg;
+                if (cudaMemsetAsync(ctr, 0, sizeof(unsigned) * pw.nbg, st) != cudaSuccess) return fail();
+                FwdRecArgs f{};
+                f.H = H; f.B = B; f.T = Tc; f.D = 1; f.p = pw; f.dt = l.dt;
+                f.gx = gxk + (size_t)t0 * B * G;
+                f.wpk = P(workspace, l.whh_wf) + (size_t)k * whh_layer;
+                char* hn_k = static_cast<char*>(h_n) + (size_t)k * state_elems * es;
+                float* cn_k = c_n + (size_t)k * state_elems;
+                if (c == 0) {
+                    f.h0 = h0 ? static_cast<const char*>(h0) + (size_t)k * state_elems * es : nullptr;
+                    f.c0 = c0 ? c0 + (size_t)k * state_elems : nullptr;
+                } else {
+                    f.h0 = hn_k;   // the state chunk c-1 ended in
+                    f.c0 = cn_k;
+                }
+                void* hseq = reserve ? P(reserve, l.hseq[k]) : P(workspace, l.seq[k & 1]);
+                f.hseq = (k < L - 1 || reserve) ? static_cast<char*>(hseq) + (size_t)t0 * B * H * es : nullptr;
+                f.hT = P(workspace, l.hTw[k]);
+                if (k == L - 1) {
+                    f.out_st = desc->batch_first ? (long long)H : (long long)B * H;
+                    f.out_sb = desc->batch_first ? (long long)T * H : (long long)H;
+                    f.out = static_cast<char*>(out) + (size_t)t0 * f.out_st * es;
+                }
+                f.h_n = hn_k;
+                f.c_n = cn_k;
+                if (reserve) {
+                    f.act = reinterpret_cast<float*>(P(reserve, l.act[k])) + (size_t)t0 * B * G;
+                    f.cst = reinterpret_cast<float*>(P(reserve, l.cst[k])) + (size_t)t0 * B * H;
+                }
+                f.ctr = ctr;
+                f.status = status;
+                f.timeout_ns = timeout_ns();
+                f.skip_block = f.skip_step = -1;
+                if (timed(K_FWD_REC_FFMA, st, [&] { return launch_fwd_rec(f, st); }) != cudaSuccess) return fail();
+                if (cudaEventRecord(ev[(size_t)k * nch + c], st) != cudaSuccess) return fail();
+            }
+        }
+        // join: the caller's stream waits for the last chunk of every layer
+        for (int k = 1; k < L; ++k)
+            if (cudaStreamWaitEvent(stream, ev[(size_t)k * nch + nch - 1], 0) != cudaSuccess) return fail();
+        cleanup();
+        return LSTM_OK;
+    }
+
     const void* layer_in = x;
     for (int k = 0; k < L; ++k) {
         const int in = in_size(l, k);
