@@ -26,6 +26,9 @@
 //                 order after the step's barrier (a reduce-scatter whose
 //                 traffic equals the forward's all-gather of h).
 #include <algorithm>
+#include <map>
+#include <mutex>
+#include <tuple>
 
 #include "lstm_device.cuh"
 #include "lstm_internal.h"
@@ -630,7 +633,55 @@ __global__ void pack_hh_rows_kernel(PackHhBwdArgs a) {
 }  // namespace
 
 // ================================================================ planning
+namespace {
+
+// Plans depend only on their arguments: computed once per argument set.
+struct PlanKey {
+    int kind, H, B, D, dt, sms;
+    size_t smem;
+    bool operator<(const PlanKey& o) const {
+        return std::tie(kind, H, B, D, dt, sms, smem) < std::tie(o.kind, o.H, o.B, o.D, o.dt, o.sms, o.smem);
+    }
+};
+
+template <typename F>
+RecPlan cached_plan(const PlanKey& k, F&& compute) {
+    static std::mutex mu;
+    static std::map<PlanKey, RecPlan> cache;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        auto it = cache.find(k);
+        if (it != cache.end()) return it->second;
+    }
+    const RecPlan p = compute();
+    std::lock_guard<std::mutex> lk(mu);
+    if (cache.size() > 4096) cache.clear();
+    cache[k] = p;
+    return p;
+}
+
+RecPlan plan_fwd_rec_uncached(int H, int B, int D, DType dt, int num_sms, size_t smem_max);
+RecPlan plan_bwd_rec_uncached(int H, int B, int D, DType wdt, int num_sms, size_t smem_max);
+
+}  // namespace
+
 RecPlan plan_fwd_rec(int H, int B, int D, DType dt, int num_sms, size_t smem_max) {
+    return cached_plan(PlanKey{0, H, B, D, (int)dt, num_sms, smem_max},
+                       [&] { return plan_fwd_rec_uncached(H, B, D, dt, num_sms, smem_max); });
+}
+
+RecPlan plan_bwd_rec(int H, int B, int D, DType wdt, int num_sms, size_t smem_max) {
+    return cached_plan(PlanKey{1, H, B, D, (int)wdt, num_sms, smem_max},
+                       [&] { return plan_bwd_rec_uncached(H, B, D, wdt, num_sms, smem_max); });
+}
+
+namespace {
+
+// Unit slices are powers of two: the products' warp tiling rounds a block's
+// row tiles up to its lane layout, so other widths (e.g. 14 units, which
+// would fill all 148 SMs at H = 512) cost as much per step as the next power
+// of two (measured on the 2-layer workload: matvec 3.23 us either way).
+RecPlan plan_fwd_rec_uncached(int H, int B, int D, DType dt, int num_sms, size_t smem_max) {
     const size_t es = dtype_size(dt);
     const int Hp = (H + 3) & ~3;
     RecPlan best{};
@@ -676,7 +727,7 @@ RecPlan plan_fwd_rec(int H, int B, int D, DType dt, int num_sms, size_t smem_max
     return best;
 }
 
-RecPlan plan_bwd_rec(int H, int B, int D, DType wdt, int num_sms, size_t smem_max) {
+RecPlan plan_bwd_rec_uncached(int H, int B, int D, DType wdt, int num_sms, size_t smem_max) {
     const int Hp = (H + 3) & ~3;
     const size_t wes = dtype_size(wdt);
     RecPlan best{};
@@ -718,6 +769,8 @@ RecPlan plan_bwd_rec(int H, int B, int D, DType wdt, int num_sms, size_t smem_ma
     }
     return best;
 }
+
+}  // namespace
 
 // ================================================================ launchers
 cudaError_t launch_fwd_rec(const FwdRecArgs& a, cudaStream_t s) {
