@@ -30,6 +30,8 @@
 //               d_ready.
 // Only bf16 inference uses this kernel.  Every wait is bounded: on a timeout
 // the kernel records LSTM_ERR_TIMEOUT in the status word and returns.
+#include <cuda_fp16.h>
+
 #include <algorithm>
 
 #include "lstm_device.cuh"
@@ -97,6 +99,21 @@ __device__ __forceinline__ float tanh_fast(float z) {
 // sigma(z) = (1 + tanh(z/2)) / 2: one special-function op instead of an
 // exponential and a reciprocal
 __device__ __forceinline__ float sigmoid_fast(float z) { return fmaf(0.5f, tanh_fast(0.5f * z), 0.5f); }
+
+// tanh of two values with one special-function op (f16x2: arguments and
+// results rounded to half precision, error near 2^-10 -- below the rounding
+// of h to bf16 that this path applies every step).
+__device__ __forceinline__ float2 tanh2(float a, float b) {
+    const __half2 x = __floats2half2_rn(a, b);
+    uint32_t r;
+    asm("tanh.approx.f16x2 %0, %1;" : "=r"(r) : "r"(*reinterpret_cast<const uint32_t*>(&x)));
+    return __half22float2(*reinterpret_cast<const __half2*>(&r));
+}
+
+__device__ __forceinline__ float2 sigmoid2(float a, float b) {
+    const float2 t = tanh2(0.5f * a, 0.5f * b);
+    return make_float2(fmaf(0.5f, t.x, 0.5f), fmaf(0.5f, t.y, 0.5f));
+}
 
 __device__ __forceinline__ uint32_t cluster_rank() {
     uint32_t r;
@@ -492,6 +509,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // v[4m + i]: gate gq at column 16cc + 4m + i.  Three xor
                     // exchanges inside each 4-lane group give lane gq all four
                     // gates at column 16cc + 4gq + i (gate X arrives in round gq ^ X).
+                    float gi[4], gf[4], gc[4], go[4];
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         float rcv[4];
@@ -500,34 +518,47 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int rr = 1; rr < 4; ++rr)
                             rcv[rr] =
                                 __shfl_xor_sync(0xffffffffu, sel4(v[i], v[4 + i], v[8 + i], v[12 + i], gq ^ rr), rr);
-                        const float pi = sel4(rcv[0], rcv[1], rcv[2], rcv[3], gq ^ 0);
-                        const float pf = sel4(rcv[0], rcv[1], rcv[2], rcv[3], gq ^ 1);
-                        const float pgg = sel4(rcv[0], rcv[1], rcv[2], rcv[3], gq ^ 2);
-                        const float po = sel4(rcv[0], rcv[1], rcv[2], rcv[3], gq ^ 3);
-                        const int lc = 16 * cc + 4 * gq + i;   // column within the own half
-                        const int col = own0 + lc;
-                        if (col >= nB) continue;
-                        const int bb = b0 + col;
-                        float c = creg[k][i];
-                        bf16 hv;
-                        if (!a.len || t < a.len[bb]) {
-                            const float ig = sigmoid_fast(pi), fg = sigmoid_fast(pf), gg = tanh_fast(pgg);
-                            const float og = sigmoid_fast(po);
-                            c = fg * c + ig * gg;
-                            creg[k][i] = c;
-                            hv = __float2bfloat16_rn(og * tanh_fast(c));
-                        } else {
-                            // padding of a variable-length row: the state stays
-                            hv = __ldcg(a.hx + ((size_t)(d * (T + 1) + s) * B + bb) * H + u);
-                        }
-                        // unit octet q of column lc, stored at octet q ^ gq
-                        // ((lc >> 2) & 3 == gq): the four columns of a warp's
-                        // store fall in different banks
-                        sh[lc * 32 + 8 * (q ^ gq) + (lane >> 2)] = hv;
-                        if (s == T - 1) {
-                            const int b = b0 + col;
-                            a.h_n[((size_t)d * B + b) * H + u] = hv;
-                            a.c_n[((size_t)d * B + b) * H + u] = c;
+                        gi[i] = sel4(rcv[0], rcv[1], rcv[2], rcv[3], gq ^ 0);
+                        gf[i] = sel4(rcv[0], rcv[1], rcv[2], rcv[3], gq ^ 1);
+                        gc[i] = sel4(rcv[0], rcv[1], rcv[2], rcv[3], gq ^ 2);
+                        go[i] = sel4(rcv[0], rcv[1], rcv[2], rcv[3], gq ^ 3);
+                    }
+                    // the cells of two columns at a time: every nonlinearity
+                    // is one f16x2 tanh for both
+#pragma unroll
+                    for (int i = 0; i < 4; i += 2) {
+                        const float2 ig = sigmoid2(gi[i], gi[i + 1]), fg = sigmoid2(gf[i], gf[i + 1]);
+                        const float2 og = sigmoid2(go[i], go[i + 1]), gg = tanh2(gc[i], gc[i + 1]);
+                        const float cn0 = fg.x * creg[k][i] + ig.x * gg.x;
+                        const float cn1 = fg.y * creg[k][i + 1] + ig.y * gg.y;
+                        const float2 tcn = tanh2(cn0, cn1);
+                        const float hn[2] = {og.x * tcn.x, og.y * tcn.y};
+                        const float cn[2] = {cn0, cn1};
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int lc = 16 * cc + 4 * gq + i + e;   // column within the own half
+                            const int col = own0 + lc;
+                            if (col >= nB) continue;
+                            const int bb = b0 + col;
+                            bf16 hv;
+                            float c = creg[k][i + e];
+                            if (!a.len || t < a.len[bb]) {
+                                c = cn[e];
+                                creg[k][i + e] = c;
+                                hv = __float2bfloat16_rn(hn[e]);
+                            } else {
+                                // padding of a variable-length row: the state stays
+                                hv = __ldcg(a.hx + ((size_t)(d * (T + 1) + s) * B + bb) * H + u);
+                            }
+                            // unit octet q of column lc, stored at octet q ^ gq
+                            // ((lc >> 2) & 3 == gq): the four columns of a warp's
+                            // store fall in different banks
+                            sh[lc * 32 + 8 * (q ^ gq) + (lane >> 2)] = hv;
+                            if (s == T - 1) {
+                                const int b = b0 + col;
+                                a.h_n[((size_t)d * B + b) * H + u] = hv;
+                                a.c_n[((size_t)d * B + b) * H + u] = c;
+                            }
                         }
                     }
                 }
@@ -545,6 +576,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int b = b0 + own0 + lc;
                     const uint4 val = *reinterpret_cast<const uint4*>(sh + lc * 32 + 8 * (oct ^ ((lc >> 2) & 3)));
                     *reinterpret_cast<uint4*>(hxo + (size_t)b * H + 8 * oct) = val;
+                }
+            }
+            tc::fence_proxy_async_global();
+            tc::named_bar_sync(1, kEpi);
+            if (warp == 2 && lane == 0) {
+                red_release_add(ctr, 1u);
+            }
+            trace_mark(a.trace, tr2, s, 8);
+            if (s + 1 < T) {
+                preload_gx(a.gx, d == 0 ? s + 1 : T - 2 - s, B, ldgx, prow0 + r, b0, own0, pcol0, ncc, nB, half, trow,
+                           d_ready);
+                trace_mark(a.trace, tr2, s + 1, 10);
+            }
+            // the layer output and the user output leave after the release
+            // and the accumulator hand-over: the group's next step waits only
+            // for the exchange copy
+            {
+                for (int idx = e; idx < NH * 4; idx += kEpi) {
+                    const int lc = idx >> 2, oct = idx & 3;
+                    if (own0 + lc >= nB) continue;
+                    const int b = b0 + own0 + lc;
+                    const uint4 val = *reinterpret_cast<const uint4*>(sh + lc * 32 + 8 * (oct ^ ((lc >> 2) & 3)));
                     const size_t uo = (size_t)d * H + 32 * j + 8 * oct;
                     if (a.hseq) *reinterpret_cast<uint4*>(a.hseq + ((size_t)t * B + b) * ldseq + uo) = val;
                     if (a.out && a.len && t >= a.len[b]) {   // padding: the user output is 0
@@ -563,17 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            tc::fence_proxy_async_global();
-            tc::named_bar_sync(1, kEpi);
-            if (warp == 2 && lane == 0) {
-                red_release_add(ctr, 1u);
-            }
-            trace_mark(a.trace, tr2, s, 8);
-            if (s + 1 < T) {
-                preload_gx(a.gx, d == 0 ? s + 1 : T - 2 - s, B, ldgx, prow0 + r, b0, own0, pcol0, ncc, nB, half, trow,
-                           d_ready);
-                trace_mark(a.trace, tr2, s + 1, 10);
-            }
+
         }
     }
     tc::tc_fence_before();
