@@ -246,6 +246,13 @@ __device__ __forceinline__ void preload_gx(const float* gx, int t, int B, size_t
     tc::mbar_arrive(d_ready);
 }
 
+// kWsmem: some of the block's W_hh chunks live in shared memory (plans with
+// more K chunks than tensor memory holds).  The two operand forms of
+// tcgen05.mma are compiled into separate kernels: a loop that can issue
+// either form (a branch between them) runs at 120-160 cycles per MMA, a loop
+// of one form at the tensor pipe's rate (55 cycles at N = 32, 128 at
+// N = 256; measured with the tcgen05.mma issue probe).
+template <bool kWsmem>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_rec_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmW, TcRecParams a) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -257,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int KT = H / 64;
     const int c_beg = (int)rank * a.KH, c_end = min(KT, c_beg + a.KH);
     const int nch = c_end - c_beg;                     // K chunks of this block (>= 1)
-    const int kc_smem = min(nch, a.kc_smem);           // of which in shared memory
+    const int kc_smem = kWsmem ? min(nch, a.kc_smem) : 0;   // of which in shared memory
     unsigned char* sW = smem;
     unsigned char* sH = smem + a.kc_smem * kChunkW;
     // partner's partial sums of the own columns, [NH/4][128 rows] float4 (a
@@ -401,16 +408,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int c = rot + i < nch ? rot + i : rot + i - nch;
                     if (i == 0) trace_mark(a.trace, tr0, s, 9);
                     const uint32_t b_base = tc::smem_u32(sH + st * hstage);
+                    if (kWsmem && c < kc_smem) {
+                        const uint32_t a_base = tc::smem_u32(sW + c * kChunkW);
 #pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        const uint64_t bd = tc::smem_desc_sw128(b_base + 32 * jj);
-                        if (c < kc_smem) {
-                            const uint64_t ad = tc::smem_desc_sw128(tc::smem_u32(sW + c * kChunkW) + 32 * jj);
-                            tc::mma_bf16(tmem, ad, bd, idesc, 1);
-                        } else {
-                            const uint32_t at = tmem + kAcol + (uint32_t)(c - kc_smem) * 32 + 8 * jj;
-                            tc::mma_bf16_ts(tmem, at, bd, idesc, 1);
-                        }
+                        for (int jj = 0; jj < 4; ++jj)
+                            tc::mma_bf16(tmem, tc::smem_desc_sw128(a_base + 32 * jj),
+                                         tc::smem_desc_sw128(b_base + 32 * jj), idesc, 1);
+                    } else {
+                        const uint32_t at = tmem + kAcol + (uint32_t)(c - kc_smem) * 32;
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj)
+                            tc::mma_bf16_ts(tmem, at + 8 * jj, tc::smem_desc_sw128(b_base + 32 * jj), idesc, 1);
                     }
                     tc::mma_commit(&empty[st]);
                     last = idx;
@@ -705,7 +713,10 @@ cudaError_t launch_tc_rec(const TcRecArgs& a, cudaStream_t s) {
     prm.trace = a.trace;
     prm.len = a.len;
     prm.ctr = a.ctr; prm.status = a.status; prm.timeout_ns = a.timeout_ns;
-    cudaError_t e = cudaFuncSetAttribute(tc_rec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
+    // one operand form per kernel: tensor memory only, unless chunks spill
+    // to shared memory
+    const auto kern = p.kc_smem > 0 ? tc_rec_kernel<true> : tc_rec_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(p.ctas);
@@ -726,10 +737,10 @@ cudaError_t launch_tc_rec(const TcRecArgs& a, cudaStream_t s) {
     // not be co-scheduled all the same, the bounded waits end the call with
     // LSTM_ERR_TIMEOUT instead of a hang.
     int clusters = 0;
-    e = cudaOccupancyMaxActiveClusters(&clusters, tc_rec_kernel, &cfg);
+    e = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
     if (e != cudaSuccess) return e;
     if (2 * clusters < p.ctas) return cudaErrorCooperativeLaunchTooLarge;
-    return cudaLaunchKernelEx(&cfg, tc_rec_kernel, tmH, tmW, prm);
+    return cudaLaunchKernelEx(&cfg, kern, tmH, tmW, prm);
 }
 
 }  // namespace lstm
