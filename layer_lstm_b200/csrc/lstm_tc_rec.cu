@@ -252,9 +252,13 @@ __device__ __forceinline__ void preload_gx(const float* gx, int t, int B, size_t
 // either form (a branch between them) runs at 120-160 cycles per MMA, a loop
 // of one form at the tensor pipe's rate (55 cycles at N = 32, 128 at
 // N = 256; measured with the tcgen05.mma issue probe).
-template <bool kWsmem>
+// kWhole: the block's whole K share of h_{t-1} fits the stage ring and comes
+// in as one 3-D TMA box per step (tmH3), chunk i into stage i; otherwise the
+// chunks stream through the ring one 2-D box each (tmH).
+template <bool kWsmem, bool kWhole>
 __global__ void __launch_bounds__(kThreads, 1)
-    tc_rec_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmW, TcRecParams a) {
+    tc_rec_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmH3,
+                  const __grid_constant__ CUtensorMap tmW, TcRecParams a) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);
     const int H = a.H, B = a.B, T = a.T, D = a.D, G = 4 * H;
@@ -325,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // memory by TMA, the rest in tensor memory (row r of the slice on lane r,
     // two bf16 per column) by the first four epilogue warps.
     if (warp == 0 && lane == 0) {
-        tc::prefetch_tmap(&tmH);
+        tc::prefetch_tmap(kWhole ? &tmH3 : &tmH);
         tc::prefetch_tmap(&tmW);
         if (kc_smem > 0) {
             tc::mbar_arrive_expect_tx(w_full, (uint32_t)(kc_smem * kChunkW));
@@ -370,6 +374,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 trace_mark(a.trace, tr0, s, 0);
                 const int row0 = (d * (T + 1) + s) * B + b0;
+                if (kWhole) {
+                    // the whole K share in one box: chunk i into stage i; the
+                    // ring is free once the previous step's MMAs completed
+                    if (s > 0 && !tc::mbar_wait(&empty[0], (s - 1) & 1, abort_flag, a.status, a.timeout_ns)) break;
+                    tc::mbar_arrive_expect_tx(&full[0], (uint32_t)(a.KH * hstage));
+                    tc::tma_load_3d(sH, &tmH3, 0, row0, c_beg, &full[0]);
+                    ++issued;
+                    trace_mark(a.trace, tr0, s, 1);
+                    continue;
+                }
                 for (int i = 0; i < nch; ++i) {
                     const int c = rot + i < nch ? rot + i : rot + i - nch;
                     const int st = issued % S, rnd = issued / S;
@@ -384,8 +398,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 trace_mark(a.trace, tr0, s, 1);
             }
             if (*abort_flag) {
-                for (int idx = issued > S ? issued - S : 0; idx < issued; ++idx)
-                    drain_wait(&full[idx % S], (idx / S) & 1);
+                if (kWhole) {
+                    if (issued > 0) drain_wait(&full[0], (issued - 1) & 1);
+                } else {
+                    for (int idx = issued > S ? issued - S : 0; idx < issued; ++idx)
+                        drain_wait(&full[idx % S], (idx / S) & 1);
+                }
             }
         }
     } else if (warp == 1) {
@@ -398,6 +416,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!tc::mbar_wait(d_ready, s & 1, abort_flag, a.status, a.timeout_ns)) break;
                 tc::tc_fence_after();
                 trace_mark(a.trace, tr0, s, 2);
+                if (kWhole) {
+                    if (!tc::mbar_wait(&full[0], s & 1, abort_flag, a.status, a.timeout_ns)) break;
+                    tc::tc_fence_after();
+                    trace_mark(a.trace, tr0, s, 9);
+                    for (int i = 0; i < nch; ++i) {
+                        const int c = i;
+                        const uint32_t b_base = tc::smem_u32(sH + i * hstage);
+                        if (kWsmem && c < kc_smem) {
+                            const uint32_t a_base = tc::smem_u32(sW + c * kChunkW);
+#pragma unroll
+                            for (int jj = 0; jj < 4; ++jj)
+                                tc::mma_bf16(tmem, tc::smem_desc_sw128(a_base + 32 * jj),
+                                             tc::smem_desc_sw128(b_base + 32 * jj), idesc, 1);
+                        } else {
+                            const uint32_t at = tmem + kAcol + (uint32_t)(c - kc_smem) * 32;
+#pragma unroll
+                            for (int jj = 0; jj < 4; ++jj)
+                                tc::mma_bf16_ts(tmem, at + 8 * jj, tc::smem_desc_sw128(b_base + 32 * jj), idesc, 1);
+                        }
+                    }
+                    tc::mma_commit(&empty[0]);
+                    last = s;
+                    tc::mma_commit(mma_done);
+                    trace_mark(a.trace, tr0, s, 3);
+                    continue;
+                }
                 for (int i = 0; i < nch; ++i) {
                     const int idx = s * nch + i, st = idx % S, rnd = idx / S;
                     if (!tc::mbar_wait(&full[st], rnd & 1, abort_flag, a.status, a.timeout_ns)) {
@@ -427,7 +471,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc::mma_commit(mma_done);
                 trace_mark(a.trace, tr0, s, 3);
             }
-            if (*abort_flag && last >= 0) drain_wait(&empty[last % S], (last / S) & 1);
+            if (*abort_flag && last >= 0) {
+                if (kWhole)
+                    drain_wait(&empty[0], last & 1);
+                else
+                    drain_wait(&empty[last % S], (last / S) & 1);
+            }
         }
     } else {
         // ------------------------------------------------------- epilogue
@@ -691,13 +740,39 @@ bool make_map_bf16(CUtensorMap* map, const void* base, long long rows, long long
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+// h_{t-1} as a 3-D tensor (k within a 64-wide chunk, row, chunk): a box of
+// {64, rows, chunks} lands the chunks one after another, each a 128-byte-
+// swizzled [rows][64] tile, as the 2-D boxes of single chunks would.
+bool make_map_bf16_chunks(CUtensorMap* map, const void* base, long long rows, long long cols, int box_rows,
+                          int box_chunks) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+        return false;
+    const EncodeTiledFn fn = reinterpret_cast<EncodeTiledFn>(p);
+    cuuint64_t dims[3] = {64, (cuuint64_t)rows, (cuuint64_t)(cols / 64)};
+    cuuint64_t strides[2] = {(cuuint64_t)(cols * 2), 128};
+    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, (cuuint32_t)box_chunks};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 cudaError_t launch_tc_rec(const TcRecArgs& a, cudaStream_t s) {
     const TcRecPlan& p = a.p;
-    CUtensorMap tmH, tmW;
+    CUtensorMap tmH, tmH3, tmW;
     const long long hrows = (long long)a.D * (a.T + 1) * a.B;
     if (!make_map_bf16(&tmH, a.hx, hrows, a.H, p.N)) return cudaErrorInvalidValue;
+    // one box per step when both blocks of a pair hold KH chunks and the
+    // ring holds them all
+    const int KT = a.H / 64;
+    const bool whole = KT % 2 == 0 && p.stages >= p.KH && p.KH <= 256 &&
+                       make_map_bf16_chunks(&tmH3, a.hx, hrows, a.H, p.N, p.KH);
+    if (!whole) tmH3 = tmH;
     if (!make_map_bf16(&tmW, a.wpk, (long long)a.D * 4 * a.H, a.H, kRows)) return cudaErrorInvalidValue;
     TcRecParams prm{};
     prm.H = a.H; prm.B = a.B; prm.T = a.T; prm.D = a.D;
@@ -715,7 +790,8 @@ cudaError_t launch_tc_rec(const TcRecArgs& a, cudaStream_t s) {
     prm.ctr = a.ctr; prm.status = a.status; prm.timeout_ns = a.timeout_ns;
     // one operand form per kernel: tensor memory only, unless chunks spill
     // to shared memory
-    const auto kern = p.kc_smem > 0 ? tc_rec_kernel<true> : tc_rec_kernel<false>;
+    const auto kern = p.kc_smem > 0 ? (whole ? tc_rec_kernel<true, true> : tc_rec_kernel<true, false>)
+                                    : (whole ? tc_rec_kernel<false, true> : tc_rec_kernel<false, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
@@ -740,7 +816,7 @@ cudaError_t launch_tc_rec(const TcRecArgs& a, cudaStream_t s) {
     e = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
     if (e != cudaSuccess) return e;
     if (2 * clusters < p.ctas) return cudaErrorCooperativeLaunchTooLarge;
-    return cudaLaunchKernelEx(&cfg, kern, tmH, tmW, prm);
+    return cudaLaunchKernelEx(&cfg, kern, tmH, tmH3, tmW, prm);
 }
 
 }  // namespace lstm
