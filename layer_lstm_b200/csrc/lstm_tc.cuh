@@ -170,6 +170,21 @@ __device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a_desc, uint6
         : "memory");
 }
 
+// One lane of a converged warp, chosen by elect.sync (the same lane each time
+// the full warp executes it); every lane of the warp must take part.  Issue
+// code of a whole-warp role: the warp waits on mbarriers together (a wait by
+// one lane of a diverged warp costs about 600 cycles on this device, by the
+// whole warp about 100) and the elected lane issues TMA, MMA and commits.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t p;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "elect.sync _|p, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(p));
+    return p != 0;
+}
+
 // Arrive on `bar` once all previously issued tcgen05.mma of this thread finish.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(

@@ -53,6 +53,7 @@ constexpr int kMaxTmemChunks = 8;      // 8 x 32 columns of W in tensor memory
 // never share an SM (each allocates all 512 tensor-memory columns).
 constexpr size_t kMinSmem = 120 * 1024;
 constexpr int kCtrStride = 32;         // unsigned words between group counters (one 128-byte line each)
+constexpr unsigned kFullMask = 0xffffffffu;
 
 struct TcRecParams {
     int H, B, T, D;
@@ -362,64 +363,82 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc::tc_fence_after();
 
+    // The producer and MMA warps run their loops as whole warps: every lane
+    // waits (warp-uniform outcome through a vote), one elected lane issues.
     if (warp == 0) {
         // ------------------------------------------------------ h producer
-        if (lane == 0) {
-            int issued = 0;
-            bool ok = true;
-            for (int s = 0; s < T && ok; ++s) {
-                if (s > 0) {
-                    if (!ctr_wait(ctr, (unsigned)(2 * a.nu * s), abort_flag, a.status, a.timeout_ns)) break;
-                    tc::fence_proxy_async_global();
-                }
-                trace_mark(a.trace, tr0, s, 0);
-                const int row0 = (d * (T + 1) + s) * B + b0;
-                if (kWhole) {
-                    // the whole K share in one box: chunk i into stage i; the
-                    // ring is free once the previous step's MMAs completed
-                    if (s > 0 && !tc::mbar_wait(&empty[0], (s - 1) & 1, abort_flag, a.status, a.timeout_ns)) break;
+        int issued = 0;
+        bool ok = true;
+        for (int s = 0; s < T && ok; ++s) {
+            if (s > 0) {
+                // the group counter is polled by one lane (a global load, not
+                // an mbarrier); __syncwarp orders its acquire before the
+                // elected lane's copy
+                bool got = true;
+                if (lane == 0) got = ctr_wait(ctr, (unsigned)(2 * a.nu * s), abort_flag, a.status, a.timeout_ns);
+                got = __shfl_sync(kFullMask, got, 0);
+                __syncwarp();
+                if (!got) break;
+                tc::fence_proxy_async_global();
+            }
+            trace_mark(a.trace, tr0, s, 0);
+            const int row0 = (d * (T + 1) + s) * B + b0;
+            if (kWhole) {
+                // the whole K share in one box: chunk i into stage i; the
+                // ring is free once the previous step's MMAs completed
+                if (s > 0 &&
+                    !__all_sync(kFullMask, tc::mbar_wait(&empty[0], (s - 1) & 1, abort_flag, a.status, a.timeout_ns)))
+                    break;
+                if (tc::elect_one()) {
                     tc::mbar_arrive_expect_tx(&full[0], (uint32_t)(a.KH * hstage));
                     tc::tma_load_3d(sH, &tmH3, 0, row0, c_beg, &full[0]);
-                    ++issued;
-                    trace_mark(a.trace, tr0, s, 1);
-                    continue;
                 }
-                for (int i = 0; i < nch; ++i) {
-                    const int c = rot + i < nch ? rot + i : rot + i - nch;
-                    const int st = issued % S, rnd = issued / S;
-                    if (!tc::mbar_wait(&empty[st], (rnd & 1) ^ 1, abort_flag, a.status, a.timeout_ns)) {
-                        ok = false;
-                        break;
-                    }
+                __syncwarp();
+                ++issued;
+                trace_mark(a.trace, tr0, s, 1);
+                continue;
+            }
+            for (int i = 0; i < nch; ++i) {
+                const int c = rot + i < nch ? rot + i : rot + i - nch;
+                const int st = issued % S, rnd = issued / S;
+                if (!__all_sync(kFullMask,
+                                tc::mbar_wait(&empty[st], (rnd & 1) ^ 1, abort_flag, a.status, a.timeout_ns))) {
+                    ok = false;
+                    break;
+                }
+                if (tc::elect_one()) {
                     tc::mbar_arrive_expect_tx(&full[st], (uint32_t)hstage);
                     tc::tma_load_2d(sH + st * hstage, &tmH, 64 * (c_beg + c), row0, &full[st]);
-                    ++issued;
                 }
-                trace_mark(a.trace, tr0, s, 1);
+                __syncwarp();
+                ++issued;
             }
-            if (*abort_flag) {
-                if (kWhole) {
-                    if (issued > 0) drain_wait(&full[0], (issued - 1) & 1);
-                } else {
-                    for (int idx = issued > S ? issued - S : 0; idx < issued; ++idx)
-                        drain_wait(&full[idx % S], (idx / S) & 1);
-                }
+            trace_mark(a.trace, tr0, s, 1);
+        }
+        if (*abort_flag) {
+            if (kWhole) {
+                if (issued > 0) drain_wait(&full[0], (issued - 1) & 1);
+            } else {
+                for (int idx = issued > S ? issued - S : 0; idx < issued; ++idx)
+                    drain_wait(&full[idx % S], (idx / S) & 1);
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA
-        if (lane == 0) {
-            const uint32_t idesc = tc::instr_desc(1, kRows, N);
-            bool ok = kc_smem == 0 || tc::mbar_wait(w_full, 0, abort_flag, a.status, a.timeout_ns);
-            int last = -1;
-            for (int s = 0; s < T && ok; ++s) {
-                if (!tc::mbar_wait(d_ready, s & 1, abort_flag, a.status, a.timeout_ns)) break;
+        // Each elected block issues its MMAs and their commits together, so
+        // a commit always follows the MMAs of its own thread.
+        const uint32_t idesc = tc::instr_desc(1, kRows, N);
+        bool ok = kc_smem == 0 || __all_sync(kFullMask, tc::mbar_wait(w_full, 0, abort_flag, a.status, a.timeout_ns));
+        int last = -1;
+        for (int s = 0; s < T && ok; ++s) {
+            if (!__all_sync(kFullMask, tc::mbar_wait(d_ready, s & 1, abort_flag, a.status, a.timeout_ns))) break;
+            tc::tc_fence_after();
+            trace_mark(a.trace, tr0, s, 2);
+            if (kWhole) {
+                if (!__all_sync(kFullMask, tc::mbar_wait(&full[0], s & 1, abort_flag, a.status, a.timeout_ns))) break;
                 tc::tc_fence_after();
-                trace_mark(a.trace, tr0, s, 2);
-                if (kWhole) {
-                    if (!tc::mbar_wait(&full[0], s & 1, abort_flag, a.status, a.timeout_ns)) break;
-                    tc::tc_fence_after();
-                    trace_mark(a.trace, tr0, s, 9);
+                trace_mark(a.trace, tr0, s, 9);
+                if (tc::elect_one()) {
                     for (int i = 0; i < nch; ++i) {
                         const int c = i;
                         const uint32_t b_base = tc::smem_u32(sH + i * hstage);
@@ -437,21 +456,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                     tc::mma_commit(&empty[0]);
-                    last = s;
                     tc::mma_commit(mma_done);
-                    trace_mark(a.trace, tr0, s, 3);
-                    continue;
                 }
-                for (int i = 0; i < nch; ++i) {
-                    const int idx = s * nch + i, st = idx % S, rnd = idx / S;
-                    if (!tc::mbar_wait(&full[st], rnd & 1, abort_flag, a.status, a.timeout_ns)) {
-                        ok = false;
-                        break;
-                    }
-                    tc::tc_fence_after();
-                    const int c = rot + i < nch ? rot + i : rot + i - nch;
-                    if (i == 0) trace_mark(a.trace, tr0, s, 9);
-                    const uint32_t b_base = tc::smem_u32(sH + st * hstage);
+                __syncwarp();
+                last = s;
+                trace_mark(a.trace, tr0, s, 3);
+                continue;
+            }
+            for (int i = 0; i < nch; ++i) {
+                const int idx = s * nch + i, st = idx % S, rnd = idx / S;
+                if (!__all_sync(kFullMask, tc::mbar_wait(&full[st], rnd & 1, abort_flag, a.status, a.timeout_ns))) {
+                    ok = false;
+                    break;
+                }
+                tc::tc_fence_after();
+                const int c = rot + i < nch ? rot + i : rot + i - nch;
+                if (i == 0) trace_mark(a.trace, tr0, s, 9);
+                const uint32_t b_base = tc::smem_u32(sH + st * hstage);
+                if (tc::elect_one()) {
                     if (kWsmem && c < kc_smem) {
                         const uint32_t a_base = tc::smem_u32(sW + c * kChunkW);
 #pragma unroll
@@ -465,18 +487,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tc::mma_bf16_ts(tmem, at + 8 * jj, tc::smem_desc_sw128(b_base + 32 * jj), idesc, 1);
                     }
                     tc::mma_commit(&empty[st]);
-                    last = idx;
+                    if (i == nch - 1) tc::mma_commit(mma_done);
                 }
-                if (!ok) break;
-                tc::mma_commit(mma_done);
-                trace_mark(a.trace, tr0, s, 3);
+                __syncwarp();
+                last = idx;
             }
-            if (*abort_flag && last >= 0) {
-                if (kWhole)
-                    drain_wait(&empty[0], last & 1);
-                else
-                    drain_wait(&empty[last % S], (last / S) & 1);
-            }
+            if (!ok) break;
+            trace_mark(a.trace, tr0, s, 3);
+        }
+        if (*abort_flag && last >= 0) {
+            if (kWhole)
+                drain_wait(&empty[0], last & 1);
+            else
+                drain_wait(&empty[last % S], (last / S) & 1);
         }
     } else {
         // ------------------------------------------------------- epilogue
