@@ -95,6 +95,14 @@ SMALL = {
                              state_std=0.3, seed=112),
     "bf16_tc_seqfirst": Workload("s", L=1, D=2, I=64, H=256, T=6, B=130, dtype="bf16",
                                  batch_first=False, seed=113),
+    # 256 batch columns per cluster, K chunks streamed through the stage ring
+    # (two groups of 245 columns, ragged); the same with a W_hh chunk in
+    # shared memory and an odd number of K chunks (H = 1088: 9 and 8 per
+    # block of a pair)
+    "bf16_tc_split": Workload("s", L=1, D=1, I=64, H=1024, T=3, B=490, dtype="bf16",
+                              state_std=0.3, seed=115),
+    "bf16_tc_split_wsmem": Workload("s", L=1, D=1, I=64, H=1088, T=3, B=480, dtype="bf16",
+                                    state_std=0.3, seed=116),
     "H1": Workload("s", L=1, D=1, I=3, H=1, T=4, B=3, dtype="f32", state_std=0.5, seed=108),
     # bf16 projection on 256 x 256 tiles (M = B*T >= 1024) with ragged M (1073) and K (72)
     "bf16_gemm256_ragged": Workload("s", L=2, D=1, I=72, H=128, T=29, B=37, dtype="bf16",
