@@ -49,7 +49,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-workloads", action="store_true",
-                    help="skip the per-workload lines (c1-c4) added beside the headline")
+                    help="skip the per-workload lines (the other configurations and the bf16 training step on c3's shape) added beside the headline")
     ap.add_argument("--rank-probe", action="store_true", help=argparse.SUPPRESS)
     return ap.parse_args()
 
@@ -578,7 +578,7 @@ def run_ours(args):
     # ------------------------------------------ the other workloads (1 GPU)
     others = None
     if rank == 0 and world == 1 and not args.no_workloads:
-        names = [n for n in ("c1", "c2", "c3", "c4", "c5") if n != wl.name]
+        names = [n for n in ("c1", "c2", "c3", "c4", "c5", "c3t") if n != wl.name]
         others = measure_workloads(names, steps=10, warmup=3, local=local, flush=flush, peaks=peaks,
                                    sm_mhz=sm_mhz)
 

@@ -635,7 +635,7 @@ lstm_status lstm_forward_varlen(const lstm_desc* desc, const int* lengths, const
         return timed(K_PROJ_SIMT, st, [&] { return launch_gemm(g, st); });
     };
 
-    const bool tc_path = l.tcr.ok && !reserve && tc_rec_enabled();
+    const bool tc_path = l.tcr.ok && tc_rec_enabled();
     if (l.wf && !lengths && !(reserve && l.dropout > 0.f) && !tc_path) {
         // ------------------------------------------------ layer wavefront
         // Layer k runs on stream k (the caller's stream for k = 0, a pool
@@ -769,7 +769,7 @@ lstm_status lstm_forward_varlen(const lstm_desc* desc, const int* lengths, const
         }
 
         void* hseq_tc = reserve ? P(reserve, l.hseq[k]) : P(workspace, l.seq[k & 1]);
-        if (!reserve && l.tcr.ok && tc_rec_enabled()) {
+        if (tc_path) {
             // tensor-core recurrence: packed W_hh rows, h0 into exchange slot 0
             PackIhArgs pw{};
             pw.H = H; pw.in = H; pw.D = D; pw.dt = l.dt;
@@ -791,7 +791,7 @@ lstm_status lstm_forward_varlen(const lstm_desc* desc, const int* lengths, const
             tr.wpk = P(workspace, l.whh_tc);
             tr.c0 = c0 ? c0 + (size_t)k * state_elems : nullptr;
             tr.hx = P(workspace, l.hx);
-            tr.hseq = k < L - 1 ? hseq_tc : nullptr;
+            tr.hseq = (k < L - 1 || reserve) ? hseq_tc : nullptr;
             if (k == L - 1) {
                 tr.out = out;
                 tr.out_st = desc->batch_first ? (long long)D * H : (long long)B * D * H;
@@ -804,8 +804,18 @@ lstm_status lstm_forward_varlen(const lstm_desc* desc, const int* lengths, const
             tr.timeout_ns = timeout_ns();
             tr.trace = trace_for(LSTM_TRACE_FWD_REC_TC, T, stream);
             tr.len = lengths;
+            if (reserve) {
+                tr.act = reinterpret_cast<float*>(P(reserve, l.act[k]));
+                tr.cst = reinterpret_cast<float*>(P(reserve, l.cst[k]));
+            }
             LSTM_CUDA(timed(K_FWD_REC_TC, stream, [&] { return launch_tc_rec(tr, stream); }));
             layer_in = hseq_tc;
+            if (reserve && l.dropout > 0.f && k < L - 1) {
+                void* dropped = P(reserve, l.hdrop[k]);
+                const DropoutArgs da = dropout_args(desc, k, hseq_tc, dropped, l.dt, (long long)B * T * D * H);
+                LSTM_CUDA(timed(K_DROPOUT, stream, [&] { return launch_dropout(da, stream); }));
+                layer_in = dropped;
+            }
             continue;
         }
 

@@ -140,7 +140,7 @@ struct FwdRecArgs {
 cudaError_t launch_fwd_rec(const FwdRecArgs& a, cudaStream_t s);
 RecPlan plan_fwd_rec(int H, int B, int D, DType dt, int num_sms, size_t smem_max);
 
-// Tensor-core forward recurrence (bf16, inference).  W_hh packed rows
+// Tensor-core forward recurrence (bf16; inference, and training with act/cst).  W_hh packed rows
 // [D*4H][H] bf16 (order 4u+q); hx exchange [D][T+1][B][H] bf16 with slot 0 =
 // h0 (or zeros) filled before the launch.
 struct TcRecPlan {
@@ -165,6 +165,8 @@ struct TcRecArgs {
     uint64_t timeout_ns;
     unsigned long long* trace;  // [kTraceSteps][kTraceEvents] or null
     const int* len;             // [B] valid steps per row, or null (all T)
+    float* act;                 // training: [D][T][B][4H] gate activations, or null (inference)
+    float* cst;                 // training: [D][T][B][H] cell states
 };
 cudaError_t launch_tc_rec(const TcRecArgs& a, cudaStream_t s);
 

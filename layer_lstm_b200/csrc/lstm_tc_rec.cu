@@ -28,8 +28,9 @@
 //               h_t and arrive on the group counter; then load Gx[t+1] (L2
 //               prefetched one step ahead) into the accumulator and signal
 //               d_ready.
-// Only bf16 inference uses this kernel.  Every wait is bounded: on a timeout
-// the kernel records LSTM_ERR_TIMEOUT in the status word and returns.
+// bf16 only.  In training the cells also write the gate activations and cell
+// states the backward reads.  Every wait is bounded: on a timeout the kernel
+// records LSTM_ERR_TIMEOUT in the status word and returns.
 #include <cuda_fp16.h>
 
 #include <algorithm>
@@ -71,6 +72,8 @@ struct TcRecParams {
     uint64_t timeout_ns;
     unsigned long long* trace;   // per-step timeline of block 0, or null
     const int* len;              // [B] valid steps per row, or null (all T)
+    float* act;                  // training: [D][T][B][G] gate activations (i, f, g, o of unit u at 4u), or null
+    float* cst;                  // training: [D][T][B][H] cell states
 };
 
 // Branch-free choice among four registers by a lane-dependent index k in
@@ -256,7 +259,9 @@ __device__ __forceinline__ void preload_gx(const float* gx, int t, int B, size_t
 // kWhole: the block's whole K share of h_{t-1} fits the stage ring and comes
 // in as one 3-D TMA box per step (tmH3), chunk i into stage i; otherwise the
 // chunks stream through the ring one 2-D box each (tmH).
-template <bool kWsmem, bool kWhole>
+// kTrain: the cells also store the gate activations and cell states the
+// backward reads (a separate instance, so inference carries none of it).
+template <bool kWsmem, bool kWhole, bool kTrain>
 __global__ void __launch_bounds__(kThreads, 1)
     tc_rec_kernel(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmH3,
                   const __grid_constant__ CUtensorMap tmW, TcRecParams a) {
@@ -622,13 +627,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const int bb = b0 + col;
                             bf16 hv;
                             float c = creg[k][i + e];
-                            if (!a.len || t < a.len[bb]) {
+                            const bool valid = !a.len || t < a.len[bb];
+                            if (valid) {
                                 c = cn[e];
                                 creg[k][i + e] = c;
                                 hv = __float2bfloat16_rn(hn[e]);
                             } else {
                                 // padding of a variable-length row: the state stays
                                 hv = __ldcg(a.hx + ((size_t)(d * (T + 1) + s) * B + bb) * H + u);
+                            }
+                            if (kTrain) {   // what the backward reads (zero gates at padding)
+                                const size_t row = ((size_t)d * T + t) * B + bb;
+                                *reinterpret_cast<float4*>(a.act + row * G + 4 * u) =
+                                    valid ? make_float4(e ? ig.y : ig.x, e ? fg.y : fg.x, e ? gg.y : gg.x,
+                                                        e ? og.y : og.x)
+                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+                                a.cst[row * H + u] = c;
                             }
                             // unit octet q of column lc, stored at octet q ^ gq
                             // ((lc >> 2) & 3 == gq): the four columns of a warp's
@@ -811,10 +825,16 @@ cudaError_t launch_tc_rec(const TcRecArgs& a, cudaStream_t s) {
     prm.trace = a.trace;
     prm.len = a.len;
     prm.ctr = a.ctr; prm.status = a.status; prm.timeout_ns = a.timeout_ns;
+    prm.act = a.act; prm.cst = a.cst;
     // one operand form per kernel: tensor memory only, unless chunks spill
     // to shared memory
-    const auto kern = p.kc_smem > 0 ? (whole ? tc_rec_kernel<true, true> : tc_rec_kernel<true, false>)
-                                    : (whole ? tc_rec_kernel<false, true> : tc_rec_kernel<false, false>);
+    const bool train = a.act != nullptr;
+    using Kern = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, TcRecParams);
+    static const Kern kTable[8] = {tc_rec_kernel<false, false, false>, tc_rec_kernel<false, false, true>,
+                                   tc_rec_kernel<false, true, false>,  tc_rec_kernel<false, true, true>,
+                                   tc_rec_kernel<true, false, false>,  tc_rec_kernel<true, false, true>,
+                                   tc_rec_kernel<true, true, false>,   tc_rec_kernel<true, true, true>};
+    const auto kern = kTable[(p.kc_smem > 0 ? 4 : 0) + (whole ? 2 : 0) + (train ? 1 : 0)];
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};

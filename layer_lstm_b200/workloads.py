@@ -75,6 +75,9 @@ WORKLOADS = {
                    w_k=1.0 / 32, seed=1004),
     "c5": Workload("c5", L=2, D=1, I=256, H=512, T=128, B=64, dtype="f32",
                    train=True, state_std=0.1, w_k=1.0 / math.sqrt(512), seed=1005),
+    # bf16 BPTT on c3's shape (bidirectional, bf16 weights and activations)
+    "c3t": Workload("c3t", L=2, D=2, I=512, H=1024, T=256, B=32, dtype="bf16",
+                    train=True, w_k=1.0 / 32, seed=1006),
 }
 
 DESCRIPTIONS = {
@@ -83,6 +86,7 @@ DESCRIPTIONS = {
     "c3": "2-layer bidirectional LSTM I512 H1024 T256 B32 bf16 forward",
     "c4": "1-layer LSTM I1024 H1024 T64 B512 bf16 forward",
     "c5": "2-layer LSTM I256 H512 T128 B64 fp32 forward + BPTT training step",
+    "c3t": "2-layer bidirectional LSTM I512 H1024 T256 B32 bf16 forward + BPTT training step",
 }
 
 

@@ -144,6 +144,11 @@ TRAIN = {
     # c3's layer shapes (H = 1024, bidirectional, 2 layers) on a short sequence
     "bf16_c3_shape": Workload("s", L=2, D=2, I=512, H=1024, T=12, B=8, dtype="bf16", w_k=1 / 32,
                               train=True, seed=145),
+    # tensor-core forward in training (H = 128) with inter-layer dropout and
+    # variable lengths: saved gates are zero and c is carried at padding
+    "bf16_tc_dropout_varlen": Workload("s", L=2, D=2, I=32, H=128, T=8, B=12, dtype="bf16",
+                                       state_std=0.3, train=True, dropout=0.25, dropout_seed=19,
+                                       varlen=True, seed=146),
 }
 
 
