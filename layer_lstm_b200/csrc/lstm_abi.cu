@@ -1030,11 +1030,17 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
         float* din = k == 0 ? dxf : reinterpret_cast<float*>(P(workspace, l.dseq[cur]));
         // Tensor-core weight phase: dW = dG^T [In | H_prev] per direction over
         // K = B*T (one GEMM writes dW_ih and dW_hh), dIn = dG [W_ih_0; W_ih_1].
-        float* dGT = reinterpret_cast<float*>(P(workspace, l.dGT));
-        float* bop = reinterpret_cast<float*>(P(workspace, l.bop));
-        float* wcatT = reinterpret_cast<float*>(P(workspace, l.wcatT));
+        // bf16 problems run it in bf16 (dG rounded to bf16, the other
+        // operands exact in bf16, float32 accumulation), float32 problems in
+        // 3xTF32.  The operand buffers hold either element type.
+        const bool wbf = bf;
+        const DType wdt = wbf ? DType::BF16 : DType::F32;
+        const size_t wes = wbf ? 2 : 4;
+        char* dGT = P(workspace, l.dGT);
+        char* bop = P(workspace, l.bop);
+        char* wcatT = P(workspace, l.wcatT);
         TcGemmArgs tw{};
-        tw.M = G; tw.N = in + H; tw.K = (int)BTl; tw.dt = DType::F32;
+        tw.M = G; tw.N = in + H; tw.K = (int)BTl; tw.dt = wdt;
         tw.A = dGT; tw.lda = BTl; tw.B = bop; tw.ldb = BTl;
         tw.C = dw_ih[k * D]; tw.ldc = in; tw.C1 = dw_hh[k * D]; tw.ldc1 = H; tw.n_split = in;
         tw.status = status; tw.timeout_ns = timeout_ns(); tw.num_sms = device_info().sms;
@@ -1042,8 +1048,10 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
         tw.ws = reinterpret_cast<float*>(P(workspace, l.gemm_ws));
         tw.ws_floats = (long long)l.gemm_ws_floats;
         TcGemmArgs tx{};
-        tx.M = (int)BTl; tx.N = in; tx.K = D * G; tx.dt = DType::F32;
-        tx.A = dG; tx.lda = ldg; tx.B = wcatT; tx.ldb = (long long)D * G;
+        tx.M = (int)BTl; tx.N = in; tx.K = D * G; tx.dt = wdt;
+        // bf16: a bf16 copy of dG, written into dGT's space once the dW GEMMs are done
+        tx.A = wbf ? static_cast<const void*>(dGT) : static_cast<const void*>(dG);
+        tx.lda = ldg; tx.B = wcatT; tx.ldb = (long long)D * G;
         tx.C = din; tx.ldc = in;
         if (k == 0 && desc->batch_first) { tx.remap_T = -T; tx.remap_B = B; }
         tx.status = status; tx.timeout_ns = timeout_ns(); tx.num_sms = device_info().sms;
@@ -1052,10 +1060,10 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
         if (tc_ok) {
             TransposeArgs ta{};
             ta.M = (int)BTl; ta.C = D * G; ta.mode = 0; ta.src = dG; ta.lds = ldg;
-            ta.dst = dGT; ta.ldd = BTl;
+            ta.dst = dGT; ta.ldd = BTl; ta.dst_bf16 = wbf;
             LSTM_CUDA(timed(K_TRANSPOSE, stream, [&] { return launch_transpose(ta, stream); }));
             for (int d = 0; d < D; ++d) {
-                float* bo = bop + (size_t)d * (in + H) * BTl;
+                char* bo = bop + (size_t)d * (in + H) * BTl * wes;
                 TransposeArgs ti{};
                 ti.M = (int)BTl; ti.C = in; ti.mode = 0;
                 if (k == 0) {
@@ -1065,16 +1073,16 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
                     ti.src = layer_in;
                     ti.lds = in;
                 }
-                ti.dst = bo; ti.ldd = BTl;
+                ti.dst = bo; ti.ldd = BTl; ti.dst_bf16 = wbf;
                 LSTM_CUDA(timed(K_TRANSPOSE, stream, [&] { return launch_transpose(ti, stream); }));
                 TransposeArgs th{};
                 th.M = (int)BTl; th.C = H; th.mode = 1;
                 th.src = hs + (size_t)d * H; th.lds = ldh; th.T = T; th.B = B; th.dir = d;
                 th.h0 = h0f ? h0f + ((size_t)k * D + d) * B * H : nullptr;
-                th.dst = bo + (size_t)in * BTl; th.ldd = BTl;
+                th.dst = bo + (size_t)in * BTl * wes; th.ldd = BTl; th.dst_bf16 = wbf;
                 LSTM_CUDA(timed(K_TRANSPOSE, stream, [&] { return launch_transpose(th, stream); }));
                 TcGemmArgs twd = tw;
-                twd.A = dGT + (size_t)d * G * BTl;
+                twd.A = dGT + (size_t)d * G * BTl * wes;
                 twd.B = bo;
                 twd.C = dw_ih[k * D + d];
                 twd.C1 = dw_hh[k * D + d];
@@ -1085,9 +1093,13 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
                 TransposeArgs tww{};
                 tww.M = G; tww.C = in; tww.mode = 0;
                 tww.src = wihf[k * D + d]; tww.lds = in;
-                tww.dst = wcatT + (size_t)d * G; tww.ldd = (long long)D * G;
+                tww.dst = wcatT + (size_t)d * G * wes; tww.ldd = (long long)D * G; tww.dst_bf16 = wbf;
                 LSTM_CUDA(timed(K_TRANSPOSE, stream, [&] { return launch_transpose(tww, stream); }));
             }
+            if (wbf)
+                LSTM_CUDA(timed(K_TRANSPOSE, stream, [&] {
+                    return launch_convert(dG, DType::F32, dGT, DType::BF16, BTl * ldg, stream);
+                }));
             {
                 int nl = 1;
                 LSTM_CUDA(timed(K_DX_TC, stream, [&] { return launch_tc_gemm(tx, stream, &nl); }, &nl));

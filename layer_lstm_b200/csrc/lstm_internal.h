@@ -62,7 +62,8 @@ bool tc_gemm_supported(const TcGemmArgs& g);
 // *nlaunch (if given) = kernels launched: 2 when K was split (GEMM + reduction).
 cudaError_t launch_tc_gemm(const TcGemmArgs& g, cudaStream_t s, int* nlaunch = nullptr);
 
-// dst[c*ldd + m] = src(m, c) for m < M, c < C (float32).
+// dst[c*ldd + m] = src(m, c) for m < M, c < C (float32 source; float32
+// destination, or bf16 rounded to nearest even when dst_bf16).
 //  mode 0: src(m, c) = src[row(m)*lds + c], row(m) = m, or with bt_remap the
 //          time-major index m = t*B + b read from a batch-first (b*T + t) array.
 //  mode 1: h_{t-1} of one direction in its own time order: for m = t*B + b,
@@ -73,7 +74,8 @@ struct TransposeArgs {
     const float* src; long long lds;
     int bt_remap, T, B, dir;
     const float* h0;
-    float* dst; long long ldd;
+    void* dst; long long ldd;
+    int dst_bf16;
 };
 cudaError_t launch_transpose(const TransposeArgs& a, cudaStream_t s);
 

@@ -495,7 +495,12 @@ __global__ void transpose_kernel(TransposeArgs a) {
     __syncthreads();
     for (int i = ty; i < 32; i += 8) {
         const int c = c0 + i, m = m0 + tx;
-        if (m < a.M && c < a.C) a.dst[(long long)c * a.ldd + m] = tile[tx][i];
+        if (m < a.M && c < a.C) {
+            if (a.dst_bf16)
+                static_cast<bf16*>(a.dst)[(long long)c * a.ldd + m] = __float2bfloat16_rn(tile[tx][i]);
+            else
+                static_cast<float*>(a.dst)[(long long)c * a.ldd + m] = tile[tx][i];
+        }
     }
 }
 

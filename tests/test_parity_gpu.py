@@ -125,7 +125,8 @@ TRAIN = {
     "B1_T1": SMALL["B1_T1"].replace(train=True),
     "f32_bi_wide": Workload("s", L=1, D=2, I=33, H=64, T=6, B=40, dtype="f32", state_std=0.2,
                             train=True, seed=110),
-    # bf16 BPTT (float32 arithmetic on widened copies; W_hh rows resident in bf16)
+    # bf16 BPTT: the recurrence in float32 on widened copies (W_hh rows resident
+    # in bf16); the weight phase in bf16 (dG rounded to bf16) with float32 sums
     "bf16_bi_2layer": Workload("s", L=2, D=2, I=64, H=96, T=11, B=9, dtype="bf16", state_std=0.3,
                                train=True, seed=141),
     "bf16_uni_ragged": Workload("s", L=1, D=1, I=50, H=130, T=8, B=20, dtype="bf16", state_std=0.3,
