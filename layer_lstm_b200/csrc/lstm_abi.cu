@@ -93,12 +93,12 @@ uint64_t timeout_ns() {
 // CUDA cores.
 enum Kind {
     K_PACK = 0, K_PROJ_TC, K_PROJ_SIMT, K_FWD_REC_TC, K_FWD_REC_FFMA, K_BWD_REC_FFMA, K_DW_TC, K_DW_SIMT,
-    K_DX_TC, K_DX_SIMT, K_DB, K_COPY, K_TRANSPOSE, K_DROPOUT, K_COUNT
+    K_DX_TC, K_DX_SIMT, K_DB, K_COPY, K_TRANSPOSE, K_DROPOUT, K_BWD_REC_TC, K_COUNT
 };
 const char* const kKindNames[K_COUNT] = {"pack",       "proj_gemm_tc", "proj_gemm_simt", "fwd_rec_tc",
                                          "fwd_rec_ffma", "bwd_rec_ffma", "dw_gemm_tc",   "dw_gemm_simt",
                                          "dx_gemm_tc", "dx_gemm_simt", "db_reduce",    "seq_copy",
-                                         "transpose",  "dropout"};
+                                         "transpose",  "dropout", "bwd_rec_tc"};
 
 // Dropout launch for boundary `layer` over n time-major elements.
 DropoutArgs dropout_args(const lstm_desc* d, int layer, const void* src, void* dst, DType dt, long long n) {
@@ -236,6 +236,8 @@ struct Layout {
     int nbg_ctr;       // counter stride per (layer, direction) of the FFMA forward recurrence
     bool bwd_ok;
     // workspace offsets
+    TcBwdPlan tcb;     // tensor-core BPTT recurrence (bf16), if it fits
+    size_t ctr_tcb, dax, wT_tcb;
     size_t status, ctr_f, ctr_b, ctr_tc, ctr_end, wih[32], bias[32], whh_f, whh_b, gx, hT, seq[2], dG, dseq[2], xt,
         dbpart, P, dGT, bop, wcatT, hx, whh_tc, bias_dummy, gemm_ws, total;
     size_t gemm_ws_floats;
@@ -296,6 +298,7 @@ bool make_layout(const lstm_desc* d, Layout& l) {
     l.bwd = plan_bwd_rec(l.H, Bp, l.D, l.dt, dev.sms, smem_max);
     l.bwd_ok = l.bwd.ctas > 0;
     l.tcr = l.dt == DType::BF16 ? plan_tc_rec(l.H, Bp, l.D, dev.sms, smem_max) : TcRecPlan{};
+    l.tcb = l.dt == DType::BF16 ? plan_tc_bwd(l.H, Bp, l.D, dev.sms, smem_max) : TcBwdPlan{};
     const size_t TB = (size_t)l.T * l.B;
     size_t o = 0;
     l.status = o; o += al(sizeof(int));
@@ -305,6 +308,7 @@ bool make_layout(const lstm_desc* d, Layout& l) {
     // tensor-core recurrence: one counter per (layer, direction, group), each
     // on its own 128-byte line
     l.ctr_tc = o; o += al(l.tcr.ok ? sizeof(unsigned) * 32 * (size_t)l.L * l.D * l.tcr.nbg : 0);
+    l.ctr_tcb = o; o += al(l.tcb.ok ? sizeof(unsigned) * 32 * (size_t)l.L * l.D * l.tcb.nbg : 0);
     l.ctr_end = o;
     for (int k = 0; k < l.L; ++k) {
         l.wih[k] = o; o += al((size_t)l.D * l.G * in_size(l, k) * l.es);
@@ -347,7 +351,11 @@ bool make_layout(const lstm_desc* d, Layout& l) {
     l.dseq[0] = o; o += al(TB * maxin * 4);
     l.dseq[1] = o; o += al(TB * maxin * 4);
     l.xt = o; o += al(TB * l.I * 4);
-    l.dbpart = o; o += al((size_t)l.D * (l.bwd_ok ? l.bwd.nbg : 1) * l.G * 4);
+    const int nbg_db = std::max(l.bwd_ok ? l.bwd.nbg : 1, l.tcb.ok ? l.tcb.nbg : 1);
+    l.dbpart = o; o += al((size_t)l.D * nbg_db * l.G * 4);
+    // tensor-core BPTT: packed W_hh^T and the bf16 exchange of the gate gradients
+    l.wT_tcb = o; o += al(l.tcb.ok ? (size_t)l.D * l.H * l.G * 2 : 0);
+    l.dax = o; o += al(l.tcb.ok ? (size_t)l.D * (l.T + 1) * l.B * l.G * 2 : 0);
     l.P = o; o += al(l.bwd_ok ? (size_t)2 * l.D * l.bwd.nbg * l.bwd.nu * l.bwd.Bg * Hp * 4 : 0);
     l.dGT = o; o += al(TB * l.D * l.G * 4);
     l.bop = o; o += al((size_t)l.D * (maxin + l.H) * TB * 4);
@@ -985,12 +993,17 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
     int cur = 0;
     for (int k = L - 1; k >= 0; --k) {
         const int in = in_size(l, k);
-        PackHhBwdArgs pb{};
-        pb.H = H; pb.D = D; pb.nu = l.bwd.nu; pb.U = l.bwd.U;
-        pb.dt = l.dt;
-        for (int d = 0; d < D; ++d) pb.w[d] = w_hh[k * D + d];
-        pb.out = P(workspace, l.whh_b);
-        LSTM_CUDA(timed(K_PACK, stream, [&] { return launch_pack_hh_rows(pb, stream); }));
+        // bf16: the tensor-core BPTT recurrence when its plan fits (the same
+        // switch as the forward's engine), else the CUDA-core one
+        const bool tcb = bf && l.tcb.ok && tc_rec_enabled();
+        if (!tcb) {
+            PackHhBwdArgs pb{};
+            pb.H = H; pb.D = D; pb.nu = l.bwd.nu; pb.U = l.bwd.U;
+            pb.dt = l.dt;
+            for (int d = 0; d < D; ++d) pb.w[d] = w_hh[k * D + d];
+            pb.out = P(workspace, l.whh_b);
+            LSTM_CUDA(timed(K_PACK, stream, [&] { return launch_pack_hh_rows(pb, stream); }));
+        }
 
         BwdRecArgs b{};
         b.H = H; b.B = B; b.T = T; b.D = D; b.p = l.bwd;
@@ -1014,11 +1027,34 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
         b.len = lengths;
         b.skip_block = skip_arrival().bwd_block;
         b.skip_step = skip_arrival().bwd_step;
-        LSTM_CUDA(timed(K_BWD_REC_FFMA, stream, [&] { return launch_bwd_rec(b, stream); }));
+        if (tcb) {
+            PackWtArgs pw{};
+            pw.H = H; pw.D = D;
+            for (int d = 0; d < D; ++d) pw.w[d] = w_hh[k * D + d];
+            pw.out = P(workspace, l.wT_tcb);
+            LSTM_CUDA(timed(K_PACK, stream, [&] { return launch_pack_wT(pw, stream); }));
+            TcBwdArgs tb{};
+            tb.H = H; tb.B = B; tb.T = T; tb.D = D; tb.p = l.tcb;
+            tb.wT = pw.out;
+            tb.act = b.act; tb.cst = b.cst; tb.c0 = b.c0;
+            tb.dy = b.dy; tb.dy_st = b.dy_st; tb.dy_sb = b.dy_sb;
+            tb.grad_hn = b.grad_hn; tb.grad_cn = b.grad_cn;
+            tb.dG = dG;
+            tb.dax = P(workspace, l.dax);
+            tb.dh0 = b.dh0; tb.dc0 = b.dc0; tb.dbpart = b.dbpart;
+            tb.ctr = reinterpret_cast<unsigned*>(P(workspace, l.ctr_tcb)) + (size_t)k * D * l.tcb.nbg * 32;
+            tb.status = status;
+            tb.timeout_ns = timeout_ns();
+            tb.len = lengths;
+            int nl = 1;
+            LSTM_CUDA(timed(K_BWD_REC_TC, stream, [&] { return launch_tc_bwd(tb, stream, &nl); }, &nl));
+        } else {
+            LSTM_CUDA(timed(K_BWD_REC_FFMA, stream, [&] { return launch_bwd_rec(b, stream); }));
+        }
 
         if (desc->bias) {
             DbArgs db{};
-            db.G = G; db.D = D; db.nbg = l.bwd.nbg; db.dbpart = b.dbpart;
+            db.G = G; db.D = D; db.nbg = tcb ? l.tcb.nbg : l.bwd.nbg; db.dbpart = b.dbpart;
             for (int d = 0; d < D; ++d) { db.db_ih[d] = db_ih[k * D + d]; db.db_hh[d] = db_hh[k * D + d]; }
             LSTM_CUDA(timed(K_DB, stream, [&] { return launch_db_reduce(db, stream); }));
         }

@@ -172,6 +172,47 @@ struct TcRecArgs {
 };
 cudaError_t launch_tc_rec(const TcRecArgs& a, cudaStream_t s);
 
+// Tensor-core BPTT recurrence (bf16 W_hh; float32 state and gate
+// gradients; the gate gradients of each step exchanged in bf16).  Clusters of
+// 8 blocks per (direction, batch group, 128-unit slice) split K = 4H.
+struct TcBwdPlan {
+    bool ok;
+    int nbg, Bg, N, nsl, nch, ctas;   // nsl slices of 128 units, nch 64-gate chunks per block
+    size_t smem;
+};
+TcBwdPlan plan_tc_bwd(int H, int B, int D, int num_sms, size_t smem_max);
+
+struct TcBwdArgs {
+    int H, B, T, D;
+    TcBwdPlan p;
+    const void* wT;             // [D][H][4H] bf16: row u, column 4u'+q holds W_hh[q*H + u'][u]
+    const float* act;           // [D][T][B][4H] gate activations (i, f, g, o of unit u at 4u)
+    const float* cst;           // [D][T][B][H] cell states
+    const float* c0;            // [D][B][H] or null
+    const float* dy; long long dy_st, dy_sb;   // dL/dh_t of this layer's output, element (t, b, d*H + u)
+    const float* grad_hn;       // [D][B][H] or null
+    const float* grad_cn;       // [D][B][H] or null
+    float* dG;                  // [T][B][D*4H] gate gradients, standard row order q*H + u
+    void* dax;                  // [D][T+1][B][4H] bf16 exchange of the gate gradients (order 4u+q)
+    float* dh0; float* dc0;     // [D][B][H]
+    float* dbpart;              // [D][nbg][4H] bias-gradient partial of each batch group
+    unsigned* ctr;              // [D][nbg] group counters, 32 words apart, zeroed
+    int* status;
+    uint64_t timeout_ns;
+    const int* len;             // [B] valid steps per row, or null (all T)
+};
+// *nlaunch (if given) = kernels launched: D when the directions run one after another.
+cudaError_t launch_tc_bwd(const TcBwdArgs& a, cudaStream_t s, int* nlaunch = nullptr);
+
+// out[d][u][4u'+q] = W_hh[d][q*H + u'][u] (bf16), the rows of W_hh^T in the
+// packed gate order of the tensor-core BPTT recurrence.
+struct PackWtArgs {
+    int H, D;
+    const void* w[2];           // W_hh of each direction, [4H][H] bf16
+    void* out;
+};
+cudaError_t launch_pack_wT(const PackWtArgs& a, cudaStream_t s);
+
 struct BwdRecArgs {
     int H, B, T, D;
     RecPlan p;

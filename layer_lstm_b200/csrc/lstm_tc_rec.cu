@@ -38,6 +38,7 @@
 #include "lstm_device.cuh"
 #include "lstm_internal.h"
 #include "lstm_tc.cuh"
+#include "lstm_tc_cluster.cuh"
 
 namespace lstm {
 namespace {
@@ -117,101 +118,6 @@ __device__ __forceinline__ float2 tanh2(float a, float b) {
 __device__ __forceinline__ float2 sigmoid2(float a, float b) {
     const float2 t = tanh2(0.5f * a, 0.5f * b);
     return make_float2(fmaf(0.5f, t.x, 0.5f), fmaf(0.5f, t.y, 0.5f));
-}
-
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-
-__device__ __forceinline__ void cluster_sync() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// Shared-memory address of the same offset in block `rank` of the cluster.
-__device__ __forceinline__ uint32_t map_rank(uint32_t saddr, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-    return r;
-}
-
-// Asynchronous 16-byte store into another block of the cluster; its bytes
-// count against the transaction count of that block's mbarrier remote_bar,
-// so the storing thread does not wait for it to land.
-__device__ __forceinline__ void st_async_v4(uint32_t addr, float a, float b, float c, float d, uint32_t remote_bar) {
-    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
-                 ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d), "r"(remote_bar)
-                 : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(tc::smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// Bounded wait for the partner's partial sums: gives up on this block's abort
-// flag, on an error anywhere in the grid, or after timeout_ns.
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort, int* status,
-                                                  uint64_t timeout_ns) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    uint32_t it = 0;
-    while (!mbar_try_wait_cluster(bar, parity)) {
-        if ((++it & 255u) == 0) {
-            if (*abort || ld_volatile(status) != kStatusOk) {
-                *abort = 1;
-                return false;
-            }
-            if (globaltimer_ns() - t0 > timeout_ns) {
-                atomicCAS(status, kStatusOk, kStatusTimeout);
-                *abort = 1;
-                return false;
-            }
-        }
-    }
-    return true;
-}
-
-// Bounded wait until *ctr >= target (single thread).
-__device__ __forceinline__ bool ctr_wait(const unsigned* ctr, unsigned target, volatile int* abort, int* status,
-                                         uint64_t timeout_ns) {
-    if (ld_acquire(ctr) >= target) return true;
-    const uint64_t t0 = globaltimer_ns();
-    unsigned it = 0;
-    while (ld_acquire(ctr) < target) {
-        if ((++it & 63u) == 0) {
-            if (*abort || ld_volatile(status) != kStatusOk) {
-                *abort = 1;
-                return false;
-            }
-            if (globaltimer_ns() - t0 > timeout_ns) {
-                atomicCAS(status, kStatusOk, kStatusTimeout);
-                *abort = 1;
-                return false;
-            }
-        }
-    }
-    return true;
-}
-
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
-    const uint64_t t0 = globaltimer_ns();
-    while (!tc::mbar_try_wait(bar, parity)) {
-        if (globaltimer_ns() - t0 > 100000000ull) break;
-    }
-}
-
-__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
-                 : "memory");
 }
 
 // Accumulator initialisation for one step: Gx[t] of packed row `prow` in the
@@ -777,6 +683,8 @@ bool make_map_bf16(CUtensorMap* map, const void* base, long long rows, long long
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+}  // namespace
+
 // h_{t-1} as a 3-D tensor (k within a 64-wide chunk, row, chunk): a box of
 // {64, rows, chunks} lands the chunks one after another, each a 128-byte-
 // swizzled [rows][64] tile, as the 2-D boxes of single chunks would.
@@ -796,8 +704,6 @@ bool make_map_bf16_chunks(CUtensorMap* map, const void* base, long long rows, lo
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-
-}  // namespace
 
 cudaError_t launch_tc_rec(const TcRecArgs& a, cudaStream_t s) {
     const TcRecPlan& p = a.p;
