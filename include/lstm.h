@@ -141,11 +141,16 @@ lstm_status lstm_forward(const lstm_desc* desc, const void* x, const void* h0, c
  *   dw_ih, dw_hh, db_ih, db_hh: host arrays of L*D device pointers to float32
  *     gradients, OVERWRITTEN (not accumulated); db arrays ignored if !bias.
  *     db_ih and db_hh receive the same values (the biases enter as a sum).
- * Both dtypes compute in float32.  For LSTM_BF16, x, h0, weights, grad_out,
- * grad_hn and the saved layer outputs are widened to float32 copies in the
- * workspace, and dx and dh0 are rounded to bf16 (nearest even) at the end;
- * the weight and bias gradients stay float32.  LSTM_ERR_UNSUPPORTED only
- * when no recurrent plan fits the device.
+ * LSTM_F32 computes in float32 (3xTF32 tensor-core products in the weight
+ * phase).  LSTM_BF16 keeps the cell arithmetic, the dc carry and every sum in
+ * float32, with bf16 products on the tensor cores: the recurrent products
+ * W_hh^T da take the previous step's gate gradients rounded to bf16, and the
+ * weight phase takes the gate gradients rounded to bf16 (x, the saved layer
+ * outputs and W_ih are exact in bf16); dx and dh0 are rounded to bf16
+ * (nearest even) at the end, the weight and bias gradients stay float32.
+ * (Shapes outside the tensor-core plans, or LSTM_B200_REC=simt, run the
+ * recurrence on the CUDA cores in float32.)  LSTM_ERR_UNSUPPORTED only when
+ * no recurrent plan fits the device.
  */
 lstm_status lstm_backward(const lstm_desc* desc, const void* x, const void* h0, const float* c0,
                           const void* const* w_ih, const void* const* w_hh,
@@ -240,8 +245,9 @@ const char* lstm_status_string(lstm_status status);
  * it returns the number of records written (the number of kinds when out is
  * NULL), or -1 if an event could not be read.  Kinds (the suffix names the
  * engine: _tc tensor cores, _ffma / _simt CUDA cores): pack, proj_gemm_tc,
- * proj_gemm_simt, fwd_rec_tc, fwd_rec_ffma, bwd_rec_ffma, dw_gemm_tc,
- * dw_gemm_simt, dx_gemm_tc, dx_gemm_simt, db_reduce, seq_copy, transpose.
+ * proj_gemm_simt, fwd_rec_tc, fwd_rec_ffma, bwd_rec_tc, bwd_rec_ffma,
+ * dw_gemm_tc, dw_gemm_simt, dx_gemm_tc, dx_gemm_simt, db_reduce, seq_copy,
+ * transpose, dropout.
  * lstm_timing_reset
  * zeroes the totals.  Process-wide and thread-safe; event recording adds a
  * few microseconds per launch, so leave it off outside measurements.
