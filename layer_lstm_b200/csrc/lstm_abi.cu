@@ -940,10 +940,28 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
     }
     int* status = reinterpret_cast<int*>(P(workspace, l.status));
     float* dG = reinterpret_cast<float*>(P(workspace, l.dG));
-    // Everything below computes in float32.  A bf16 problem reads float32
-    // copies of its bf16 inputs (x, h0, weights, grad_out, grad_hn and the
-    // saved layer outputs) and writes dx and dh0 through float32 staging.
+    // Cell arithmetic, states and sums are float32.  A bf16 problem on the
+    // tensor cores end to end (bfd) has the BPTT kernel store dG in bf16 and
+    // the weight phase read its bf16 operands where they are (x, h0, W_ih,
+    // the saved sequences); otherwise it reads float32 copies of its bf16
+    // inputs.  grad_out and grad_hn enter the recurrence as float32 copies,
+    // dx and dh0 leave through float32 staging.
     const bool bf = l.dt == DType::BF16;
+    const long long BTl0 = (long long)B * T;
+    // the tensor-core weight phase of layer k with operands of type wdt
+    auto weight_phase_tc = [&](int k, DType wdt) {
+        const int in = in_size(l, k);
+        TcGemmArgs tw{};
+        tw.M = G; tw.N = in + H; tw.K = (int)BTl0; tw.dt = wdt;
+        tw.A = P(workspace, l.dGT); tw.lda = BTl0; tw.B = P(workspace, l.bop); tw.ldb = BTl0;
+        TcGemmArgs tx{};
+        tx.M = (int)BTl0; tx.N = in; tx.K = D * G; tx.dt = wdt;
+        tx.A = dG; tx.lda = (long long)D * G; tx.B = P(workspace, l.wcatT); tx.ldb = (long long)D * G;
+        return tc_gemm_enabled() && tc_gemm_supported(tw) && tc_gemm_supported(tx) &&
+               (reinterpret_cast<uintptr_t>(dw_ih[k * D]) & 3) == 0;
+    };
+    bool bfd = bf && l.tcb.ok && tc_rec_enabled();
+    for (int k = 0; k < L && bfd; ++k) bfd = weight_phase_tc(k, DType::BF16);
     auto stage = [&](const void* src, size_t off, size_t n) -> const float* {
         if (!src) return nullptr;
         if (!bf) return static_cast<const float*>(src);
@@ -952,13 +970,13 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
         return e == cudaSuccess ? dst : nullptr;
     };
     const size_t BTs = (size_t)B * T;
-    const float* xf = stage(x, l.s_x, BTs * l.I);
-    const float* h0f = stage(h0, l.s_h0, (size_t)L * state);
+    const float* xf = bfd ? nullptr : stage(x, l.s_x, BTs * l.I);
+    const float* h0f = bfd ? nullptr : stage(h0, l.s_h0, (size_t)L * state);
     const float* goutf = stage(grad_out, l.s_gout, BTs * D * H);
     const float* ghnf = stage(grad_hn, l.s_ghn, (size_t)L * state);
-    if (!xf || !goutf || (h0 && !h0f) || (grad_hn && !ghnf)) return LSTM_ERR_CUDA;
+    if ((!bfd && !xf) || !goutf || (h0 && !bfd && !h0f) || (grad_hn && !ghnf)) return LSTM_ERR_CUDA;
     std::vector<const float*> wihf(L * D);   // W_hh stays in its own type (resident rows)
-    for (int k = 0; k < L; ++k)
+    for (int k = 0; k < L && !bfd; ++k)
         for (int d = 0; d < D; ++d) {
             const int i = k * D + d;
             const size_t nih = (size_t)G * in_size(l, k);
@@ -979,7 +997,7 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
     float* dxf = bf ? reinterpret_cast<float*>(P(workspace, l.s_dx)) : static_cast<float*>(dx);
     // time-major copy of x for the layer-0 weight gradient
     const float* x_tm = xf;
-    if (desc->batch_first) {
+    if (desc->batch_first && !bfd) {
         SeqCopyArgs sc{};
         sc.T = T; sc.B = B; sc.W = l.I; sc.dt = DType::F32;
         sc.src = xf; sc.s_st = l.I; sc.s_sb = (long long)T * l.I;
@@ -1040,6 +1058,7 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
             tb.dy = b.dy; tb.dy_st = b.dy_st; tb.dy_sb = b.dy_sb;
             tb.grad_hn = b.grad_hn; tb.grad_cn = b.grad_cn;
             tb.dG = dG;
+            tb.dG_bf16 = bfd;
             tb.dax = P(workspace, l.dax);
             tb.dh0 = b.dh0; tb.dc0 = b.dc0; tb.dbpart = b.dbpart;
             tb.ctr = reinterpret_cast<unsigned*>(P(workspace, l.ctr_tcb)) + (size_t)k * D * l.tcb.nbg * 32;
@@ -1058,9 +1077,23 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
             for (int d = 0; d < D; ++d) { db.db_ih[d] = db_ih[k * D + d]; db.db_hh[d] = db_hh[k * D + d]; }
             LSTM_CUDA(timed(K_DB, stream, [&] { return launch_db_reduce(db, stream); }));
         }
-        const float* layer_in = k == 0 ? x_tm : saved_seq(dropped ? l.hdrop[k - 1] : l.hseq[k - 1], 1);
-        const float* hs = saved_seq(l.hseq[k], 0);
-        if (!layer_in || !hs) return LSTM_ERR_CUDA;
+        // the layer's input and output sequences: bf16 where they are (bfd),
+        // else float32 (copies)
+        const float* layer_in = nullptr;
+        const float* hs = nullptr;
+        const void* lin_v;
+        const void* hs_v;
+        if (bfd) {
+            lin_v = k == 0 ? x : static_cast<const char*>(reserve) + (dropped ? l.hdrop[k - 1] : l.hseq[k - 1]);
+            hs_v = static_cast<const char*>(reserve) + l.hseq[k];
+        } else {
+            layer_in = k == 0 ? x_tm : saved_seq(dropped ? l.hdrop[k - 1] : l.hseq[k - 1], 1);
+            hs = saved_seq(l.hseq[k], 0);
+            if (!layer_in || !hs) return LSTM_ERR_CUDA;
+            lin_v = k == 0 ? static_cast<const void*>(xf) : static_cast<const void*>(layer_in);
+            hs_v = hs;
+        }
+        const size_t ses = bfd ? 2 : 4;   // element size of those sources
         const long long ldg = (long long)D * G, ldh = (long long)D * H;
         const long long BTl = (long long)B * T;
         float* din = k == 0 ? dxf : reinterpret_cast<float*>(P(workspace, l.dseq[cur]));
@@ -1085,36 +1118,37 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
         tw.ws_floats = (long long)l.gemm_ws_floats;
         TcGemmArgs tx{};
         tx.M = (int)BTl; tx.N = in; tx.K = D * G; tx.dt = wdt;
-        // bf16: a bf16 copy of dG, written into dGT's space once the dW GEMMs are done
-        tx.A = wbf ? static_cast<const void*>(dGT) : static_cast<const void*>(dG);
+        // bf16: dG itself (bfd) or a bf16 copy of it, written into dGT's space
+        // once the dW GEMMs are done
+        tx.A = (wbf && !bfd) ? static_cast<const void*>(dGT) : static_cast<const void*>(dG);
         tx.lda = ldg; tx.B = wcatT; tx.ldb = (long long)D * G;
         tx.C = din; tx.ldc = in;
         if (k == 0 && desc->batch_first) { tx.remap_T = -T; tx.remap_B = B; }
         tx.status = status; tx.timeout_ns = timeout_ns(); tx.num_sms = device_info().sms;
-        const bool tc_ok = tc_gemm_enabled() && tc_gemm_supported(tw) && tc_gemm_supported(tx) &&
-                           (reinterpret_cast<uintptr_t>(dw_ih[k * D]) & 3) == 0;
+        const bool tc_ok = weight_phase_tc(k, wdt);
         if (tc_ok) {
             TransposeArgs ta{};
-            ta.M = (int)BTl; ta.C = D * G; ta.mode = 0; ta.src = dG; ta.lds = ldg;
+            ta.M = (int)BTl; ta.C = D * G; ta.mode = 0; ta.src = dG; ta.lds = ldg; ta.src_bf16 = bfd;
             ta.dst = dGT; ta.ldd = BTl; ta.dst_bf16 = wbf;
             LSTM_CUDA(timed(K_TRANSPOSE, stream, [&] { return launch_transpose(ta, stream); }));
             for (int d = 0; d < D; ++d) {
                 char* bo = bop + (size_t)d * (in + H) * BTl * wes;
                 TransposeArgs ti{};
                 ti.M = (int)BTl; ti.C = in; ti.mode = 0;
+                ti.src = lin_v; ti.lds = in; ti.src_bf16 = bfd;
                 if (k == 0) {
-                    ti.src = xf; ti.lds = in;
                     ti.bt_remap = desc->batch_first; ti.T = T; ti.B = B;
-                } else {
-                    ti.src = layer_in;
-                    ti.lds = in;
                 }
                 ti.dst = bo; ti.ldd = BTl; ti.dst_bf16 = wbf;
                 LSTM_CUDA(timed(K_TRANSPOSE, stream, [&] { return launch_transpose(ti, stream); }));
                 TransposeArgs th{};
                 th.M = (int)BTl; th.C = H; th.mode = 1;
-                th.src = hs + (size_t)d * H; th.lds = ldh; th.T = T; th.B = B; th.dir = d;
-                th.h0 = h0f ? h0f + ((size_t)k * D + d) * B * H : nullptr;
+                th.src = static_cast<const char*>(hs_v) + (size_t)d * H * ses;
+                th.lds = ldh; th.T = T; th.B = B; th.dir = d; th.src_bf16 = bfd;
+                if (bfd)
+                    th.h0 = h0 ? static_cast<const char*>(h0) + ((size_t)k * D + d) * B * H * 2 : nullptr;
+                else
+                    th.h0 = h0f ? h0f + ((size_t)k * D + d) * B * H : nullptr;
                 th.dst = bo + (size_t)in * BTl * wes; th.ldd = BTl; th.dst_bf16 = wbf;
                 LSTM_CUDA(timed(K_TRANSPOSE, stream, [&] { return launch_transpose(th, stream); }));
                 TcGemmArgs twd = tw;
@@ -1128,11 +1162,12 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
                 }
                 TransposeArgs tww{};
                 tww.M = G; tww.C = in; tww.mode = 0;
-                tww.src = wihf[k * D + d]; tww.lds = in;
+                tww.src = bfd ? w_ih[k * D + d] : static_cast<const void*>(wihf[k * D + d]);
+                tww.lds = in; tww.src_bf16 = bfd;
                 tww.dst = wcatT + (size_t)d * G * wes; tww.ldd = (long long)D * G; tww.dst_bf16 = wbf;
                 LSTM_CUDA(timed(K_TRANSPOSE, stream, [&] { return launch_transpose(tww, stream); }));
             }
-            if (wbf)
+            if (wbf && !bfd)
                 LSTM_CUDA(timed(K_TRANSPOSE, stream, [&] {
                     return launch_convert(dG, DType::F32, dGT, DType::BF16, BTl * ldg, stream);
                 }));

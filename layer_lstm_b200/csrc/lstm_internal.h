@@ -62,8 +62,9 @@ bool tc_gemm_supported(const TcGemmArgs& g);
 // *nlaunch (if given) = kernels launched: 2 when K was split (GEMM + reduction).
 cudaError_t launch_tc_gemm(const TcGemmArgs& g, cudaStream_t s, int* nlaunch = nullptr);
 
-// dst[c*ldd + m] = src(m, c) for m < M, c < C (float32 source; float32
-// destination, or bf16 rounded to nearest even when dst_bf16).
+// dst[c*ldd + m] = src(m, c) for m < M, c < C.  src and h0 are float32, or
+// bf16 when src_bf16; dst is float32, or bf16 rounded to nearest even when
+// dst_bf16.
 //  mode 0: src(m, c) = src[row(m)*lds + c], row(m) = m, or with bt_remap the
 //          time-major index m = t*B + b read from a batch-first (b*T + t) array.
 //  mode 1: h_{t-1} of one direction in its own time order: for m = t*B + b,
@@ -71,11 +72,11 @@ cudaError_t launch_tc_gemm(const TcGemmArgs& g, cudaStream_t s, int* nlaunch = n
 //          (dir 1) when 0 <= ts < T, else h0[b*C + c] (zero if h0 is null).
 struct TransposeArgs {
     int M, C, mode;
-    const float* src; long long lds;
+    const void* src; long long lds;
     int bt_remap, T, B, dir;
-    const float* h0;
+    const void* h0;
     void* dst; long long ldd;
-    int dst_bf16;
+    int dst_bf16, src_bf16;
 };
 cudaError_t launch_transpose(const TransposeArgs& a, cudaStream_t s);
 
@@ -192,7 +193,8 @@ struct TcBwdArgs {
     const float* dy; long long dy_st, dy_sb;   // dL/dh_t of this layer's output, element (t, b, d*H + u)
     const float* grad_hn;       // [D][B][H] or null
     const float* grad_cn;       // [D][B][H] or null
-    float* dG;                  // [T][B][D*4H] gate gradients, standard row order q*H + u
+    void* dG;                   // [T][B][D*4H] gate gradients, standard row order q*H + u
+    int dG_bf16;                // dG in bf16 (rounded to nearest even) rather than float32
     void* dax;                  // [D][T+1][B][4H] bf16 exchange of the gate gradients (order 4u+q)
     float* dh0; float* dc0;     // [D][B][H]
     float* dbpart;              // [D][nbg][4H] bias-gradient partial of each batch group

@@ -21,7 +21,7 @@
 // sums to the block that owns the unit (16 units per block; asynchronous
 // distributed-shared-memory stores completing on the owner's mbarrier).  The
 // owner adds the 8 partials, computes the gate gradients of its 16 units,
-// stores them (float32, for the weight phase) and publishes them in bf16 for
+// stores them (for the weight phase, float32 or bf16) and publishes them in bf16 for
 // the next step; the blocks of a (direction, batch group) meet on a counter,
 // as in the tensor-core forward.  Roles: warp 0 TMA, warp 1 MMA (both whole
 // warps, elect.sync for issue), warps 2-9 partial sums and gate gradients.
@@ -60,7 +60,8 @@ struct TcBwdParams {
     const float* dy; long long dy_st, dy_sb;
     const float* grad_hn;
     const float* grad_cn;
-    float* dG;
+    void* dG;
+    int dG_bf16;
     bf16* dax;
     float* dh0; float* dc0;
     float* dbpart;
@@ -352,11 +353,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int g = 0; g < 4; ++g) dbs[g] += da[g];
                 }
-                float* dgp = a.dG + ((size_t)t * B + bb) * ldg + (size_t)d * G + u;
-                dgp[0] = da[0];
-                dgp[H] = da[1];
-                dgp[2 * H] = da[2];
-                dgp[3 * H] = da[3];
+                const size_t gi = ((size_t)t * B + bb) * ldg + (size_t)d * G + u;
+                if (a.dG_bf16) {
+                    bf16* dgp = static_cast<bf16*>(a.dG) + gi;
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) dgp[(size_t)g * H] = __float2bfloat16_rn(da[g]);
+                } else {
+                    float* dgp = static_cast<float*>(a.dG) + gi;
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) dgp[(size_t)g * H] = da[g];
+                }
                 const __nv_bfloat162 p01 = __floats2bfloat162_rn(da[0], da[1]);
                 const __nv_bfloat162 p23 = __floats2bfloat162_rn(da[2], da[3]);
                 uint2 pk;
@@ -441,7 +447,7 @@ cudaError_t launch_tc_bwd(const TcBwdArgs& a, cudaStream_t s, int* nlaunch) {
     prm.act = a.act; prm.cst = a.cst; prm.c0 = a.c0;
     prm.dy = a.dy; prm.dy_st = a.dy_st; prm.dy_sb = a.dy_sb;
     prm.grad_hn = a.grad_hn; prm.grad_cn = a.grad_cn;
-    prm.dG = a.dG; prm.dax = static_cast<bf16*>(a.dax);
+    prm.dG = a.dG; prm.dG_bf16 = a.dG_bf16; prm.dax = static_cast<bf16*>(a.dax);
     prm.dh0 = a.dh0; prm.dc0 = a.dc0; prm.dbpart = a.dbpart;
     prm.ctr = a.ctr; prm.status = a.status; prm.timeout_ns = a.timeout_ns;
     prm.len = a.len;

@@ -471,6 +471,10 @@ cudaError_t launch_tc_gemm(const TcGemmArgs& g, cudaStream_t s, int* nlaunch) {
 // ---------------------------------------------------------------- transposes
 namespace {
 
+__device__ __forceinline__ float ld_elem(const void* p, long long i, int bf) {
+    return bf ? __bfloat162float(static_cast<const bf16*>(p)[i]) : static_cast<const float*>(p)[i];
+}
+
 __global__ void transpose_kernel(TransposeArgs a) {
     __shared__ float tile[32][33];
     const int m0 = blockIdx.x * 32, c0 = blockIdx.y * 32;
@@ -482,12 +486,12 @@ __global__ void transpose_kernel(TransposeArgs a) {
             if (a.mode == 0) {
                 long long row = m;
                 if (a.bt_remap) row = (long long)(m % a.B) * a.T + m / a.B;   // m = t*B + b -> b*T + t
-                v = a.src[row * a.lds + c];
+                v = ld_elem(a.src, row * a.lds + c, a.src_bf16);
             } else {
                 const int t = m / a.B, b = m % a.B;
                 const int ts = a.dir == 0 ? t - 1 : t + 1;
-                if (ts >= 0 && ts < a.T) v = a.src[((long long)ts * a.B + b) * a.lds + c];
-                else if (a.h0) v = a.h0[(long long)b * a.C + c];
+                if (ts >= 0 && ts < a.T) v = ld_elem(a.src, ((long long)ts * a.B + b) * a.lds + c, a.src_bf16);
+                else if (a.h0) v = ld_elem(a.h0, (long long)b * a.C + c, a.src_bf16);
             }
         }
         tile[i][tx] = v;
