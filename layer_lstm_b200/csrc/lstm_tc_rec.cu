@@ -176,6 +176,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int H = a.H, B = a.B, T = a.T, D = a.D, G = 4 * H;
     const int S = a.stages, N = a.N, NH = N / 2;
     const int hstage = N * 128;
+    // epilogue column chunks: 8 wide for the small groups of whole-box plans
+    // (both halves of the epilogue warps busy at N = 32), else 16
+    constexpr int kCW = kWhole ? 8 : 16;
+    constexpr int kQW = kCW / 4;   // columns per lane after the gate exchange
     const uint32_t rank = cluster_rank();
     const int KT = H / 64;
     const int c_beg = (int)rank * a.KH, c_end = min(KT, c_beg + a.KH);
@@ -417,7 +421,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int e = threadIdx.x - 64;             // epilogue thread index
         const int gq = lane & 3;                    // gate of this lane's row
         const int u = j * 32 + q * 8 + (lane >> 2); // unit of this lane's row group
-        const int ncc = NH / 16;                    // own 16-column chunks
+        const int ncc = NH / kCW;                   // own column chunks
+        const int ncc16 = NH / 16;                  // own 16-column chunks (the Gx preload's unit)
         const uint32_t partner = rank ^ 1u;
         const uint32_t recv_remote = map_rank(tc::smem_u32(recv), partner);
         const uint32_t recv_bar_remote = map_rank(tc::smem_u32(recv_full), partner);
@@ -429,10 +434,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int cc = half + 2 * k;
-                const int col = own0 + 16 * cc + 4 * gq + i;
-                creg[k][i] = (cc < ncc && col < nB && a.c0) ? a.c0[((size_t)d * B + b0 + col) * H + u] : 0.f;
+                const int col = own0 + kCW * cc + kQW * gq + i;
+                creg[k][i] = (i < kQW && cc < ncc && col < nB && a.c0) ? a.c0[((size_t)d * B + b0 + col) * H + u]
+                                                                       : 0.f;
             }
-        preload_gx(a.gx, d == 0 ? 0 : T - 1, B, ldgx, prow0 + r, b0, own0, pcol0, ncc, nB, half, trow, d_ready);
+        preload_gx(a.gx, d == 0 ? 0 : T - 1, B, ldgx, prow0 + r, b0, own0, pcol0, ncc16, nB, half, trow, d_ready);
         for (int s = 0; s < T; ++s) {
             const int t = d == 0 ? s : T - 1 - s;
             // this step's phase of recv_full completes when the partner's
@@ -449,15 +455,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::tc_fence_after();
             trace_mark(a.trace, tr2, s, 4);
             // 1) this block's partial sums of the partner's columns -> partner,
-            //    two 16-column chunks at a time
+            //    two column chunks at a time (recv holds column quads)
 #pragma unroll
             for (int k0 = 0; k0 < kCcPerHalf; k0 += 2) {
                 if (half + 2 * k0 >= ncc) break;
-                float pv[2][16];
+                float pv[2][kCW];
 #pragma unroll
                 for (int kk = 0; kk < 2; ++kk) {
                     const int cc = half + 2 * (k0 + kk);
-                    if (cc < ncc) tc::tmem_ld16(trow + (uint32_t)(pcol0 + 16 * cc), pv[kk]);
+                    if (cc < ncc) tc::tmem_ldw<kCW>(trow + (uint32_t)(pcol0 + kCW * cc), pv[kk]);
                 }
                 tc::tmem_ld_wait();
 #pragma unroll
@@ -465,8 +471,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int cc = half + 2 * (k0 + kk);
                     if (cc >= ncc) break;
 #pragma unroll
-                    for (int m = 0; m < 4; ++m)
-                        st_async_v4(recv_remote + (uint32_t)(((4 * cc + m) * kRows + r) * 16), pv[kk][4 * m],
+                    for (int m = 0; m < kCW / 4; ++m)
+                        st_async_v4(recv_remote + (uint32_t)((((kCW / 4) * cc + m) * kRows + r) * 16), pv[kk][4 * m],
                                     pv[kk][4 * m + 1], pv[kk][4 * m + 2], pv[kk][4 * m + 3], recv_bar_remote);
                 }
             }
@@ -479,11 +485,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int k0 = 0; k0 < kCcPerHalf; k0 += 2) {
                 if (half + 2 * k0 >= ncc) break;
-                float ov[2][16];
+                float ov[2][kCW];
 #pragma unroll
                 for (int kk = 0; kk < 2; ++kk) {
                     const int cc = half + 2 * (k0 + kk);
-                    if (cc < ncc) tc::tmem_ld16(trow + (uint32_t)(own0 + 16 * cc), ov[kk]);
+                    if (cc < ncc) tc::tmem_ldw<kCW>(trow + (uint32_t)(own0 + kCW * cc), ov[kk]);
                 }
                 tc::tmem_ld_wait();
 #pragma unroll
@@ -493,22 +499,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (cc >= ncc) break;
                     float* v = ov[kk];
 #pragma unroll
-                    for (int m = 0; m < 4; ++m) {
-                        const float4 p4 = recv[(4 * cc + m) * kRows + r];
+                    for (int m = 0; m < kCW / 4; ++m) {
+                        const float4 p4 = recv[((kCW / 4) * cc + m) * kRows + r];
                         v[4 * m] += p4.x; v[4 * m + 1] += p4.y; v[4 * m + 2] += p4.z; v[4 * m + 3] += p4.w;
                     }
-                    // v[4m + i]: gate gq at column 16cc + 4m + i.  Three xor
-                    // exchanges inside each 4-lane group give lane gq all four
-                    // gates at column 16cc + 4gq + i (gate X arrives in round gq ^ X).
-                    float gi[4], gf[4], gc[4], go[4];
+                    // v[kQW m + i]: gate gq at column kCW cc + kQW m + i.  Three
+                    // xor exchanges inside each 4-lane group give lane gq all
+                    // four gates at column kCW cc + kQW gq + i (gate X arrives in
+                    // round gq ^ X).
+                    float gi[kQW], gf[kQW], gc[kQW], go[kQW];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
+                    for (int i = 0; i < kQW; ++i) {
                         float rcv[4];
-                        rcv[0] = sel4(v[i], v[4 + i], v[8 + i], v[12 + i], gq);
+                        rcv[0] = sel4(v[i], v[kQW + i], v[2 * kQW + i], v[3 * kQW + i], gq);
 #pragma unroll
                         for (int rr = 1; rr < 4; ++rr)
-                            rcv[rr] =
-                                __shfl_xor_sync(0xffffffffu, sel4(v[i], v[4 + i], v[8 + i], v[12 + i], gq ^ rr), rr);
+                            rcv[rr] = __shfl_xor_sync(
+                                0xffffffffu, sel4(v[i], v[kQW + i], v[2 * kQW + i], v[3 * kQW + i], gq ^ rr), rr);
                         gi[i] = sel4(rcv[0], rcv[1], rcv[2], rcv[3], gq ^ 0);
                         gf[i] = sel4(rcv[0], rcv[1], rcv[2], rcv[3], gq ^ 1);
                         gc[i] = sel4(rcv[0], rcv[1], rcv[2], rcv[3], gq ^ 2);
@@ -517,7 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // the cells of two columns at a time: every nonlinearity
                     // is one f16x2 tanh for both
 #pragma unroll
-                    for (int i = 0; i < 4; i += 2) {
+                    for (int i = 0; i < kQW; i += 2) {
                         const float2 ig = sigmoid2(gi[i], gi[i + 1]), fg = sigmoid2(gf[i], gf[i + 1]);
                         const float2 og = sigmoid2(go[i], go[i + 1]), gg = tanh2(gc[i], gc[i + 1]);
                         const float cn0 = fg.x * creg[k][i] + ig.x * gg.x;
@@ -527,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float cn[2] = {cn0, cn1};
 #pragma unroll
                         for (int e = 0; e < 2; ++e) {
-                            const int lc = 16 * cc + 4 * gq + i + e;   // column within the own half
+                            const int lc = kCW * cc + kQW * gq + i + e;   // column within the own half
                             const int col = own0 + lc;
                             if (col >= nB) continue;
                             const int bb = b0 + col;
@@ -550,10 +557,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                                           : make_float4(0.f, 0.f, 0.f, 0.f);
                                 a.cst[row * H + u] = c;
                             }
-                            // unit octet q of column lc, stored at octet q ^ gq
-                            // ((lc >> 2) & 3 == gq): the four columns of a warp's
-                            // store fall in different banks
-                            sh[lc * 32 + 8 * (q ^ gq) + (lane >> 2)] = hv;
+                            // unit octet q of column lc, stored at octet
+                            // q ^ ((lc >> 2) & 3) (= gq with 16-column chunks):
+                            // the columns of a warp's store fall in different banks
+                            sh[lc * 32 + 8 * (q ^ ((lc >> 2) & 3)) + (lane >> 2)] = hv;
                             if (s == T - 1) {
                                 const int b = b0 + col;
                                 a.h_n[((size_t)d * B + b) * H + u] = hv;
@@ -585,7 +592,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             trace_mark(a.trace, tr2, s, 8);
             if (s + 1 < T) {
-                preload_gx(a.gx, d == 0 ? s + 1 : T - 2 - s, B, ldgx, prow0 + r, b0, own0, pcol0, ncc, nB, half, trow,
+                preload_gx(a.gx, d == 0 ? s + 1 : T - 2 - s, B, ldgx, prow0 + r, b0, own0, pcol0, ncc16, nB, half, trow,
                            d_ready);
                 trace_mark(a.trace, tr2, s + 1, 10);
             }
