@@ -123,6 +123,15 @@ size_t lstm_reserve_size(const lstm_desc* desc);
  * Enqueued on `stream`; returns before the GPU finishes.  Only
  * stream-ordered work is enqueued (no host synchronisation), so a call may be
  * captured into a CUDA graph and replayed.
+ * LSTM_F32 runs the input projection, and where a tensor-core plan fits (H a
+ * multiple of 128 from 256 to 1024, batch groups of at most 64 rows) the
+ * recurrent product W_hh h_{t-1} too, as 3xTF32: each operand is split into
+ * its tf32 part and the float32 remainder and the three larger cross
+ * products are summed in float32 (the remainder-by-remainder term, relative
+ * size 2^-22, is dropped); gates and cell update in float32.  LSTM_BF16
+ * multiplies bf16 operands on the tensor cores with float32 sums and cell
+ * arithmetic; h_t is rounded to bf16 where it is stored.  (Other shapes, or
+ * LSTM_B200_REC=simt, run the recurrence on the CUDA cores in float32.)
  */
 lstm_status lstm_forward(const lstm_desc* desc, const void* x, const void* h0, const float* c0,
                          const void* const* w_ih, const void* const* w_hh,
@@ -286,11 +295,20 @@ void lstm_timing_reset(void);
  *     to the partner block, 6 partner's partial sums received, 7 cell update
  *     done, 8 h_t published, 10 Gx of this step loaded into the accumulator
  *     (stamped at the end of the previous step).
+ *   LSTM_TRACE_FWD_REC_TC32: 0 producer passed the group wait, 9 h tiles
+ *     landed (first issuer), 3 its MMAs committed, 4 epilogue saw all MMAs
+ *     complete, 5 partial sums sent to the column owners, 6 the owners'
+ *     partial sums received, 7 cell update done, 8 h_t published.
  * Process-wide; tracing adds one timer read and store per event to block 0.
  */
 #define LSTM_TRACE_MAX_STEPS 512
 #define LSTM_TRACE_EVENTS 16
-enum { LSTM_TRACE_FWD_REC_FFMA = 1, LSTM_TRACE_BWD_REC_FFMA = 2, LSTM_TRACE_FWD_REC_TC = 3 };
+enum {
+    LSTM_TRACE_FWD_REC_FFMA = 1,
+    LSTM_TRACE_BWD_REC_FFMA = 2,
+    LSTM_TRACE_FWD_REC_TC = 3,
+    LSTM_TRACE_FWD_REC_TC32 = 4
+};
 
 lstm_status lstm_trace_enable(int enable);
 int lstm_trace_read(unsigned long long* out, int max_steps, int* kind);

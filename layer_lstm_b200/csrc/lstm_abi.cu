@@ -238,6 +238,8 @@ struct Layout {
     // workspace offsets
     TcBwdPlan tcb;     // tensor-core BPTT recurrence (bf16), if it fits
     size_t ctr_tcb, dax, wT_tcb;
+    TcRec32Plan tc32;  // tensor-core forward recurrence for float32 (3xTF32), if it fits
+    size_t ctr_tc32, hx32;
     size_t status, ctr_f, ctr_b, ctr_tc, ctr_end, wih[32], bias[32], whh_f, whh_b, gx, hT, seq[2], dG, dseq[2], xt,
         dbpart, P, dGT, bop, wcatT, hx, whh_tc, bias_dummy, gemm_ws, total;
     size_t gemm_ws_floats;
@@ -299,6 +301,7 @@ bool make_layout(const lstm_desc* d, Layout& l) {
     l.bwd_ok = l.bwd.ctas > 0;
     l.tcr = l.dt == DType::BF16 ? plan_tc_rec(l.H, Bp, l.D, dev.sms, smem_max) : TcRecPlan{};
     l.tcb = l.dt == DType::BF16 ? plan_tc_bwd(l.H, Bp, l.D, dev.sms, smem_max) : TcBwdPlan{};
+    l.tc32 = l.dt == DType::F32 ? plan_tc_rec32(l.H, Bp, l.D, dev.sms, smem_max) : TcRec32Plan{};
     const size_t TB = (size_t)l.T * l.B;
     size_t o = 0;
     l.status = o; o += al(sizeof(int));
@@ -309,6 +312,7 @@ bool make_layout(const lstm_desc* d, Layout& l) {
     // on its own 128-byte line
     l.ctr_tc = o; o += al(l.tcr.ok ? sizeof(unsigned) * 32 * (size_t)l.L * l.D * l.tcr.nbg : 0);
     l.ctr_tcb = o; o += al(l.tcb.ok ? sizeof(unsigned) * 32 * (size_t)l.L * l.D * l.tcb.nbg : 0);
+    l.ctr_tc32 = o; o += al(l.tc32.ok ? sizeof(unsigned) * 32 * (size_t)l.L * l.D * l.tc32.nbg : 0);
     l.ctr_end = o;
     for (int k = 0; k < l.L; ++k) {
         l.wih[k] = o; o += al((size_t)l.D * l.G * in_size(l, k) * l.es);
@@ -338,12 +342,13 @@ bool make_layout(const lstm_desc* d, Layout& l) {
         }
     }
     l.wf_end = o;
-    if (l.tcr.ok) {
-        l.hx = o; o += al((size_t)l.D * (l.T + 1) * l.B * l.H * 2);
-        l.whh_tc = o; o += al((size_t)l.D * l.G * l.H * 2);
+    l.hx = l.hx32 = l.whh_tc = l.bias_dummy = 0;
+    if (l.tcr.ok || l.tc32.ok) {
+        // exchange of h: bf16 [D][T+1][B][H], or float32 hi | lo [D][T+1][B][2H]
+        if (l.tcr.ok) { l.hx = o; o += al((size_t)l.D * (l.T + 1) * l.B * l.H * 2); }
+        if (l.tc32.ok) { l.hx32 = o; o += al((size_t)l.D * (l.T + 1) * l.B * 2 * l.H * 4); }
+        l.whh_tc = o; o += al((size_t)l.D * l.G * l.H * l.es);
         l.bias_dummy = o; o += al((size_t)l.D * l.G * 4);
-    } else {
-        l.hx = l.whh_tc = l.bias_dummy = 0;
     }
     // backward (float32 arithmetic for both dtypes)
     const size_t maxin = (size_t)(l.I > l.D * l.H ? l.I : l.D * l.H);
@@ -412,7 +417,7 @@ bool desc_is_valid(const lstm_desc* desc) { return valid_desc(desc); }
 size_t forward_workspace_prefix(const lstm_desc* desc) {
     Layout l;
     if (!make_layout(desc, l)) return 0;
-    if (l.tcr.ok) return l.bias_dummy + al((size_t)l.D * l.G * 4);
+    if (l.tcr.ok || l.tc32.ok) return l.bias_dummy + al((size_t)l.D * l.G * 4);
     return l.wf_end;
 }
 
@@ -643,7 +648,7 @@ lstm_status lstm_forward_varlen(const lstm_desc* desc, const int* lengths, const
         return timed(K_PROJ_SIMT, st, [&] { return launch_gemm(g, st); });
     };
 
-    const bool tc_path = l.tcr.ok && tc_rec_enabled();
+    const bool tc_path = (l.tcr.ok || l.tc32.ok) && tc_rec_enabled();
     if (l.wf && !lengths && !(reserve && l.dropout > 0.f) && !tc_path) {
         // ------------------------------------------------ layer wavefront
         // Layer k runs on stream k (the caller's stream for k = 0, a pool
@@ -777,6 +782,50 @@ lstm_status lstm_forward_varlen(const lstm_desc* desc, const int* lengths, const
         }
 
         void* hseq_tc = reserve ? P(reserve, l.hseq[k]) : P(workspace, l.seq[k & 1]);
+        if (tc_path && l.tc32.ok) {
+            // float32 tensor-core recurrence (3xTF32): packed W_hh rows in
+            // float32; the launcher fills exchange slot 0 from h0
+            PackIhArgs pw{};
+            pw.H = H; pw.in = H; pw.D = D; pw.dt = l.dt;
+            for (int d = 0; d < D; ++d) pw.w[d] = w_hh[k * D + d];
+            pw.wp = P(workspace, l.whh_tc);
+            pw.bias_p = reinterpret_cast<float*>(P(workspace, l.bias_dummy));
+            LSTM_CUDA(timed(K_PACK, stream, [&] { return launch_pack_ih(pw, stream); }));
+            TcRec32Args tr{};
+            tr.H = H; tr.B = B; tr.T = T; tr.D = D; tr.p = l.tc32;
+            tr.gx = reinterpret_cast<const float*>(P(workspace, l.gx));
+            tr.wpk = reinterpret_cast<const float*>(P(workspace, l.whh_tc));
+            tr.h0 = h0 ? static_cast<const float*>(h0) + (size_t)k * state_elems : nullptr;
+            tr.c0 = c0 ? c0 + (size_t)k * state_elems : nullptr;
+            tr.hx = reinterpret_cast<float*>(P(workspace, l.hx32));
+            tr.hseq = (k < L - 1 || reserve) ? static_cast<float*>(hseq_tc) : nullptr;
+            if (k == L - 1) {
+                tr.out = static_cast<float*>(out);
+                tr.out_st = desc->batch_first ? (long long)D * H : (long long)B * D * H;
+                tr.out_sb = desc->batch_first ? (long long)T * D * H : (long long)D * H;
+            }
+            tr.h_n = static_cast<float*>(h_n) + (size_t)k * state_elems;
+            tr.c_n = c_n + (size_t)k * state_elems;
+            if (reserve) {
+                tr.act = reinterpret_cast<float*>(P(reserve, l.act[k]));
+                tr.cst = reinterpret_cast<float*>(P(reserve, l.cst[k]));
+            }
+            tr.ctr = reinterpret_cast<unsigned*>(P(workspace, l.ctr_tc32)) + (size_t)k * D * l.tc32.nbg * 32;
+            tr.status = status;
+            tr.timeout_ns = timeout_ns();
+            tr.len = lengths;
+            tr.trace = trace_for(LSTM_TRACE_FWD_REC_TC32, T, stream);
+            int nl = 1;
+            LSTM_CUDA(timed(K_FWD_REC_TC, stream, [&] { return launch_tc_rec32(tr, stream, &nl); }, &nl));
+            layer_in = hseq_tc;
+            if (reserve && l.dropout > 0.f && k < L - 1) {
+                void* dropped = P(reserve, l.hdrop[k]);
+                const DropoutArgs da = dropout_args(desc, k, hseq_tc, dropped, l.dt, (long long)B * T * D * H);
+                LSTM_CUDA(timed(K_DROPOUT, stream, [&] { return launch_dropout(da, stream); }));
+                layer_in = dropped;
+            }
+            continue;
+        }
         if (tc_path) {
             // tensor-core recurrence: packed W_hh rows, h0 into exchange slot 0
             PackIhArgs pw{};

@@ -173,6 +173,38 @@ struct TcRecArgs {
 };
 cudaError_t launch_tc_rec(const TcRecArgs& a, cudaStream_t s);
 
+// Tensor-core forward recurrence for float32 (3xTF32: W_hh and h split into
+// tf32 hi and lo parts, products hi*hi + hi*lo + lo*hi, float32 sums).
+// Clusters of C = H/128 blocks per (direction, batch group, 128 packed gate
+// rows) split K = H; each block owns N/C of the group's N batch columns.
+struct TcRec32Plan {
+    bool ok;
+    int nbg, Bg, N, nsl, C, KP, ctas;   // nsl slices of 128 rows, K part KP = H / C
+    size_t smem;
+};
+TcRec32Plan plan_tc_rec32(int H, int B, int D, int num_sms, size_t smem_max);
+
+struct TcRec32Args {
+    int H, B, T, D;
+    TcRec32Plan p;
+    const float* gx;            // [T][B][D*4H] packed rows 4u+q, biases included
+    const float* wpk;           // [D*4H][H] W_hh packed rows 4u+q, float32
+    const float* h0;            // [D][B][H] or null
+    const float* c0;            // [D][B][H] or null
+    float* hx;                  // exchange [D][T+1][B][2H]: tf32 hi | remainder of h (slot 0 = h0)
+    float* hseq;                // [T][B][D*H] or null
+    float* out; long long out_st, out_sb;   // user output of the last layer, or null
+    float* h_n; float* c_n;     // [D][B][H]
+    float* act; float* cst;     // training: gate activations [D][T][B][4H] and cell states, or null
+    unsigned* ctr;              // [D][nbg] counters, 32 words apart, zeroed
+    int* status;
+    uint64_t timeout_ns;
+    const int* len;             // [B] valid steps per row, or null (all T)
+    unsigned long long* trace;  // [kTraceSteps][kTraceEvents] or null
+};
+// *nlaunch (if given) = kernels launched (the slot-0 fill included).
+cudaError_t launch_tc_rec32(const TcRec32Args& a, cudaStream_t s, int* nlaunch = nullptr);
+
 // Tensor-core BPTT recurrence (bf16 W_hh; float32 state and gate
 // gradients; the gate gradients of each step exchanged in bf16).  Clusters of
 // 8 blocks per (direction, batch group, 128-unit slice) split K = 4H.

@@ -170,6 +170,18 @@ __device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a_desc, uint6
         : "memory");
 }
 
+// kind::tf32 with the A operand in tensor memory (M rows on lanes, one tf32
+// per 32-bit column along K) and B in shared memory.
+__device__ __forceinline__ void mma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // One lane of a converged warp, chosen by elect.sync (the same lane each time
 // the full warp executes it); every lane of the warp must take part.  Issue
 // code of a whole-warp role: the warp waits on mbarriers together (a wait by

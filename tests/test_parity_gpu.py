@@ -104,6 +104,9 @@ SMALL = {
     "bf16_tc_split_wsmem": Workload("s", L=1, D=1, I=64, H=1088, T=3, B=480, dtype="bf16",
                                     state_std=0.3, seed=116),
     "H1": Workload("s", L=1, D=1, I=3, H=1, T=4, B=3, dtype="f32", state_std=0.5, seed=108),
+    # float32 tensor-core recurrence (3xTF32, clusters of H/128 = 2 blocks),
+    # bidirectional, one group of 40 of 64 columns
+    "f32_tc_bi": Workload("s", L=2, D=2, I=48, H=256, T=7, B=40, dtype="f32", state_std=0.3, seed=117),
     # bf16 projection on 256 x 256 tiles (M = B*T >= 1024) with ragged M (1073) and K (72)
     "bf16_gemm256_ragged": Workload("s", L=2, D=1, I=72, H=128, T=29, B=37, dtype="bf16",
                                     state_std=0.3, seed=114),
@@ -125,6 +128,10 @@ TRAIN = {
     "B1_T1": SMALL["B1_T1"].replace(train=True),
     "f32_bi_wide": Workload("s", L=1, D=2, I=33, H=64, T=6, B=40, dtype="f32", state_std=0.2,
                             train=True, seed=110),
+    # float32 tensor-core forward in training (gate activations and cell
+    # states for the CUDA-core BPTT), with inter-layer dropout
+    "f32_tc_bi": Workload("s", L=2, D=2, I=48, H=256, T=7, B=40, dtype="f32", state_std=0.3, train=True,
+                          dropout=0.2, dropout_seed=23, seed=147),
     # bf16 BPTT: the recurrence in float32 on widened copies (W_hh rows resident
     # in bf16); the weight phase in bf16 (dG rounded to bf16) with float32 sums
     "bf16_bi_2layer": Workload("s", L=2, D=2, I=64, H=96, T=11, B=9, dtype="bf16", state_std=0.3,

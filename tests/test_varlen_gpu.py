@@ -23,6 +23,9 @@ FWD = {
                            varlen=True, seed=164),
     "bf16_tc_seqfirst": Workload("v", L=1, D=2, I=64, H=128, T=8, B=70, dtype="bf16",
                                  batch_first=False, varlen=True, seed=165),
+    # float32 tensor-core recurrence (3xTF32): padding holds h and c
+    "f32_tc_bi": Workload("v", L=2, D=2, I=40, H=256, T=8, B=36, dtype="f32", state_std=0.3,
+                          varlen=True, seed=167),
 }
 
 TRAIN = {
@@ -31,6 +34,7 @@ TRAIN = {
     "f32_bi_wide": Workload("v", L=1, D=2, I=33, H=64, T=6, B=40, dtype="f32", state_std=0.2,
                             train=True, varlen=True, seed=166),
     "bf16_bi": FWD["bf16_ffma_bi"].replace(train=True),
+    "f32_tc_bi": FWD["f32_tc_bi"].replace(train=True),
 }
 
 
