@@ -435,7 +435,8 @@ def recurrence_target(wl, kern, steps, peaks, sm_mhz):
     small batch: reading every on-chip-resident W_hh element once per step,
     at the aggregate shared-memory rate 148 SMs x 128 B/clk x the SM clock
     observed during the run (small-batch recurrence).  float32: the FP32 FMA
-    peak."""
+    peak on the CUDA cores, the 3xTF32 tensor peak (bf16 x 1.1/2.25 / 3) on
+    the tensor cores."""
     rec = [(k, v) for k, v in kern.items() if kind_base(k) == "fwd_rec" and v[0] > 0]
     if not rec:
         return None
@@ -455,6 +456,10 @@ def recurrence_target(wl, kern, steps, peaks, sm_mhz):
         return {"bound": "tensor", "kernel": kind, "us_per_step": per_step_s * 1e6, "achieved": ach,
                 "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"]}
     ach = flop / per_step_s / 1e12
+    if kind_bound(kind) == "tensor":
+        peak = peaks["bf16_tflops"] * TF32_OVER_BF16 / 3.0
+        return {"bound": "tensor", "kernel": kind, "us_per_step": per_step_s * 1e6, "achieved": ach,
+                "peak": peak, "unit": "TFLOP/s", "frac": ach / peak}
     return {"bound": "alu", "kernel": kind, "us_per_step": per_step_s * 1e6, "achieved": ach,
             "peak": alu_peak_tflops(), "unit": "TFLOP/s", "frac": ach / alu_peak_tflops()}
 

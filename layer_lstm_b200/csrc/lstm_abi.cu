@@ -815,6 +815,7 @@ lstm_status lstm_forward_varlen(const lstm_desc* desc, const int* lengths, const
             tr.timeout_ns = timeout_ns();
             tr.len = lengths;
             tr.trace = trace_for(LSTM_TRACE_FWD_REC_TC32, T, stream);
+            LSTM_CUDA(timed(K_PACK, stream, [&] { return launch_rec32_slot0(tr, stream); }));
             int nl = 1;
             LSTM_CUDA(timed(K_FWD_REC_TC, stream, [&] { return launch_tc_rec32(tr, stream, &nl); }, &nl));
             layer_in = hseq_tc;

@@ -202,7 +202,9 @@ struct TcRec32Args {
     const int* len;             // [B] valid steps per row, or null (all T)
     unsigned long long* trace;  // [kTraceSteps][kTraceEvents] or null
 };
-// *nlaunch (if given) = kernels launched (the slot-0 fill included).
+// Exchange slot 0 (hi | lo of h0, or zeros); precedes launch_tc_rec32.
+cudaError_t launch_rec32_slot0(const TcRec32Args& a, cudaStream_t s);
+// *nlaunch (if given) = recurrent kernels launched (1, or D per direction).
 cudaError_t launch_tc_rec32(const TcRec32Args& a, cudaStream_t s, int* nlaunch = nullptr);
 
 // Tensor-core BPTT recurrence (bf16 W_hh; float32 state and gate

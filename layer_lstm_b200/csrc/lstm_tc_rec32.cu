@@ -449,17 +449,20 @@ bool make_map_f32_chunks(CUtensorMap* map, const void* base, long long rows, lon
 }
 }  // namespace
 
+cudaError_t launch_rec32_slot0(const TcRec32Args& a, cudaStream_t s) {
+    if (a.T <= 0 || a.B <= 0) return cudaSuccess;
+    const long long n0 = (long long)a.D * a.B * a.H;
+    rec32_slot0_kernel<<<(int)std::min<long long>((n0 + 255) / 256, 4096), 256, 0, s>>>(a.h0, a.hx, a.D, a.T, a.B,
+                                                                                        a.H);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_tc_rec32(const TcRec32Args& a, cudaStream_t s, int* nlaunch) {
     const TcRec32Plan& p = a.p;
     if (nlaunch) *nlaunch = 0;
     if (!p.ok) return cudaErrorInvalidValue;
     if (a.T <= 0 || a.B <= 0) return cudaSuccess;
-    const long long n0 = (long long)a.D * a.B * a.H;
-    rec32_slot0_kernel<<<(int)std::min<long long>((n0 + 255) / 256, 4096), 256, 0, s>>>(a.h0, a.hx, a.D, a.T, a.B,
-                                                                                        a.H);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    if (nlaunch) *nlaunch = 1;
+    cudaError_t e;
     CUtensorMap tmX;
     const long long rows = (long long)a.D * (a.T + 1) * a.B;
     if (!make_map_f32_chunks(&tmX, a.hx, rows, 2LL * a.H, p.N, p.KP / 32)) return cudaErrorInvalidValue;
@@ -494,7 +497,7 @@ cudaError_t launch_tc_rec32(const TcRec32Args& a, cudaStream_t s, int* nlaunch) 
     if (e != cudaSuccess) return e;
     if (p.C * clusters >= p.ctas) {
         e = cudaLaunchKernelEx(&cfg, kern, tmX, prm);
-        if (e == cudaSuccess && nlaunch) *nlaunch = 2;
+        if (e == cudaSuccess && nlaunch) *nlaunch = 1;
         return e;
     }
     const int per_dir = p.ctas / a.D;
@@ -505,7 +508,7 @@ cudaError_t launch_tc_rec32(const TcRec32Args& a, cudaStream_t s, int* nlaunch) 
         e = cudaLaunchKernelEx(&cfg, kern, tmX, prm);
         if (e != cudaSuccess) return e;
     }
-    if (nlaunch) *nlaunch = 1 + a.D;
+    if (nlaunch) *nlaunch = a.D;
     return cudaSuccess;
 }
 

@@ -131,6 +131,22 @@ def test_recurrence_target_large_batch_is_tensor_peak():
     assert r["frac"] == pytest.approx(r["achieved"] / peaks["bf16_tflops"])
 
 
+def test_recurrence_target_float32_by_engine():
+    """c2 (float32): the CUDA-core recurrence against the FP32 FMA peak, the
+    tensor-core one against the 3xTF32 peak (bf16 x 1.1/2.25, three products
+    per float32 product)."""
+    wl = WORKLOADS["c2"]
+    peaks = bench.load_peaks()
+    flop = 2.0 * wl.B * 4 * wl.H * wl.H
+    r = bench.recurrence_target(wl, {"fwd_rec_tc": (4, 4 * wl.T * 5e-3)}, 2, peaks, None)
+    assert r["bound"] == "tensor"
+    assert r["achieved"] == pytest.approx(flop / 5e-6 / 1e12)
+    assert r["peak"] == pytest.approx(peaks["bf16_tflops"] * 1.1 / 2.25 / 3)
+    r = bench.recurrence_target(wl, {"fwd_rec_ffma": (4, 4 * wl.T * 5e-3)}, 2, peaks, None)
+    assert r["bound"] == "alu"
+    assert r["peak"] == pytest.approx(bench.alu_peak_tflops())
+
+
 def test_roofline_picks_largest_counted_kind():
     wl = WORKLOADS["c5"]
     kern = {"fwd_rec_ffma": (4, 3.0), "bwd_rec_ffma": (4, 4.0), "transpose": (40, 9.0),
