@@ -14,7 +14,7 @@ LIB_PATH = os.path.join(HERE, "liblstm_b200.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
 
 SOURCES = ["lstm_abi.cu", "lstm_simt.cu", "lstm_rec.cu", "lstm_tc_gemm.cu", "lstm_tc_rec.cu", "lstm_tc_rec32.cu",
-           "lstm_tc_bwd.cu", "lstm_noalloc.cu"]
+           "lstm_tc_bwd.cu", "lstm_tc_bwd32.cu", "lstm_noalloc.cu"]
 HEADERS = ["lstm_device.cuh", "lstm_internal.h", "lstm_tc.cuh", "lstm_tc_cluster.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

@@ -240,6 +240,8 @@ struct Layout {
     size_t ctr_tcb, dax, wT_tcb;
     TcRec32Plan tc32;  // tensor-core forward recurrence for float32 (3xTF32), if it fits
     size_t ctr_tc32, hx32;
+    TcBwd32Plan tcb32; // tensor-core BPTT recurrence for float32 (3xTF32), if it fits
+    size_t ctr_tcb32, dax32, wT32;
     size_t status, ctr_f, ctr_b, ctr_tc, ctr_end, wih[32], bias[32], whh_f, whh_b, gx, hT, seq[2], dG, dseq[2], xt,
         dbpart, P, dGT, bop, wcatT, hx, whh_tc, bias_dummy, gemm_ws, total;
     size_t gemm_ws_floats;
@@ -302,6 +304,7 @@ bool make_layout(const lstm_desc* d, Layout& l) {
     l.tcr = l.dt == DType::BF16 ? plan_tc_rec(l.H, Bp, l.D, dev.sms, smem_max) : TcRecPlan{};
     l.tcb = l.dt == DType::BF16 ? plan_tc_bwd(l.H, Bp, l.D, dev.sms, smem_max) : TcBwdPlan{};
     l.tc32 = l.dt == DType::F32 ? plan_tc_rec32(l.H, Bp, l.D, dev.sms, smem_max) : TcRec32Plan{};
+    l.tcb32 = l.dt == DType::F32 ? plan_tc_bwd32(l.H, Bp, l.D, dev.sms, smem_max) : TcBwd32Plan{};
     const size_t TB = (size_t)l.T * l.B;
     size_t o = 0;
     l.status = o; o += al(sizeof(int));
@@ -313,6 +316,7 @@ bool make_layout(const lstm_desc* d, Layout& l) {
     l.ctr_tc = o; o += al(l.tcr.ok ? sizeof(unsigned) * 32 * (size_t)l.L * l.D * l.tcr.nbg : 0);
     l.ctr_tcb = o; o += al(l.tcb.ok ? sizeof(unsigned) * 32 * (size_t)l.L * l.D * l.tcb.nbg : 0);
     l.ctr_tc32 = o; o += al(l.tc32.ok ? sizeof(unsigned) * 32 * (size_t)l.L * l.D * l.tc32.nbg : 0);
+    l.ctr_tcb32 = o; o += al(l.tcb32.ok ? sizeof(unsigned) * 32 * (size_t)l.L * l.D * l.tcb32.nbg : 0);
     l.ctr_end = o;
     for (int k = 0; k < l.L; ++k) {
         l.wih[k] = o; o += al((size_t)l.D * l.G * in_size(l, k) * l.es);
@@ -356,11 +360,14 @@ bool make_layout(const lstm_desc* d, Layout& l) {
     l.dseq[0] = o; o += al(TB * maxin * 4);
     l.dseq[1] = o; o += al(TB * maxin * 4);
     l.xt = o; o += al(TB * l.I * 4);
-    const int nbg_db = std::max(l.bwd_ok ? l.bwd.nbg : 1, l.tcb.ok ? l.tcb.nbg : 1);
+    const int nbg_db = std::max({l.bwd_ok ? l.bwd.nbg : 1, l.tcb.ok ? l.tcb.nbg : 1, l.tcb32.ok ? l.tcb32.nbg : 1});
     l.dbpart = o; o += al((size_t)l.D * nbg_db * l.G * 4);
     // tensor-core BPTT: packed W_hh^T and the bf16 exchange of the gate gradients
     l.wT_tcb = o; o += al(l.tcb.ok ? (size_t)l.D * l.H * l.G * 2 : 0);
     l.dax = o; o += al(l.tcb.ok ? (size_t)l.D * (l.T + 1) * l.B * l.G * 2 : 0);
+    // float32 tensor-core BPTT: packed W_hh^T and the ring of split gate gradients
+    l.wT32 = o; o += al(l.tcb32.ok ? (size_t)l.D * l.H * l.G * 4 : 0);
+    l.dax32 = o; o += al(l.tcb32.ok ? (size_t)l.D * l.tcb32.slots * l.B * 2 * l.G * 4 : 0);
     l.P = o; o += al(l.bwd_ok ? (size_t)2 * l.D * l.bwd.nbg * l.bwd.nu * l.bwd.Bg * Hp * 4 : 0);
     l.dGT = o; o += al(TB * l.D * l.G * 4);
     l.bop = o; o += al((size_t)l.D * (maxin + l.H) * TB * 4);
@@ -1064,7 +1071,8 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
         // bf16: the tensor-core BPTT recurrence when its plan fits (the same
         // switch as the forward's engine), else the CUDA-core one
         const bool tcb = bf && l.tcb.ok && tc_rec_enabled();
-        if (!tcb) {
+        const bool tcb32 = !bf && l.tcb32.ok && tc_rec_enabled();
+        if (!tcb && !tcb32) {
             PackHhBwdArgs pb{};
             pb.H = H; pb.D = D; pb.nu = l.bwd.nu; pb.U = l.bwd.U;
             pb.dt = l.dt;
@@ -1097,7 +1105,7 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
         b.skip_step = skip_arrival().bwd_step;
         if (tcb) {
             PackWtArgs pw{};
-            pw.H = H; pw.D = D;
+            pw.H = H; pw.D = D; pw.dt = DType::BF16;
             for (int d = 0; d < D; ++d) pw.w[d] = w_hh[k * D + d];
             pw.out = P(workspace, l.wT_tcb);
             LSTM_CUDA(timed(K_PACK, stream, [&] { return launch_pack_wT(pw, stream); }));
@@ -1117,13 +1125,34 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
             tb.len = lengths;
             int nl = 1;
             LSTM_CUDA(timed(K_BWD_REC_TC, stream, [&] { return launch_tc_bwd(tb, stream, &nl); }, &nl));
+        } else if (tcb32) {
+            PackWtArgs pw{};
+            pw.H = H; pw.D = D; pw.dt = DType::F32;
+            for (int d = 0; d < D; ++d) pw.w[d] = w_hh[k * D + d];
+            pw.out = P(workspace, l.wT32);
+            LSTM_CUDA(timed(K_PACK, stream, [&] { return launch_pack_wT(pw, stream); }));
+            TcBwd32Args tb{};
+            tb.H = H; tb.B = B; tb.T = T; tb.D = D; tb.p = l.tcb32;
+            tb.wT = reinterpret_cast<const float*>(pw.out);
+            tb.act = b.act; tb.cst = b.cst; tb.c0 = b.c0;
+            tb.dy = b.dy; tb.dy_st = b.dy_st; tb.dy_sb = b.dy_sb;
+            tb.grad_hn = b.grad_hn; tb.grad_cn = b.grad_cn;
+            tb.dG = dG;
+            tb.dax = reinterpret_cast<float*>(P(workspace, l.dax32));
+            tb.dh0 = b.dh0; tb.dc0 = b.dc0; tb.dbpart = b.dbpart;
+            tb.ctr = reinterpret_cast<unsigned*>(P(workspace, l.ctr_tcb32)) + (size_t)k * D * l.tcb32.nbg * 32;
+            tb.status = status;
+            tb.timeout_ns = timeout_ns();
+            tb.len = lengths;
+            int nl = 1;
+            LSTM_CUDA(timed(K_BWD_REC_TC, stream, [&] { return launch_tc_bwd32(tb, stream, &nl); }, &nl));
         } else {
             LSTM_CUDA(timed(K_BWD_REC_FFMA, stream, [&] { return launch_bwd_rec(b, stream); }));
         }
 
         if (desc->bias) {
             DbArgs db{};
-            db.G = G; db.D = D; db.nbg = tcb ? l.tcb.nbg : l.bwd.nbg; db.dbpart = b.dbpart;
+            db.G = G; db.D = D; db.nbg = tcb ? l.tcb.nbg : tcb32 ? l.tcb32.nbg : l.bwd.nbg; db.dbpart = b.dbpart;
             for (int d = 0; d < D; ++d) { db.db_ih[d] = db_ih[k * D + d]; db.db_hh[d] = db_hh[k * D + d]; }
             LSTM_CUDA(timed(K_DB, stream, [&] { return launch_db_reduce(db, stream); }));
         }

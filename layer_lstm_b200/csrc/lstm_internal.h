@@ -207,6 +207,38 @@ cudaError_t launch_rec32_slot0(const TcRec32Args& a, cudaStream_t s);
 // *nlaunch (if given) = recurrent kernels launched (1, or D per direction).
 cudaError_t launch_tc_rec32(const TcRec32Args& a, cudaStream_t s, int* nlaunch = nullptr);
 
+// Tensor-core BPTT recurrence for float32 problems (3xTF32): clusters of
+// H/32 blocks per 128-unit slice split K = 4H in parts of 128 gates (H = 128,
+// 256 or 512); the gate gradients are exchanged split tf32 part | remainder
+// through a ring of `slots` slots.
+struct TcBwd32Plan {
+    bool ok;
+    int nbg, Bg, N, nsl, Cl, ctas, slots;
+    size_t smem;
+};
+TcBwd32Plan plan_tc_bwd32(int H, int B, int D, int num_sms, size_t smem_max);
+struct TcBwd32Args {
+    int H, B, T, D;
+    TcBwd32Plan p;
+    const float* wT;            // [D][H][4H] packed W_hh^T (launch_pack_wT, float32)
+    const float* act;           // [D][T][B][4H] saved gate activations (i, f, g, o per unit)
+    const float* cst;           // [D][T][B][H] saved cell states
+    const float* c0;            // [D][B][H] or null
+    const float* dy; long long dy_st, dy_sb;   // gradient reaching the layer output
+    const float* grad_hn;       // [D][B][H] or null
+    const float* grad_cn;       // [D][B][H] or null
+    float* dG;                  // [T][B][D*4H] gate gradients, standard row order
+    float* dax;                 // exchange [D][slots][B][8H]
+    float* dh0; float* dc0;     // [D][B][H]
+    float* dbpart;              // [D][nbg][4H] bias-gradient partials
+    unsigned* ctr;              // [D][nbg] counters, 32 words apart, zeroed
+    int* status;
+    uint64_t timeout_ns;
+    const int* len;             // [B] valid steps per row, or null (all T)
+};
+// *nlaunch (if given) = kernels launched.
+cudaError_t launch_tc_bwd32(const TcBwd32Args& a, cudaStream_t s, int* nlaunch = nullptr);
+
 // Tensor-core BPTT recurrence (bf16 W_hh; float32 state and gate
 // gradients; the gate gradients of each step exchanged in bf16).  Clusters of
 // 8 blocks per (direction, batch group, 128-unit slice) split K = 4H.
@@ -244,8 +276,9 @@ cudaError_t launch_tc_bwd(const TcBwdArgs& a, cudaStream_t s, int* nlaunch = nul
 // packed gate order of the tensor-core BPTT recurrence.
 struct PackWtArgs {
     int H, D;
-    const void* w[2];           // W_hh of each direction, [4H][H] bf16
-    void* out;
+    DType dt;                   // element type of w and out
+    const void* w[2];           // W_hh of each direction, [4H][H]
+    void* out;                  // [D][H][4H]: out[d][u][4u'+q] = W[d][q*H + u'][u]
 };
 cudaError_t launch_pack_wT(const PackWtArgs& a, cudaStream_t s);
 

@@ -71,18 +71,20 @@ struct TcBwdParams {
     const int* len;
 };
 
-// out[d][u][4u'+q] = W[d][q*H + u'][u]: a 32 x 32 tile transpose per gate q.
+// out[d][u][4u'+q] = W[d][q*H + u'][u]: a 32 x 32 tile transpose per gate q
+// (bf16 for this kernel, float32 for the 3xTF32 one).
+template <typename E>
 __global__ void pack_wT_kernel(PackWtArgs a) {
-    __shared__ bf16 tile[32][34];
+    __shared__ E tile[32][34];
     const int H = a.H;
     const int u0 = blockIdx.x * 32, v0 = blockIdx.y * 32;   // u: column of W (row of out), v = u'
     const int q = blockIdx.z % 4, d = blockIdx.z / 4;
-    const bf16* w = static_cast<const bf16*>(a.w[d]);
-    bf16* out = static_cast<bf16*>(a.out) + (size_t)d * H * 4 * H;
+    const E* w = static_cast<const E*>(a.w[d]);
+    E* out = static_cast<E*>(a.out) + (size_t)d * H * 4 * H;
     const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 32 x 8 threads
     for (int i = ty; i < 32; i += 8) {
         const int v = v0 + i, u = u0 + tx;
-        tile[i][tx] = (v < H && u < H) ? w[((size_t)q * H + v) * H + u] : __float2bfloat16_rn(0.f);
+        tile[i][tx] = (v < H && u < H) ? w[((size_t)q * H + v) * H + u] : E(0.f);
     }
     __syncthreads();
     for (int i = ty; i < 32; i += 8) {
@@ -428,7 +430,10 @@ TcBwdPlan plan_tc_bwd(int H, int B, int D, int num_sms, size_t smem_max) {
 cudaError_t launch_pack_wT(const PackWtArgs& a, cudaStream_t s) {
     if (a.H <= 0 || a.D <= 0) return cudaSuccess;
     const dim3 grid((a.H + 31) / 32, (a.H + 31) / 32, 4 * a.D);
-    pack_wT_kernel<<<grid, 256, 0, s>>>(a);
+    if (a.dt == DType::F32)
+        pack_wT_kernel<float><<<grid, 256, 0, s>>>(a);
+    else
+        pack_wT_kernel<bf16><<<grid, 256, 0, s>>>(a);
     return cudaGetLastError();
 }
 

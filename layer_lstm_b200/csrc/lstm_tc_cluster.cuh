@@ -115,4 +115,9 @@ __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
 bool make_map_bf16_chunks(CUtensorMap* map, const void* base, long long rows, long long cols, int box_rows,
                           int box_chunks);
 
+// The same for a float32 [rows][cols] matrix and 32-wide chunks: a box
+// {32, box_rows, box_chunks} lands 128-byte-swizzled [box_rows][32] tiles.
+bool make_map_f32_chunks(CUtensorMap* map, const void* base, long long rows, long long cols, int box_rows,
+                         int box_chunks);
+
 }  // namespace lstm

@@ -427,10 +427,8 @@ namespace {
 typedef CUresult (*EncodeTiledFn32)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                     const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                     CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+}  // namespace
 
-// 3-D TMA map of the float32 exchange [rows][2H] seen as (k within a 32-wide
-// chunk, row, chunk): a box {32, box_rows, box_chunks} lands the chunks one
-// after another, each a 128-byte-swizzled [box_rows][32] tile.
 bool make_map_f32_chunks(CUtensorMap* map, const void* base, long long rows, long long cols, int box_rows,
                          int box_chunks) {
     void* p = nullptr;
@@ -447,7 +445,6 @@ bool make_map_f32_chunks(CUtensorMap* map, const void* base, long long rows, lon
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-}  // namespace
 
 cudaError_t launch_rec32_slot0(const TcRec32Args& a, cudaStream_t s) {
     if (a.T <= 0 || a.B <= 0) return cudaSuccess;

@@ -128,10 +128,16 @@ TRAIN = {
     "B1_T1": SMALL["B1_T1"].replace(train=True),
     "f32_bi_wide": Workload("s", L=1, D=2, I=33, H=64, T=6, B=40, dtype="f32", state_std=0.2,
                             train=True, seed=110),
-    # float32 tensor-core forward in training (gate activations and cell
-    # states for the CUDA-core BPTT), with inter-layer dropout
+    # float32 on the tensor cores end to end (3xTF32 forward and BPTT
+    # recurrences; BPTT clusters of H/32 blocks): H = 256 bidirectional with
+    # inter-layer dropout (clusters of 8, two batch groups), H = 128 (clusters
+    # of 4, a ragged second batch group), H = 512 (clusters of 16)
     "f32_tc_bi": Workload("s", L=2, D=2, I=48, H=256, T=7, B=40, dtype="f32", state_std=0.3, train=True,
                           dropout=0.2, dropout_seed=23, seed=147),
+    "f32_tc_h128": Workload("s", L=2, D=1, I=24, H=128, T=9, B=50, dtype="f32", state_std=0.3, train=True,
+                            seed=148),
+    "f32_tc_h512": Workload("s", L=1, D=1, I=32, H=512, T=5, B=20, dtype="f32", state_std=0.3, train=True,
+                            seed=149),
     # bf16 BPTT: the recurrence in float32 on widened copies (W_hh rows resident
     # in bf16); the weight phase in bf16 (dG rounded to bf16) with float32 sums
     "bf16_bi_2layer": Workload("s", L=2, D=2, I=64, H=96, T=11, B=9, dtype="bf16", state_std=0.3,
