@@ -150,8 +150,10 @@ lstm_status lstm_forward(const lstm_desc* desc, const void* x, const void* h0, c
  *   dw_ih, dw_hh, db_ih, db_hh: host arrays of L*D device pointers to float32
  *     gradients, OVERWRITTEN (not accumulated); db arrays ignored if !bias.
  *     db_ih and db_hh receive the same values (the biases enter as a sum).
- * LSTM_F32 computes in float32 (3xTF32 tensor-core products in the weight
- * phase).  LSTM_BF16 keeps the cell arithmetic, the dc carry and every sum in
+ * LSTM_F32 computes in float32: 3xTF32 tensor-core products in the weight
+ * phase and, where a tensor-core plan fits (H = 128, 256 or 512, batch groups
+ * of at most 64 rows), in the recurrent products W_hh^T da too (operands
+ * split as in the forward); gate derivatives, carries and sums in float32.  LSTM_BF16 keeps the cell arithmetic, the dc carry and every sum in
  * float32, with bf16 products on the tensor cores: the recurrent products
  * W_hh^T da take the previous step's gate gradients rounded to bf16, and the
  * weight phase takes the gate gradients rounded to bf16 (x, the saved layer
@@ -299,6 +301,11 @@ void lstm_timing_reset(void);
  *     landed (first issuer), 3 its MMAs committed, 4 epilogue saw all MMAs
  *     complete, 5 partial sums sent to the column owners, 6 the owners'
  *     partial sums received, 7 cell update done, 8 h_t published.
+ *   LSTM_TRACE_BWD_REC_TC32 (row s = iteration s, 1..T): 0 producer passed
+ *     the group wait, 9 da tiles landed (first issuer), 3 its MMAs
+ *     committed, 4 epilogue saw all MMAs complete, 5 partial sums sent to the
+ *     unit owners, 6 the owners' partial sums received, 7 gate gradients
+ *     done; 8 (stamped in the next row) gate gradients published.
  * Process-wide; tracing adds one timer read and store per event to block 0.
  */
 #define LSTM_TRACE_MAX_STEPS 512
@@ -307,7 +314,8 @@ enum {
     LSTM_TRACE_FWD_REC_FFMA = 1,
     LSTM_TRACE_BWD_REC_FFMA = 2,
     LSTM_TRACE_FWD_REC_TC = 3,
-    LSTM_TRACE_FWD_REC_TC32 = 4
+    LSTM_TRACE_FWD_REC_TC32 = 4,
+    LSTM_TRACE_BWD_REC_TC32 = 5
 };
 
 lstm_status lstm_trace_enable(int enable);

@@ -32,6 +32,7 @@ LSTM_TRACE_FWD_REC_FFMA = 1
 LSTM_TRACE_BWD_REC_FFMA = 2
 LSTM_TRACE_FWD_REC_TC = 3
 LSTM_TRACE_FWD_REC_TC32 = 4
+LSTM_TRACE_BWD_REC_TC32 = 5
 
 
 class lstm_kernel_time(ctypes.Structure):

@@ -1144,6 +1144,7 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
             tb.status = status;
             tb.timeout_ns = timeout_ns();
             tb.len = lengths;
+            tb.trace = trace_for(LSTM_TRACE_BWD_REC_TC32, T, stream);
             int nl = 1;
             LSTM_CUDA(timed(K_BWD_REC_TC, stream, [&] { return launch_tc_bwd32(tb, stream, &nl); }, &nl));
         } else {

@@ -235,6 +235,7 @@ struct TcBwd32Args {
     int* status;
     uint64_t timeout_ns;
     const int* len;             // [B] valid steps per row, or null (all T)
+    unsigned long long* trace;  // [kTraceSteps][kTraceEvents] or null
 };
 // *nlaunch (if given) = kernels launched.
 cudaError_t launch_tc_bwd32(const TcBwd32Args& a, cudaStream_t s, int* nlaunch = nullptr);

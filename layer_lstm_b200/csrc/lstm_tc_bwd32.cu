@@ -80,9 +80,23 @@ struct TcBwd32Params {
     int* status;
     uint64_t timeout_ns;
     const int* len;
+    unsigned long long* trace;   // per-step timeline of block 0, or null
 };
 
 __device__ __forceinline__ float tf32_hi(float x) { return __uint_as_float(__float_as_uint(x) & 0xFFFFE000u); }
+
+// sum over src < CL of p[src * stride], in src order: the loads carry no
+// guard, so all of them are in flight at once
+template <int CL>
+__device__ __forceinline__ float sum_sources(const float* p, size_t stride) {
+    float v[CL];
+#pragma unroll
+    for (int src = 0; src < CL; ++src) v[src] = p[src * stride];
+    float sum = 0.f;
+#pragma unroll
+    for (int src = 0; src < CL; ++src) sum += v[src];
+    return sum;
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
     tc_bwd32_kernel(const __grid_constant__ CUtensorMap tmD, TcBwd32Params a) {
@@ -118,6 +132,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nblk = a.nsl * Cl;                          // blocks of the (d, bg) group
     unsigned* ctr = a.ctr + (size_t)grp * kCtrStride;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const bool tr0 = blockIdx.x == 0 && lane == 0 && warp <= 1;              // producer, first issuer
+    const bool tre = blockIdx.x == 0 && warp == 1 + kIss && lane == 0;       // an epilogue thread
 
     if (threadIdx.x == 0) {
         tc::mbar_init(full, 1);
@@ -191,6 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (s >= 2 &&
                 !__all_sync(kFullMask, tc::mbar_wait(empty, (s - 2) & 1, abort_flag, a.status, a.timeout_ns)))
                 break;
+            trace_mark(a.trace, tr0, s, 0);
             if (tc::elect_one()) {
                 const int row0 = (d * kSlots + s % kSlots) * B + b0;
                 tc::mbar_arrive_expect_tx(full, (uint32_t)(2 * nkc * tile));
@@ -219,6 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!__all_sync(kFullMask, tc::mbar_wait(full, (s - 1) & 1, abort_flag, a.status, a.timeout_ns)))
                 break;
             tc::tc_fence_after();
+            trace_mark(a.trace, tr0, s, 9);
             if (tc::elect_one()) {
                 for (int c = 0; c < nkc; ++c) {
                     const uint32_t b = tc::smem_u32(sB + c * tile);
@@ -233,6 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc::mma_commit(mma_done);
             }
             __syncwarp();
+            trace_mark(a.trace, tr0, s, 3);
             last = s;
         }
         if (*abort_flag && last > 0) {
@@ -305,6 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 tc::tc_fence_after();
+                trace_mark(a.trace, tre, s, 4);
                 // row r's partial sums over this half's columns: the three
                 // products (small cross terms first), then 4-column quads to
                 // the owner of the row's unit
@@ -329,11 +349,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc::tc_fence_before();
                 tc::mbar_arrive(d_ready);   // read: the next MMAs may overwrite the accumulators
+                trace_mark(a.trace, tre, s, 5);
                 const bool got = mbar_wait_cluster(recv_full, (s - 1) & 1, abort_flag, a.status, a.timeout_ns);
                 if (tc::named_bar_or(1, kEpi, !got)) {
                     stop = true;
                     break;
                 }
+                trace_mark(a.trace, tre, s, 6);
                 // the Cl partial sums in a fixed order, plus what padding passed on
 #pragma unroll
                 for (int k = 0; k < kMaxCells; ++k) {
@@ -341,12 +363,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (idx >= ncell) break;
                     const int b = idx / kOwn;
                     const float* p = rf + (((size_t)(b >> 2) * kOwn + ulo) * 4 + (b & 3));
-                    float sum = 0.f;
-#pragma unroll
-                    for (int src = 0; src < kMaxCl; ++src) {
-                        if (src >= Cl) break;
-                        sum += p[(size_t)src * (N / 4) * kOwn * 4];
-                    }
+                    const size_t stride = (size_t)(N / 4) * kOwn * 4;
+                    const float sum = Cl == 4 ? sum_sources<4>(p, stride)
+                                      : Cl == 8 ? sum_sources<8>(p, stride)
+                                                : sum_sources<kMaxCl>(p, stride);
                     dhin[k] = sum + dpass[k];
                 }
             }
@@ -401,10 +421,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 *reinterpret_cast<float4*>(xrow) = make_float4(hi[0], hi[1], hi[2], hi[3]);
                 *reinterpret_cast<float4*>(xrow + G) = make_float4(lo[0], lo[1], lo[2], lo[3]);
             }
+            trace_mark(a.trace, tre, s, 7);
             // publish: the exchange writes before the group's TMA reads them
             tc::fence_proxy_async_global();
             tc::named_bar_sync(1, kEpi);
             if (e == 0) red_release_add(ctr, 1u);
+            trace_mark(a.trace, tre, s + 1, 8);
         }
         // bias-gradient partial of the own units over the group's rows, in a
         // fixed order over the threads that share a unit (e = ul + kOwn m)
@@ -530,6 +552,7 @@ cudaError_t launch_tc_bwd32(const TcBwd32Args& a, cudaStream_t s, int* nlaunch) 
     prm.dh0 = a.dh0; prm.dc0 = a.dc0; prm.dbpart = a.dbpart;
     prm.ctr = a.ctr; prm.status = a.status; prm.timeout_ns = a.timeout_ns;
     prm.len = a.len;
+    prm.trace = a.trace;
     cudaLaunchConfig_t cfg;
     cudaLaunchAttribute attr[1];
     cudaError_t e = bwd32_config(p.Cl, p.smem, p.ctas, s, cfg, attr);

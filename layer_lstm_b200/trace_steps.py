@@ -63,9 +63,21 @@ PHASES = {
         ("h_t out and published", 8, 7, False),
         ("step period", 8, 8, True),
     ],
+    binding.LSTM_TRACE_BWD_REC_TC32: [
+        ("group wait (after previous publish)", 0, 8, False),
+        ("da tiles land", 9, 0, False),
+        ("MMAs issued and committed", 3, 9, False),
+        ("MMA completion seen", 4, 3, False),
+        ("partial sums sent", 5, 4, False),
+        ("owners' partial sums received", 6, 5, False),
+        ("gate gradients", 7, 6, False),
+        ("published (next row)", 8, 7, True),
+        ("step period", 0, 0, True),
+    ],
 }
 KIND_NAMES = {binding.LSTM_TRACE_FWD_REC_FFMA: "fwd_rec_ffma", binding.LSTM_TRACE_BWD_REC_FFMA: "bwd_rec_ffma",
-              binding.LSTM_TRACE_FWD_REC_TC: "fwd_rec_tc", binding.LSTM_TRACE_FWD_REC_TC32: "fwd_rec_tc32"}
+              binding.LSTM_TRACE_FWD_REC_TC: "fwd_rec_tc", binding.LSTM_TRACE_FWD_REC_TC32: "fwd_rec_tc32",
+              binding.LSTM_TRACE_BWD_REC_TC32: "bwd_rec_tc32"}
 
 
 def summarize(kind, rows):
