@@ -57,6 +57,8 @@ struct TcGemmArgs {
     int* status;
     uint64_t timeout_ns;
     int num_sms;                // persistent grid size (SMs of the device)
+    int a_mn;                   // 1: A stored [K][M] (row stride lda), contiguous in m
+    int b_mn;                   // 1: B stored [K][N] (row stride ldb), contiguous in n
 };
 bool tc_gemm_supported(const TcGemmArgs& g);
 // *nlaunch (if given) = kernels launched: 2 when K was split (GEMM + reduction).

@@ -293,7 +293,34 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
     return d;
 }
 
-// Instruction descriptor: dense, fp32 accumulator, both operands K-major.
+// Shared-memory descriptor of an MN-major operand, 128-byte swizzle: atoms of
+// 8 K-rows x 128 bytes along MN (1024 bytes, the next 8 K-rows 1024 bytes
+// further), consecutive 128-byte MN blocks `lbo` bytes apart.
+__device__ __forceinline__ uint64_t smem_desc_sw128_mn(uint32_t saddr, uint32_t lbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);          // start address
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;        // leading byte offset: MN block to MN block
+    d |= (uint64_t)(1024 >> 4) << 32;                   // stride byte offset: 8 K-rows to the next 8
+    d |= (uint64_t)1 << 46;                             // descriptor version
+    d |= (uint64_t)2 << 61;                             // SWIZZLE_128B
+    return d;
+}
+
+// The same for 32-bit (tf32) MN-major operands, which take only the 128-byte
+// swizzle on a 32-byte base: atoms of 4 K-rows x 128 bytes (the next 4 K-rows
+// 512 bytes further), 32-byte granules permuted by the K-row within the atom.
+__device__ __forceinline__ uint64_t smem_desc_sw128b32_mn(uint32_t saddr, uint32_t lbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);          // start address
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;        // leading byte offset: MN block to MN block
+    d |= (uint64_t)(512 >> 4) << 32;                    // stride byte offset: 4 K-rows to the next 4
+    d |= (uint64_t)1 << 46;                             // descriptor version
+    d |= (uint64_t)1 << 61;                             // SWIZZLE_128B_BASE32B
+    return d;
+}
+
+// Instruction descriptor: dense, fp32 accumulator, both operands K-major
+// (bit 15 / bit 16 set: A / B MN-major).
 // fmt: 1 = bf16 (kind::f16), 2 = tf32 (kind::tf32).
 __host__ __device__ constexpr uint32_t instr_desc(int fmt, int M, int N) {
     return (1u << 4) | ((uint32_t)fmt << 7) | ((uint32_t)fmt << 10) | ((uint32_t)(N >> 3) << 17) |

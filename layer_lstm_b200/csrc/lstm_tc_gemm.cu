@@ -5,8 +5,14 @@
 // sum_t da_t h_{t-1}^T (pulsatrix LSTMModule, backward()), and the
 // layer-input gradient dX = dG W_ih.
 //
-// C[M x N] = A[M x K] * B[N x K]^T with both operands K-major in global
-// memory.  A persistent grid (one CTA per SM) walks the BM x BN output tiles
+// C[M x N] = A[M x K] * B[N x K]^T, each operand K-major in global memory
+// (A[m][k] contiguous in k) or MN-major (A stored [K][M], contiguous in m:
+// the weight gradient reads dG [B*T][4H] and the layer's sequences
+// [B*T][width] as they are).  An MN-major tile lands as BM/32 (bf16: BM/64)
+// TMA boxes of [BK K-rows][128 bytes], the layout tcgen05 reads with the
+// operand's transpose bit set: bf16 with the 128-byte swizzle, float32 with
+// the 128-byte swizzle on 32-byte granules (the one MN-major layout tf32
+// operands accept).  A persistent grid (one CTA per SM) walks the BM x BN output tiles
 // (bf16 with M >= 1024: 256 x 256, two M = 128 MMAs per K step, so each
 // operand byte fetched from L2 feeds twice the products of a 128-row tile);
 // warp 0 issues TMA tile loads into a ring of shared-memory stages, warp 1
@@ -77,6 +83,7 @@ struct TcEpi {
     float* ws;                 // split-K partials [splits][M][N] or null
     int* status;
     uint64_t timeout_ns;
+    int a_mn, b_mn;            // operand stored MN-major (see launch_tc_gemm)
 };
 
 __device__ __forceinline__ long long out_row(const TcEpi& e, int m) {
@@ -174,8 +181,21 @@ __global__ void __launch_bounds__(threads_of<KIND>(), 1)
                     unsigned char* st = smem + s * Cf::STAGE_BYTES;
                     tc::mbar_arrive_expect_tx(&full[s], Cf::A_BYTES + Cf::B_BYTES);
                     const int kx = c.kbeg + kt * BK;
-                    tc::tma_load_2d(st, &tmA, kx, c.m0, &full[s]);
-                    tc::tma_load_2d(st + Cf::A_BYTES, &tmB, kx, c.n0, &full[s]);
+                    constexpr int EPB = 128 / (Cf::FMT == 2 ? 4 : 2);   // elements per 128 bytes
+                    if (!e.a_mn) {
+                        tc::tma_load_2d(st, &tmA, kx, c.m0, &full[s]);
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < Cf::BM / EPB; ++q)
+                            tc::tma_load_2d(st + q * BK * 128, &tmA, c.m0 + q * EPB, kx, &full[s]);
+                    }
+                    if (!e.b_mn) {
+                        tc::tma_load_2d(st + Cf::A_BYTES, &tmB, kx, c.n0, &full[s]);
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < BN / EPB; ++q)
+                            tc::tma_load_2d(st + Cf::A_BYTES + q * BK * 128, &tmB, c.n0 + q * EPB, kx, &full[s]);
+                    }
                 }
             }
             if (*abort_flag) {   // let this block's copies land before shared memory is released
@@ -184,7 +204,17 @@ __global__ void __launch_bounds__(threads_of<KIND>(), 1)
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            constexpr uint32_t idesc = tc::instr_desc(Cf::FMT, 128, BN);
+            const uint32_t idesc = tc::instr_desc(Cf::FMT, 128, BN) | ((uint32_t)(e.a_mn != 0) << 15) |
+                                   ((uint32_t)(e.b_mn != 0) << 16);
+            // K step j of an MMA (8 tf32 / 16 bf16 = 32 bytes of a K-major
+            // row, or that many 128-byte rows of an MN-major block)
+            constexpr uint32_t kMnStep = (Cf::FMT == 2 ? 8 : 16) * 128, kMnLbo = BK * 128;
+            const bool amn = e.a_mn != 0, bmn = e.b_mn != 0;
+            auto opd = [&](uint32_t base, int j, bool mn) {
+                if (!mn) return tc::smem_desc_sw128(base + j * 32);
+                return kTf32 ? tc::smem_desc_sw128b32_mn(base + j * kMnStep, kMnLbo)
+                             : tc::smem_desc_sw128_mn(base + j * kMnStep, kMnLbo);
+            };
             int it = 0, last = -1, i = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++i) {
@@ -208,19 +238,21 @@ __global__ void __launch_bounds__(threads_of<KIND>(), 1)
                     const uint32_t b_base = a_base + Cf::A_BYTES;
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
-                        const uint64_t ad = tc::smem_desc_sw128(a_base + j * 32);
-                        const uint64_t bd = tc::smem_desc_sw128(b_base + j * 32);
+                        const uint64_t ad = opd(a_base, j, amn);
+                        const uint64_t bd = opd(b_base, j, bmn);
                         const uint32_t acc = (kt | j) != 0;
                         if (!kTf32) {
+                            // rows [128h, 128h + 128) of the tile: 16 KB further in
+                            // either layout (128 K-major rows, or two MN blocks)
 #pragma unroll
-                            for (int h = 0; h < Cf::MH; ++h)   // rows [128h, 128h + 128) of the tile
-                                tc::mma_bf16(acc_t + (uint32_t)(h * BN), tc::smem_desc_sw128(a_base + h * 16384 + j * 32),
-                                             bd, idesc, acc);
+                            for (int h = 0; h < Cf::MH; ++h)
+                                tc::mma_bf16(acc_t + (uint32_t)(h * BN), opd(a_base + h * 16384, j, amn), bd, idesc,
+                                             acc);
                             (void)ad;
                         } else {
                             const uint32_t lo_off = Cf::A_BYTES + Cf::B_BYTES;
-                            const uint64_t adl = tc::smem_desc_sw128(a_base + lo_off + j * 32);
-                            const uint64_t bdl = tc::smem_desc_sw128(b_base + lo_off + j * 32);
+                            const uint64_t adl = opd(a_base + lo_off, j, amn);
+                            const uint64_t bdl = opd(b_base + lo_off, j, bmn);
                             tc::mma_tf32(acc_t, adl, bd, idesc, acc);   // lo * hi
                             tc::mma_tf32(acc_t, ad, bdl, idesc, 1);     // hi * lo
                             tc::mma_tf32(acc_t, ad, bd, idesc, 1);      // hi * hi
@@ -374,8 +406,9 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
+// mn32: a float32 MN-major operand (128-byte swizzle on 32-byte granules)
 bool make_map(CUtensorMap* map, DType dt, const void* base, long long rows, long long cols, long long ld,
-              int box_rows) {
+              int box_rows, bool mn32 = false) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     const size_t es = dtype_size(dt);
@@ -385,7 +418,8 @@ bool make_map(CUtensorMap* map, DType dt, const void* base, long long rows, long
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(map, dt == DType::F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                      2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     mn32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -394,9 +428,17 @@ template <int KIND>
 cudaError_t launch_kind(const TcGemmArgs& g, cudaStream_t s, int* nlaunch) {
     using Cf = Cfg<KIND>;
     CUtensorMap ta, tb;
-    if (!make_map(&ta, g.dt, g.A, g.M, g.K, g.lda, Cf::BM)) return cudaErrorInvalidValue;
-    if (!make_map(&tb, g.dt, g.B, g.N, g.K, g.ldb, Cf::BN)) return cudaErrorInvalidValue;
+    // K-major: [M][K] rows, boxes of BM rows; MN-major: [K][M] rows, boxes of
+    // BK rows (128 bytes of M each)
+    const bool f32 = g.dt == DType::F32;
+    if (!(g.a_mn ? make_map(&ta, g.dt, g.A, g.K, g.M, g.lda, Cf::BK, f32)
+                 : make_map(&ta, g.dt, g.A, g.M, g.K, g.lda, Cf::BM)))
+        return cudaErrorInvalidValue;
+    if (!(g.b_mn ? make_map(&tb, g.dt, g.B, g.K, g.N, g.ldb, Cf::BK, f32)
+                 : make_map(&tb, g.dt, g.B, g.N, g.K, g.ldb, Cf::BN)))
+        return cudaErrorInvalidValue;
     TcEpi e{};
+    e.a_mn = g.a_mn; e.b_mn = g.b_mn;
     e.M = g.M; e.N = g.N; e.K = g.K;
     const int kchunks = (g.K + Cf::BK - 1) / Cf::BK;
     const int sms = g.num_sms > 0 ? g.num_sms : 148;
@@ -452,7 +494,9 @@ bool tc_gemm_supported(const TcGemmArgs& g) {
     const size_t es = dtype_size(g.dt);
     if ((g.lda * es) % 16 != 0 || (g.ldb * es) % 16 != 0) return false;
     if ((reinterpret_cast<uintptr_t>(g.A) & 15) || (reinterpret_cast<uintptr_t>(g.B) & 15)) return false;
-    if (g.K < (long long)(128 / es)) return false;   // at least one full 128-byte K chunk
+    // the contiguous dimension of each operand spans at least one 128-byte box
+    const long long inner = 128 / (long long)es;
+    if ((g.a_mn ? g.M : g.K) < inner || (g.b_mn ? g.N : g.K) < inner) return false;
     return true;
 }
 
