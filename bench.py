@@ -253,7 +253,7 @@ def traffic_for(kind, wl_name):
         return None
     with open(p) as f:
         d = json.load(f)
-    e = d.get(kind)
+    e = d.get(f"{kind}@{wl_name}") or d.get(kind)   # one kind can name several kernels
     if not e or e.get("workload") != wl_name:
         return None
     src = os.path.join(ROOT, e["source"])
