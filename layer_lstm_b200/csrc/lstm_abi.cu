@@ -155,6 +155,15 @@ cudaError_t timed(int kind, cudaStream_t s, F&& f, const int* nlaunch = nullptr)
     return cudaSuccess;
 }
 
+// Launches of `kind` that ran inside another kind's timed interval (counted,
+// their time is part of that interval).
+void count_launches(int kind, int n) {
+    Timing& tm = timing();
+    if (!tm.on) return;
+    std::lock_guard<std::mutex> lk(tm.mu);
+    tm.launches[kind] += n;
+}
+
 // GEMM engine: tensor cores where the operands meet TMA's alignment rules,
 // the CUDA-core kernel otherwise.  LSTM_B200_GEMM=simt forces the CUDA-core
 // kernel everywhere (used by the tests to cover both engines).
@@ -1071,6 +1080,11 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
     long long dy_st = desc->batch_first ? (long long)D * H : (long long)B * D * H;
     long long dy_sb = desc->batch_first ? (long long)T * D * H : (long long)D * H;
     int cur = 0;
+    // float32: the weight-gradient GEMMs of layer k + 1 run beside layer k's
+    // tensor-core BPTT recurrence, which leaves SMs idle (its operands are
+    // copies the transposes made before; the recurrence writes none of them)
+    const bool overlap_dw = !bf && l.tcb32.ok && tc_rec_enabled() && device_info().sms > l.tcb32.ctas;
+    std::vector<TcGemmArgs> deferred_dw;
     for (int k = L - 1; k >= 0; --k) {
         const int in = in_size(l, k);
         // bf16: the tensor-core BPTT recurrence when its plan fits (the same
@@ -1150,8 +1164,25 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
             tb.timeout_ns = timeout_ns();
             tb.len = lengths;
             tb.trace = trace_for(LSTM_TRACE_BWD_REC_TC32, T, stream);
-            int nl = 1;
-            LSTM_CUDA(timed(K_BWD_REC_TC, stream, [&] { return launch_tc_bwd32(tb, stream, &nl); }, &nl));
+            int nl = 1, ndw = 0;
+            LSTM_CUDA(timed(K_BWD_REC_TC, stream, [&] {
+                cudaError_t e = launch_tc_bwd32(tb, stream, &nl);
+                // the deferred GEMMs right behind it: the first as its programmatic
+                // dependent on the SMs it leaves, the others in order after that one
+                for (size_t i = 0; i < deferred_dw.size() && e == cudaSuccess; ++i) {
+                    TcGemmArgs g = deferred_dw[i];
+                    if (i == 0) {
+                        g.pdl = 1;
+                        g.num_sms = device_info().sms - l.tcb32.ctas;
+                    }
+                    int n = 1;
+                    e = launch_tc_gemm(g, stream, &n);
+                    ndw += n;
+                }
+                return e;
+            }, &nl));
+            count_launches(K_DW_TC, ndw);
+            deferred_dw.clear();
         } else {
             LSTM_CUDA(timed(K_BWD_REC_FFMA, stream, [&] { return launch_bwd_rec(b, stream); }));
         }
@@ -1299,7 +1330,9 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
                 twd.B = bo;
                 twd.C = dw_ih[k * D + d];
                 twd.C1 = dw_hh[k * D + d];
-                {
+                if (overlap_dw && k > 0) {
+                    deferred_dw.push_back(twd);   // launched behind layer k-1's recurrence
+                } else {
                     int nl = 1;
                     LSTM_CUDA(timed(K_DW_TC, stream, [&] { return launch_tc_gemm(twd, stream, &nl); }, &nl));
                 }

@@ -59,6 +59,9 @@ struct TcGemmArgs {
     int num_sms;                // persistent grid size (SMs of the device)
     int a_mn;                   // 1: A stored [K][M] (row stride lda), contiguous in m
     int b_mn;                   // 1: B stored [K][N] (row stride ldb), contiguous in n
+    int pdl;                    // 1: launch as a programmatic dependent of the preceding kernel in
+                                // the stream (it may start once that kernel's blocks signalled and
+                                // ends only after it); the GEMM must not read what that kernel writes
 };
 bool tc_gemm_supported(const TcGemmArgs& g);
 // *nlaunch (if given) = kernels launched: 2 when K was split (GEMM + reduction).

@@ -189,6 +189,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
+    // every block is resident: a programmatic dependent launched behind this
+    // grid (a weight-gradient GEMM of the layer above) may start on the SMs left
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     if (warp == 0) {
         // ---------------------------------------------------- da producer

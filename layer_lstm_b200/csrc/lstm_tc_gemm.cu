@@ -84,6 +84,7 @@ struct TcEpi {
     int* status;
     uint64_t timeout_ns;
     int a_mn, b_mn;            // operand stored MN-major (see launch_tc_gemm)
+    int pdl_wait;              // launched as a programmatic dependent: end only after the primary grid
 };
 
 __device__ __forceinline__ long long out_row(const TcEpi& e, int m) {
@@ -372,6 +373,9 @@ __global__ void __launch_bounds__(threads_of<KIND>(), 1)
         tc::tc_fence_after();
         tc::tmem_dealloc(tmem, Cf::NACC * Cf::MH * BN);
     }
+    // A programmatic dependent of a recurrence ran beside it; it completes only
+    // after that grid has, so work behind it in the stream stays ordered after both.
+    if (e.pdl_wait) asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 __global__ void splitk_reduce_kernel(TcEpi e, int splits) {
@@ -475,8 +479,25 @@ cudaError_t launch_kind(const TcGemmArgs& g, cudaStream_t s, int* nlaunch) {
     e.splits = splits;
     const long long ntiles = (long long)e.tiles_n * e.tiles_m * splits;
     const int grid = (int)std::min<long long>(ntiles, sms);
-    tc_gemm_kernel<KIND><<<grid, threads_of<KIND>(), smem, s>>>(ta, tb, e);
-    err = cudaGetLastError();
+    if (g.pdl) {
+        // starts once every block of the preceding kernel in the stream (a
+        // persistent recurrence) has signalled; runs on the SMs it leaves free
+        e.pdl_wait = 1;
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3(threads_of<KIND>());
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        err = cudaLaunchKernelEx(&cfg, tc_gemm_kernel<KIND>, ta, tb, e);
+    } else {
+        tc_gemm_kernel<KIND><<<grid, threads_of<KIND>(), smem, s>>>(ta, tb, e);
+        err = cudaGetLastError();
+    }
     if (nlaunch) *nlaunch = 1;
     if (err != cudaSuccess || splits == 1) return err;
     const long long total = (long long)g.M * g.N;
