@@ -22,8 +22,9 @@
 // 4H gates in the packed order 4u'+q.  A cluster of Cl = H/32 blocks owns
 // one slice: block rank k keeps the K part [128k, 128k + 128) of the slice's
 // rows of W_hh^T in tensor memory, hi and lo side by side (the A operand),
-// multiplies it by the same part of da_{t+1} (hi and lo, two TMA boxes per
-// step, from a ring of 4 exchange slots) with one issuing warp per product
+// multiplies it by the same part of da_{t+1} (hi and lo, from a ring of 4
+// exchange slots, in kSeg K segments on a barrier each so the MMAs of the
+// first segment run while the next lands) with one issuing warp per product
 // into three accumulators, and sends each unit's partial sums to the block
 // that owns the unit (128/Cl units per block; asynchronous distributed-
 // shared-memory stores completing on the owner's mbarrier).  The owner adds
@@ -57,6 +58,7 @@ constexpr int kMaxCells = 4;              // gate-gradient cells per epilogue th
 constexpr uint32_t kAcol = 256;           // tensor-memory column of the resident W_hh^T part (hi, then lo)
 static_assert(kIss * kMaxN <= (int)kAcol, "the accumulators fit below the resident W_hh^T part");
 constexpr int kSlots = 4;                 // ring of gate-gradient exchange slots
+constexpr int kSeg = 2;                   // K segments of a step's da tiles, each on its own barrier
 constexpr size_t kMinSmem = 120 * 1024;   // two blocks never share an SM (512 TMEM columns each)
 constexpr int kCtrStride = 32;
 constexpr unsigned kFullMask = 0xffffffffu;
@@ -111,8 +113,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // partial sums received for the own units: [src][N/4 column quads][kOwn] float4
     float4* recv = reinterpret_cast<float4*>(sBl + nkc * tile);
     float* dbred = reinterpret_cast<float*>(recv + (size_t)Cl * (N / 4) * kOwn);   // [kEpi][4]
-    uint64_t* full = reinterpret_cast<uint64_t*>(dbred + kEpi * 4);
-    uint64_t* empty = full + 1;
+    uint64_t* full = reinterpret_cast<uint64_t*>(dbred + kEpi * 4);   // [kSeg]
+    uint64_t* empty = full + kSeg;
     uint64_t* d_ready = empty + 1;     // the accumulators were read (count kEpi)
     uint64_t* mma_done = d_ready + 1;
     uint64_t* recv_full = mma_done + 1;
@@ -136,7 +138,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool tre = blockIdx.x == 0 && warp == 1 + kIss && lane == 0;       // an epilogue thread
 
     if (threadIdx.x == 0) {
-        tc::mbar_init(full, 1);
+        for (int i = 0; i < kSeg; ++i) tc::mbar_init(full + i, 1);
         tc::mbar_init(empty, kIss);    // one commit per issuer
         tc::mbar_init(d_ready, kEpi);
         tc::mbar_init(mma_done, kIss);
@@ -213,14 +215,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             trace_mark(a.trace, tr0, s, 0);
             if (tc::elect_one()) {
                 const int row0 = (d * kSlots + s % kSlots) * B + b0;
-                tc::mbar_arrive_expect_tx(full, (uint32_t)(2 * nkc * tile));
-                tc::tma_load_3d(sBh, &tmD, 0, row0, kbeg / 32, full);
-                tc::tma_load_3d(sBl, &tmD, 0, row0, (G + kbeg) / 32, full);
+                const int cps = nkc / kSeg;   // chunks per segment
+                for (int sg = 0; sg < kSeg; ++sg) {
+                    tc::mbar_arrive_expect_tx(full + sg, (uint32_t)(2 * cps * tile));
+                    tc::tma_load_3d(sBh + sg * cps * tile, &tmD, 0, row0, kbeg / 32 + sg * cps, full + sg);
+                    tc::tma_load_3d(sBl + sg * cps * tile, &tmD, 0, row0, (G + kbeg) / 32 + sg * cps, full + sg);
+                }
             }
             __syncwarp();
             ++issued;
         }
-        if (*abort_flag && issued > 0) drain_wait(full, (issued - 1) & 1);
+        if (*abort_flag && issued > 0)
+            for (int sg = 0; sg < kSeg; ++sg) drain_wait(full + sg, (issued - 1) & 1);
     } else if (warp <= kIss) {
         // ------------------------------------------------------------ MMA
         // product pr: A = W_hi (pr < 2) or W_lo, B = da_hi (pr != 1) or da_lo,
@@ -236,26 +242,34 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!__all_sync(kFullMask, tc::mbar_wait(d_ready, (s - 1) & 1, abort_flag, a.status, a.timeout_ns)))
                 break;
             tc::tc_fence_after();
-            if (!__all_sync(kFullMask, tc::mbar_wait(full, (s - 1) & 1, abort_flag, a.status, a.timeout_ns)))
-                break;
-            tc::tc_fence_after();
-            trace_mark(a.trace, tr0, s, 9);
-            if (tc::elect_one()) {
-                for (int c = 0; c < nkc; ++c) {
-                    const uint32_t b = tc::smem_u32(sB + c * tile);
+            last = s;   // from here MMAs of iteration s may be in flight (drained on abort)
+            bool ok = true;
+            const int cps = nkc / kSeg;
+            for (int sg = 0; sg < kSeg && ok; ++sg) {
+                ok = __all_sync(kFullMask, tc::mbar_wait(full + sg, (s - 1) & 1, abort_flag, a.status, a.timeout_ns));
+                if (!ok) break;
+                tc::tc_fence_after();
+                if (sg == 0) trace_mark(a.trace, tr0, s, 9);
+                if (tc::elect_one()) {
+                    for (int c = sg * cps; c < (sg + 1) * cps; ++c) {
+                        const uint32_t b = tc::smem_u32(sB + c * tile);
 #pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {   // k-steps of 8 tf32 (32 bytes of a 128-byte row)
-                        const uint32_t aa = tmem + kAcol + aoff + (uint32_t)(32 * c + 8 * jj);
-                        tc::mma_tf32_ts(acc, aa, tc::smem_desc_sw128(b + 32 * jj), idesc,
-                                        (c | jj) != 0);   // fresh accumulator each iteration
+                        for (int jj = 0; jj < 4; ++jj) {   // k-steps of 8 tf32 (32 bytes of a 128-byte row)
+                            const uint32_t aa = tmem + kAcol + aoff + (uint32_t)(32 * c + 8 * jj);
+                            tc::mma_tf32_ts(acc, aa, tc::smem_desc_sw128(b + 32 * jj), idesc,
+                                            (c | jj) != 0);   // fresh accumulator each iteration
+                        }
                     }
                 }
+                __syncwarp();
+            }
+            if (!ok) break;
+            if (tc::elect_one()) {
                 tc::mma_commit(empty);
                 tc::mma_commit(mma_done);
             }
             __syncwarp();
             trace_mark(a.trace, tr0, s, 3);
-            last = s;
         }
         if (*abort_flag && last > 0) {
             // the other issuers may have stopped an iteration earlier: wait
@@ -542,7 +556,7 @@ cudaError_t launch_tc_bwd32(const TcBwd32Args& a, cudaStream_t s, int* nlaunch) 
     if (a.T <= 0 || a.B <= 0) return cudaSuccess;
     CUtensorMap tmD;
     const long long rows = (long long)a.D * kSlots * a.B;
-    if (!make_map_f32_chunks(&tmD, a.dax, rows, 8LL * a.H, p.N, kKP / 32)) return cudaErrorInvalidValue;
+    if (!make_map_f32_chunks(&tmD, a.dax, rows, 8LL * a.H, p.N, kKP / 32 / kSeg)) return cudaErrorInvalidValue;
     TcBwd32Params prm{};
     prm.H = a.H; prm.B = a.B; prm.T = a.T; prm.D = a.D;
     prm.nbg = p.nbg; prm.Bg = p.Bg; prm.N = p.N; prm.nsl = p.nsl; prm.Cl = p.Cl;

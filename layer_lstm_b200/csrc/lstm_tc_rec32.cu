@@ -17,7 +17,9 @@
 // tensor memory, hi and lo side by side (the A operand of tcgen05.mma), and
 // owns the columns [r*N/C, (r+1)*N/C).  Per step:
 //   warp 0:    wait for the group's h_{t-1}, TMA the block's K part of it,
-//              hi and lo (two 3-D boxes, 128-byte swizzle)
+//              hi and lo, in kSeg K segments (3-D boxes, 128-byte swizzle)
+//              completing on a barrier each, so the MMAs of the first
+//              segment run while the next lands
 //   warps 1-3: one product each (hi*hi, hi*lo, lo*hi), an MMA per k-step
 //              of 8 into an accumulator of its own: three issuing threads
 //              keep the tensor pipe busy at N <= 64, where one issues an
@@ -50,6 +52,7 @@ constexpr uint32_t kAcol = 256;           // tensor-memory column of the residen
 static_assert(kIss * kMaxN <= (int)kAcol, "the accumulators fit below the resident W_hh part");
 constexpr int kMaxKP = 128;               // K part per block: hi + lo fill the 256 columns
 constexpr int kMaxC = 8;                  // blocks per cluster (H <= 1024)
+constexpr int kSeg = 2;                   // K segments of a step's h tiles, each on its own barrier
 constexpr size_t kMinSmem = 120 * 1024;   // two blocks never share an SM (512 TMEM columns each)
 constexpr int kCtrStride = 32;
 constexpr unsigned kFullMask = 0xffffffffu;
@@ -106,8 +109,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // partial sums of the own columns from the C blocks: [src][NO/4 column
     // quads][128 lanes] float4 (4 columns of one gate row)
     float4* recv = reinterpret_cast<float4*>(sBl + nkc * tile);
-    uint64_t* full = reinterpret_cast<uint64_t*>(recv + (size_t)C * (NO / 4) * kRows);
-    uint64_t* empty = full + 1;
+    uint64_t* full = reinterpret_cast<uint64_t*>(recv + (size_t)C * (NO / 4) * kRows);   // [kSeg]
+    uint64_t* empty = full + kSeg;
     uint64_t* d_ready = empty + 1;     // the accumulator was read (count kEpi)
     uint64_t* mma_done = d_ready + 1;
     uint64_t* recv_full = mma_done + 1;
@@ -131,7 +134,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool tre = blockIdx.x == 0 && warp == 1 + kIss && lane == 0;       // an epilogue thread
 
     if (threadIdx.x == 0) {
-        tc::mbar_init(full, 1);
+        for (int i = 0; i < kSeg; ++i) tc::mbar_init(full + i, 1);
         tc::mbar_init(empty, kIss);    // one commit per issuer
         tc::mbar_init(d_ready, kEpi);
         tc::mbar_init(mma_done, kIss);
@@ -203,14 +206,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             trace_mark(a.trace, tr0, s, 0);
             if (tc::elect_one()) {
                 const int row0 = (d * (T + 1) + s) * B + b0;
-                tc::mbar_arrive_expect_tx(full, (uint32_t)(2 * nkc * tile));
-                tc::tma_load_3d(sBh, &tmX, 0, row0, kbeg / 32, full);
-                tc::tma_load_3d(sBl, &tmX, 0, row0, (H + kbeg) / 32, full);
+                const int cps = nkc / kSeg;   // chunks per segment
+                for (int sg = 0; sg < kSeg; ++sg) {
+                    tc::mbar_arrive_expect_tx(full + sg, (uint32_t)(2 * cps * tile));
+                    tc::tma_load_3d(sBh + sg * cps * tile, &tmX, 0, row0, kbeg / 32 + sg * cps, full + sg);
+                    tc::tma_load_3d(sBl + sg * cps * tile, &tmX, 0, row0, (H + kbeg) / 32 + sg * cps, full + sg);
+                }
             }
             __syncwarp();
             ++issued;
         }
-        if (*abort_flag && issued > 0) drain_wait(full, (issued - 1) & 1);
+        if (*abort_flag && issued > 0)
+            for (int sg = 0; sg < kSeg; ++sg) drain_wait(full + sg, (issued - 1) & 1);
     } else if (warp <= kIss) {
         // ------------------------------------------------------------ MMA
         // product pr: A = W_hi (pr < 2) or W_lo, B = h_hi (pr != 1) or h_lo,
@@ -224,25 +231,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < T; ++s) {
             if (!__all_sync(kFullMask, tc::mbar_wait(d_ready, s & 1, abort_flag, a.status, a.timeout_ns))) break;
             tc::tc_fence_after();
-            if (!__all_sync(kFullMask, tc::mbar_wait(full, s & 1, abort_flag, a.status, a.timeout_ns))) break;
-            tc::tc_fence_after();
-            trace_mark(a.trace, tr0, s, 9);
-            if (tc::elect_one()) {
-                for (int c = 0; c < nkc; ++c) {
-                    const uint32_t b = tc::smem_u32(sB + c * tile);
+            last = s;   // from here MMAs of step s may be in flight (drained on abort)
+            bool ok = true;
+            const int cps = nkc / kSeg;
+            for (int sg = 0; sg < kSeg && ok; ++sg) {
+                ok = __all_sync(kFullMask, tc::mbar_wait(full + sg, s & 1, abort_flag, a.status, a.timeout_ns));
+                if (!ok) break;
+                tc::tc_fence_after();
+                if (sg == 0) trace_mark(a.trace, tr0, s, 9);
+                if (tc::elect_one()) {
+                    for (int c = sg * cps; c < (sg + 1) * cps; ++c) {
+                        const uint32_t b = tc::smem_u32(sB + c * tile);
 #pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {   // k-steps of 8 tf32 (32 bytes of a 128-byte row)
-                        const uint32_t aa = tmem + kAcol + aoff + (uint32_t)(32 * c + 8 * jj);
-                        tc::mma_tf32_ts(acc, aa, tc::smem_desc_sw128(b + 32 * jj), idesc,
-                                        (c | jj) != 0);   // fresh accumulator each step
+                        for (int jj = 0; jj < 4; ++jj) {   // k-steps of 8 tf32 (32 bytes of a 128-byte row)
+                            const uint32_t aa = tmem + kAcol + aoff + (uint32_t)(32 * c + 8 * jj);
+                            tc::mma_tf32_ts(acc, aa, tc::smem_desc_sw128(b + 32 * jj), idesc,
+                                            (c | jj) != 0);   // fresh accumulator each step
+                        }
                     }
                 }
+                __syncwarp();
+            }
+            if (!ok) break;
+            if (tc::elect_one()) {
                 tc::mma_commit(empty);
                 tc::mma_commit(mma_done);
             }
             __syncwarp();
             trace_mark(a.trace, tr0, s, 3);
-            last = s;
         }
         if (*abort_flag && last >= 0) {
             // the other issuers may have stopped a step earlier: wait for this
@@ -462,7 +478,7 @@ cudaError_t launch_tc_rec32(const TcRec32Args& a, cudaStream_t s, int* nlaunch) 
     cudaError_t e;
     CUtensorMap tmX;
     const long long rows = (long long)a.D * (a.T + 1) * a.B;
-    if (!make_map_f32_chunks(&tmX, a.hx, rows, 2LL * a.H, p.N, p.KP / 32)) return cudaErrorInvalidValue;
+    if (!make_map_f32_chunks(&tmX, a.hx, rows, 2LL * a.H, p.N, p.KP / 32 / kSeg)) return cudaErrorInvalidValue;
     TcRec32Params prm{};
     prm.H = a.H; prm.B = a.B; prm.T = a.T; prm.D = a.D;
     prm.nbg = p.nbg; prm.Bg = p.Bg; prm.N = p.N; prm.nsl = p.nsl; prm.C = p.C; prm.KP = p.KP;
