@@ -536,41 +536,70 @@ cudaError_t launch_tc_gemm(const TcGemmArgs& g, cudaStream_t s, int* nlaunch) {
 // ---------------------------------------------------------------- transposes
 namespace {
 
-__device__ __forceinline__ float ld_elem(const void* p, long long i, int bf) {
-    return bf ? __bfloat162float(static_cast<const bf16*>(p)[i]) : static_cast<const float*>(p)[i];
+template <bool BF>
+__device__ __forceinline__ float ld_elem(const void* p, long long i) {
+    if constexpr (BF) return __bfloat162float(static_cast<const bf16*>(p)[i]);
+    return static_cast<const float*>(p)[i];
 }
 
-__global__ void transpose_kernel(TransposeArgs a) {
+template <bool BF>
+__device__ __forceinline__ void st_elem(void* p, long long i, float v) {
+    if constexpr (BF)
+        static_cast<bf16*>(p)[i] = __float2bfloat16_rn(v);
+    else
+        static_cast<float*>(p)[i] = v;
+}
+
+// 32 x 32 tiles, 32 x 8 threads: each thread's four source elements are all
+// loaded (predicated) before any goes to shared memory, so their latencies
+// overlap.
+template <int MODE, bool SB, bool DB>
+__global__ void __launch_bounds__(256) transpose_kernel(TransposeArgs a) {
     __shared__ float tile[32][33];
     const int m0 = blockIdx.x * 32, c0 = blockIdx.y * 32;
     const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 32 x 8 threads
-    for (int i = ty; i < 32; i += 8) {
-        const int m = m0 + i, c = c0 + tx;
-        float v = 0.f;
+    const int c = c0 + tx;
+    float v[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const int m = m0 + ty + 8 * r;
+        v[r] = 0.f;
         if (m < a.M && c < a.C) {
-            if (a.mode == 0) {
+            if (MODE == 0) {
                 long long row = m;
                 if (a.bt_remap) row = (long long)(m % a.B) * a.T + m / a.B;   // m = t*B + b -> b*T + t
-                v = ld_elem(a.src, row * a.lds + c, a.src_bf16);
-            } else {
+                v[r] = ld_elem<SB>(a.src, row * a.lds + c);
+            } else {   // h_{t-1} in the direction's order, h0 at its first step
                 const int t = m / a.B, b = m % a.B;
                 const int ts = a.dir == 0 ? t - 1 : t + 1;
-                if (ts >= 0 && ts < a.T) v = ld_elem(a.src, ((long long)ts * a.B + b) * a.lds + c, a.src_bf16);
-                else if (a.h0) v = ld_elem(a.h0, (long long)b * a.C + c, a.src_bf16);
+                if (ts >= 0 && ts < a.T)
+                    v[r] = ld_elem<SB>(a.src, ((long long)ts * a.B + b) * a.lds + c);
+                else if (a.h0)
+                    v[r] = ld_elem<SB>(a.h0, (long long)b * a.C + c);
             }
         }
-        tile[i][tx] = v;
     }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) tile[ty + 8 * r][tx] = v[r];
     __syncthreads();
-    for (int i = ty; i < 32; i += 8) {
-        const int c = c0 + i, m = m0 + tx;
-        if (m < a.M && c < a.C) {
-            if (a.dst_bf16)
-                static_cast<bf16*>(a.dst)[(long long)c * a.ldd + m] = __float2bfloat16_rn(tile[tx][i]);
-            else
-                static_cast<float*>(a.dst)[(long long)c * a.ldd + m] = tile[tx][i];
-        }
+    const int m = m0 + tx;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const int cc = c0 + ty + 8 * r;
+        if (m < a.M && cc < a.C) st_elem<DB>(a.dst, (long long)cc * a.ldd + m, tile[tx][ty + 8 * r]);
     }
+}
+
+template <int MODE>
+cudaError_t launch_transpose_mode(const TransposeArgs& a, dim3 grid, cudaStream_t s) {
+    if (a.src_bf16) {
+        if (a.dst_bf16) transpose_kernel<MODE, true, true><<<grid, 256, 0, s>>>(a);
+        else transpose_kernel<MODE, true, false><<<grid, 256, 0, s>>>(a);
+    } else {
+        if (a.dst_bf16) transpose_kernel<MODE, false, true><<<grid, 256, 0, s>>>(a);
+        else transpose_kernel<MODE, false, false><<<grid, 256, 0, s>>>(a);
+    }
+    return cudaGetLastError();
 }
 
 }  // namespace
@@ -578,8 +607,7 @@ __global__ void transpose_kernel(TransposeArgs a) {
 cudaError_t launch_transpose(const TransposeArgs& a, cudaStream_t s) {
     if (a.M <= 0 || a.C <= 0) return cudaSuccess;
     dim3 grid((a.M + 31) / 32, (a.C + 31) / 32);
-    transpose_kernel<<<grid, 256, 0, s>>>(a);
-    return cudaGetLastError();
+    return a.mode == 0 ? launch_transpose_mode<0>(a, grid, s) : launch_transpose_mode<1>(a, grid, s);
 }
 
 }  // namespace lstm
