@@ -550,43 +550,49 @@ __device__ __forceinline__ void st_elem(void* p, long long i, float v) {
         static_cast<float*>(p)[i] = v;
 }
 
-// 32 x 32 tiles, 32 x 8 threads: each thread's four source elements are all
-// loaded (predicated) before any goes to shared memory, so their latencies
-// overlap.
+// Tiles of 32 rows (m) x 64 columns (c), 32 x 8 threads: each thread's eight
+// source elements are all loaded (predicated) before any goes to shared
+// memory, so their latencies overlap.
+constexpr int kTrM = 32, kTrC = 64;
 template <int MODE, bool SB, bool DB>
 __global__ void __launch_bounds__(256) transpose_kernel(TransposeArgs a) {
-    __shared__ float tile[32][33];
-    const int m0 = blockIdx.x * 32, c0 = blockIdx.y * 32;
+    __shared__ float tile[kTrM][kTrC + 1];
+    const int m0 = blockIdx.x * kTrM, c0 = blockIdx.y * kTrC;
     const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 32 x 8 threads
-    const int c = c0 + tx;
-    float v[4];
+    float v[4][2];
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
         const int m = m0 + ty + 8 * r;
-        v[r] = 0.f;
-        if (m < a.M && c < a.C) {
-            if (MODE == 0) {
-                long long row = m;
-                if (a.bt_remap) row = (long long)(m % a.B) * a.T + m / a.B;   // m = t*B + b -> b*T + t
-                v[r] = ld_elem<SB>(a.src, row * a.lds + c);
-            } else {   // h_{t-1} in the direction's order, h0 at its first step
-                const int t = m / a.B, b = m % a.B;
-                const int ts = a.dir == 0 ? t - 1 : t + 1;
-                if (ts >= 0 && ts < a.T)
-                    v[r] = ld_elem<SB>(a.src, ((long long)ts * a.B + b) * a.lds + c);
-                else if (a.h0)
-                    v[r] = ld_elem<SB>(a.h0, (long long)b * a.C + c);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int c = c0 + 32 * h + tx;
+            v[r][h] = 0.f;
+            if (m < a.M && c < a.C) {
+                if (MODE == 0) {
+                    long long row = m;
+                    if (a.bt_remap) row = (long long)(m % a.B) * a.T + m / a.B;   // m = t*B + b -> b*T + t
+                    v[r][h] = ld_elem<SB>(a.src, row * a.lds + c);
+                } else {   // h_{t-1} in the direction's order, h0 at its first step
+                    const int t = m / a.B, b = m % a.B;
+                    const int ts = a.dir == 0 ? t - 1 : t + 1;
+                    if (ts >= 0 && ts < a.T)
+                        v[r][h] = ld_elem<SB>(a.src, ((long long)ts * a.B + b) * a.lds + c);
+                    else if (a.h0)
+                        v[r][h] = ld_elem<SB>(a.h0, (long long)b * a.C + c);
+                }
             }
         }
     }
 #pragma unroll
-    for (int r = 0; r < 4; ++r) tile[ty + 8 * r][tx] = v[r];
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) tile[ty + 8 * r][32 * h + tx] = v[r][h];
     __syncthreads();
     const int m = m0 + tx;
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        const int cc = c0 + ty + 8 * r;
-        if (m < a.M && cc < a.C) st_elem<DB>(a.dst, (long long)cc * a.ldd + m, tile[tx][ty + 8 * r]);
+    for (int r = 0; r < kTrC / 8; ++r) {
+        const int cl = ty + 8 * r, cc = c0 + cl;
+        if (m < a.M && cc < a.C) st_elem<DB>(a.dst, (long long)cc * a.ldd + m, tile[tx][cl]);
     }
 }
 
@@ -606,7 +612,7 @@ cudaError_t launch_transpose_mode(const TransposeArgs& a, dim3 grid, cudaStream_
 
 cudaError_t launch_transpose(const TransposeArgs& a, cudaStream_t s) {
     if (a.M <= 0 || a.C <= 0) return cudaSuccess;
-    dim3 grid((a.M + 31) / 32, (a.C + 31) / 32);
+    dim3 grid((a.M + kTrM - 1) / kTrM, (a.C + kTrC - 1) / kTrC);
     return a.mode == 0 ? launch_transpose_mode<0>(a, grid, s) : launch_transpose_mode<1>(a, grid, s);
 }
 
