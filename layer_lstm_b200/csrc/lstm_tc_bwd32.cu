@@ -402,6 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // gate gradients of the own cells: dG (standard row order) and the
             // exchange slot of iteration s + 1 (tf32 part | remainder, order 4u+q)
             float* dxo = a.dax + ((size_t)(d * kSlots + (s + 1) % kSlots) * B) * 2 * G + 4 * u;
+            float dak[kMaxCells][4];   // this step's gate gradients of the own cells
 #pragma unroll
             for (int k = 0; k < kMaxCells; ++k) {
                 const int idx = e + kEpi * k;
@@ -425,9 +426,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int g = 0; g < 4; ++g) dbs[g] += da[g];
                 }
-                float* dgp = a.dG + ((size_t)t * B + bb) * ldg + (size_t)d * G + u;
 #pragma unroll
-                for (int g = 0; g < 4; ++g) dgp[(size_t)g * H] = da[g];
+                for (int g = 0; g < 4; ++g) dak[k][g] = da[g];
                 float hi[4], lo[4];
 #pragma unroll
                 for (int g = 0; g < 4; ++g) {
@@ -440,10 +440,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             trace_mark(a.trace, tre, s, 7);
             // publish: the exchange writes before the group's TMA reads them
+            // (the fence waits for this thread's stores: only the exchange so far)
             tc::fence_proxy_async_global();
             tc::named_bar_sync(1, kEpi);
             if (e == 0) red_release_add(ctr, 1u);
             trace_mark(a.trace, tre, s + 1, 8);
+            // then dG, which only the weight phase reads
+#pragma unroll
+            for (int k = 0; k < kMaxCells; ++k) {
+                const int idx = e + kEpi * k;
+                const int b = idx / kOwn;
+                if (idx >= ncell || b >= nB) continue;
+                float* dgp = a.dG + ((size_t)t * B + b0 + b) * ldg + (size_t)d * G + u;
+#pragma unroll
+                for (int g = 0; g < 4; ++g) dgp[(size_t)g * H] = dak[k][g];
+            }
         }
         // bias-gradient partial of the own units over the group's rows, in a
         // fixed order over the threads that share a unit (e = ul + kOwn m)
