@@ -51,8 +51,8 @@ DevInfo device_info() {
 
 // Fault injection for the tests of the bounded waits (off unless set):
 // LSTM_B200_DEBUG_SKIP_ARRIVAL="fwd:<block>:<step>" or "bwd:<block>:<step>"
-// makes that block of every FFMA forward (backward) recurrent launch withhold
-// its arrival of that step, so the blocks of its group give up at their next
+// makes that block of every FFMA or float32 tensor-core forward (backward)
+// recurrent launch withhold its arrival of that step, so the blocks of its group give up at their next
 // counter wait (no copy is in flight there) and the call ends with
 // LSTM_ERR_TIMEOUT in the status word.
 struct SkipArrival {
@@ -831,6 +831,8 @@ lstm_status lstm_forward_varlen(const lstm_desc* desc, const int* lengths, const
             tr.timeout_ns = timeout_ns();
             tr.len = lengths;
             tr.trace = trace_for(LSTM_TRACE_FWD_REC_TC32, T, stream);
+            tr.skip_block = skip_arrival().fwd_block;
+            tr.skip_step = skip_arrival().fwd_step;
             LSTM_CUDA(timed(K_PACK, stream, [&] { return launch_rec32_slot0(tr, stream); }));
             int nl = 1;
             LSTM_CUDA(timed(K_FWD_REC_TC, stream, [&] { return launch_tc_rec32(tr, stream, &nl); }, &nl));
@@ -1164,6 +1166,8 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
             tb.timeout_ns = timeout_ns();
             tb.len = lengths;
             tb.trace = trace_for(LSTM_TRACE_BWD_REC_TC32, T, stream);
+            tb.skip_block = skip_arrival().bwd_block;
+            tb.skip_step = skip_arrival().bwd_step;
             int nl = 1, ndw = 0;
             LSTM_CUDA(timed(K_BWD_REC_TC, stream, [&] {
                 cudaError_t e = launch_tc_bwd32(tb, stream, &nl);

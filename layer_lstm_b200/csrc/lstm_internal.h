@@ -36,8 +36,8 @@ struct GemmArgs {
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s);
 
 // Tensor-core GEMM (tcgen05): C[M x N] = A[M x K] * B[N x K]^T (+ bias[n])
-// with both operands K-major (row strides lda, ldb elements, 16-byte
-// multiples).  F32 operands use 3xTF32, BF16 operands kind::f16; the
+// with each operand K-major, or MN-major when a_mn / b_mn (row strides lda,
+// ldb elements, 16-byte multiples).  F32 operands use 3xTF32, BF16 operands kind::f16; the
 // accumulator is float32.  Output column n < n_split goes to
 // C[row*ldc + n], n >= n_split to C1[row*ldc1 + n - n_split] (C1 null: all to
 // C).  Row map as in GemmArgs.  splitk > 1 needs ws (splitk*M*N floats).
@@ -206,6 +206,7 @@ struct TcRec32Args {
     uint64_t timeout_ns;
     const int* len;             // [B] valid steps per row, or null (all T)
     unsigned long long* trace;  // [kTraceSteps][kTraceEvents] or null
+    int skip_block, skip_step;  // fault injection: that block withholds that step's arrival (-1: none)
 };
 // Exchange slot 0 (hi | lo of h0, or zeros); precedes launch_tc_rec32.
 cudaError_t launch_rec32_slot0(const TcRec32Args& a, cudaStream_t s);
@@ -241,6 +242,7 @@ struct TcBwd32Args {
     uint64_t timeout_ns;
     const int* len;             // [B] valid steps per row, or null (all T)
     unsigned long long* trace;  // [kTraceSteps][kTraceEvents] or null
+    int skip_block, skip_step;  // fault injection: that block withholds that iteration's arrival (-1: none)
 };
 // *nlaunch (if given) = kernels launched.
 cudaError_t launch_tc_bwd32(const TcBwd32Args& a, cudaStream_t s, int* nlaunch = nullptr);

@@ -83,6 +83,7 @@ struct TcBwd32Params {
     uint64_t timeout_ns;
     const int* len;
     unsigned long long* trace;   // per-step timeline of block 0, or null
+    int skip_block, skip_step;   // fault injection (tests of the bounded waits), -1: none
 };
 
 __device__ __forceinline__ float tf32_hi(float x) { return __uint_as_float(__float_as_uint(x) & 0xFFFFE000u); }
@@ -443,7 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // (the fence waits for this thread's stores: only the exchange so far)
             tc::fence_proxy_async_global();
             tc::named_bar_sync(1, kEpi);
-            if (e == 0) red_release_add(ctr, 1u);
+            if (e == 0 && !((int)blockIdx.x == a.skip_block && s == a.skip_step)) red_release_add(ctr, 1u);
             trace_mark(a.trace, tre, s + 1, 8);
             // then dG, which only the weight phase reads
 #pragma unroll
@@ -581,6 +582,7 @@ cudaError_t launch_tc_bwd32(const TcBwd32Args& a, cudaStream_t s, int* nlaunch) 
     prm.ctr = a.ctr; prm.status = a.status; prm.timeout_ns = a.timeout_ns;
     prm.len = a.len;
     prm.trace = a.trace;
+    prm.skip_block = a.skip_block; prm.skip_step = a.skip_step;
     cudaLaunchConfig_t cfg;
     cudaLaunchAttribute attr[1];
     cudaError_t e = bwd32_config(p.Cl, p.smem, p.ctas, s, cfg, attr);

@@ -74,6 +74,7 @@ struct TcRec32Params {
     uint64_t timeout_ns;
     const int* len;
     unsigned long long* trace;   // per-step timeline of block 0, or null
+    int skip_block, skip_step;   // fault injection (tests of the bounded waits), -1: none
 };
 
 __device__ __forceinline__ float tf32_hi(float x) { return __uint_as_float(__float_as_uint(x) & 0xFFFFE000u); }
@@ -396,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // publish: the exchange writes before the group's TMA reads them
             tc::fence_proxy_async_global();
             tc::named_bar_sync(1, kEpi);
-            if (e == 0) red_release_add(ctr, 1u);
+            if (e == 0 && !((int)blockIdx.x == a.skip_block && s == a.skip_step)) red_release_add(ctr, 1u);
             trace_mark(a.trace, tre, s, 8);
         }
     }
@@ -487,6 +488,7 @@ cudaError_t launch_tc_rec32(const TcRec32Args& a, cudaStream_t s, int* nlaunch) 
     prm.h_n = a.h_n; prm.c_n = a.c_n; prm.act = a.act; prm.cst = a.cst;
     prm.ctr = a.ctr; prm.status = a.status; prm.timeout_ns = a.timeout_ns; prm.len = a.len;
     prm.trace = a.trace;
+    prm.skip_block = a.skip_block; prm.skip_step = a.skip_step;
     const auto kern = a.act ? tc_rec32_kernel<true> : tc_rec32_kernel<false>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
     if (e != cudaSuccess) return e;

@@ -1,4 +1,4 @@
-"""Bounded-wait failure path of the FFMA recurrences, run in a fresh process
+"""Bounded-wait failure path of the recurrences, run in a fresh process
 (the wait limit and the fault injection are read once per process).
 
 argv[1] = "fwd" or "bwd".  The environment sets LSTM_B200_WAIT_TIMEOUT_NS (a
@@ -24,11 +24,16 @@ def main():
     which = sys.argv[1]
     wl = Workload("to", L=1, D=1, I=32, H=256, T=8, B=8, dtype="f32", train=which == "bwd", seed=611)
     p = DeviceProblem(make_inputs(wl))
+    binding.lstm_timing_reset()
+    binding.lstm_timing_enable(True)
     binding.check(p.forward(), "lstm_forward")
     if which == "bwd":
         binding.check(p.backward(), "lstm_backward")
     st = p.status()
+    binding.lstm_timing_enable(False)
     print("status", binding.status_string(st))
+    # the recurrent kernels that ran (the engine under test)
+    print("kernels", " ".join(k for k, (n, _) in binding.lstm_timing_read().items() if n > 0 and "_rec_" in k))
     # the context is still usable: a plain torch computation and a sync
     v = float(torch.arange(10, device="cuda", dtype=torch.float32).sum().item())
     torch.cuda.synchronize()
