@@ -20,8 +20,10 @@
 // 4-7 drain the other accumulator through registers to global memory while
 // the next tile's MMAs run.  bf16 operands use kind::f16.  float32 operands use three
 // kind::tf32 products per K step, hi*hi + hi*lo + lo*hi with hi = x with its
-// low 13 mantissa bits cleared and lo = x - hi (exact in fp32); warps 2-3
-// split each stage in shared memory before the MMAs read it.  This is the
+// low 13 mantissa bits cleared and lo = x - hi (exact in fp32).  The stage's
+// float32 values are the hi operand as they stand (a tf32 MMA reads the top
+// 19 bits of each element); warps 2-3 write the lo tiles beside each stage
+// before the MMAs read it.  This is the
 // error-compensated 3xTF32 scheme of Ootomo & Yokota (2022), "Recovering
 // single precision accuracy from Tensor Cores while surpassing the FP32
 // theoretical peak performance"; the dropped lo*lo term and the truncation
@@ -280,18 +282,20 @@ __global__ void __launch_bounds__(threads_of<KIND>(), 1)
                     ok = false;
                     break;
                 }
-                float4* hi = reinterpret_cast<float4*>(smem + s * Cf::STAGE_BYTES);
+                // the stage's float32 values serve as the hi operand as they
+                // are (a tf32 MMA reads the top 19 bits of each); only the
+                // remainders are written
+                const float4* hi = reinterpret_cast<const float4*>(smem + s * Cf::STAGE_BYTES);
                 float4* lo = reinterpret_cast<float4*>(smem + s * Cf::STAGE_BYTES + Cf::A_BYTES + Cf::B_BYTES);
                 constexpr int NV = (Cf::A_BYTES + Cf::B_BYTES) / 16;
 #pragma unroll 4
                 for (int i = ct; i < NV; i += 64) {
                     const float4 x = hi[i];
-                    float4 h, l;
-                    h.x = __uint_as_float(__float_as_uint(x.x) & 0xFFFFE000u); l.x = x.x - h.x;
-                    h.y = __uint_as_float(__float_as_uint(x.y) & 0xFFFFE000u); l.y = x.y - h.y;
-                    h.z = __uint_as_float(__float_as_uint(x.z) & 0xFFFFE000u); l.z = x.z - h.z;
-                    h.w = __uint_as_float(__float_as_uint(x.w) & 0xFFFFE000u); l.w = x.w - h.w;
-                    hi[i] = h;
+                    float4 l;
+                    l.x = x.x - __uint_as_float(__float_as_uint(x.x) & 0xFFFFE000u);
+                    l.y = x.y - __uint_as_float(__float_as_uint(x.y) & 0xFFFFE000u);
+                    l.z = x.z - __uint_as_float(__float_as_uint(x.z) & 0xFFFFE000u);
+                    l.w = x.w - __uint_as_float(__float_as_uint(x.w) & 0xFFFFE000u);
                     lo[i] = l;
                 }
                 tc::fence_proxy_async_smem();
