@@ -11,9 +11,9 @@ all-reduces exactly as in the benchmark.  A second test checks that
 processes itself.
 """
 import os
-import socket
 import subprocess
 import sys
+import tempfile
 import types
 
 import numpy as np
@@ -29,23 +29,15 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 WL = Workload("dp", L=2, D=2, I=6, H=5, T=4, B=7, dtype="f32", state_std=0.3, train=True, seed=77)
 
 
-def _free_port():
-    s = socket.socket()
-    s.bind(("127.0.0.1", 0))
-    p = s.getsockname()[1]
-    s.close()
-    return p
-
-
 def _flat(r):
     return np.concatenate([a.ravel() for a in r["dw_ih"] + r["dw_hh"] + r["db_ih"]])
 
 
-def _worker(rank, world, port, q):
-    os.environ["MASTER_ADDR"] = "127.0.0.1"
-    os.environ["MASTER_PORT"] = str(port)
+def _worker(rank, world, rdzv, q):
     import datetime
-    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    # rendezvous through a file: no port that another process could take first
+    dist.init_process_group("gloo", init_method=f"file://{rdzv}", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
     import oracle
     oracle.set_num_threads(1)
     inp = make_inputs(WL)
@@ -78,8 +70,8 @@ def test_batch_sharded_gradients_allreduce():
     world = 2
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    rdzv = os.path.join(tempfile.mkdtemp(prefix="lstm_dp_"), "rdzv")
+    procs = [ctx.Process(target=_worker, args=(r, world, rdzv, q)) for r in range(world)]
     for p in procs:
         p.start()
     res = [q.get(timeout=120) for _ in range(world)]
