@@ -92,22 +92,10 @@ __device__ __forceinline__ float sel4(float a0, float a1, float a2, float a3, in
     return selp_f(lo, hi, (uint32_t)k & 2u);
 }
 
-// Gate nonlinearities of this bf16-only kernel: the hardware tanh
-// approximation (relative error near 2^-11, far inside the bf16 path's 2e-2
-// tolerance).
-__device__ __forceinline__ float tanh_fast(float z) {
-    float r;
-    asm("tanh.approx.f32 %0, %1;" : "=f"(r) : "f"(z));
-    return r;
-}
-
-// sigma(z) = (1 + tanh(z/2)) / 2: one special-function op instead of an
-// exponential and a reciprocal
-__device__ __forceinline__ float sigmoid_fast(float z) { return fmaf(0.5f, tanh_fast(0.5f * z), 0.5f); }
-
-// tanh of two values with one special-function op (f16x2: arguments and
-// results rounded to half precision, error near 2^-10 -- below the rounding
-// of h to bf16 that this path applies every step).
+// Gate nonlinearities of this bf16-only kernel: tanh of two values with one
+// special-function op (f16x2: arguments and results rounded to half
+// precision, error near 2^-10 -- below the rounding of h to bf16 that this
+// path applies every step).
 __device__ __forceinline__ float2 tanh2(float a, float b) {
     const __half2 x = __floats2half2_rn(a, b);
     uint32_t r;
