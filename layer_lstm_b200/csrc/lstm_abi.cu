@@ -799,18 +799,27 @@ lstm_status lstm_forward_varlen(const lstm_desc* desc, const int* lengths, const
 
         void* hseq_tc = reserve ? P(reserve, l.hseq[k]) : P(workspace, l.seq[k & 1]);
         if (tc_path && l.tc32.ok) {
-            // float32 tensor-core recurrence (3xTF32): packed W_hh rows in
-            // float32; the launcher fills exchange slot 0 from h0
-            PackIhArgs pw{};
-            pw.H = H; pw.in = H; pw.D = D; pw.dt = l.dt;
-            for (int d = 0; d < D; ++d) pw.w[d] = w_hh[k * D + d];
-            pw.wp = P(workspace, l.whh_tc);
-            pw.bias_p = reinterpret_cast<float*>(P(workspace, l.bias_dummy));
-            LSTM_CUDA(timed(K_PACK, stream, [&] { return launch_pack_ih(pw, stream); }));
+            // float32 tensor-core recurrence (3xTF32): the kernel reads W_hh
+            // as given (its gate-major rows are the order it keeps in tensor
+            // memory) when every direction's pointer is 16-byte aligned, else a
+            // packed copy; the launcher fills exchange slot 0 from h0
             TcRec32Args tr{};
             tr.H = H; tr.B = B; tr.T = T; tr.D = D; tr.p = l.tc32;
             tr.gx = reinterpret_cast<const float*>(P(workspace, l.gx));
-            tr.wpk = reinterpret_cast<const float*>(P(workspace, l.whh_tc));
+            bool w_direct = true;
+            for (int d = 0; d < D; ++d) {
+                tr.w[d] = static_cast<const float*>(w_hh[k * D + d]);
+                w_direct = w_direct && (reinterpret_cast<uintptr_t>(w_hh[k * D + d]) & 15) == 0;
+            }
+            if (!w_direct) {
+                PackIhArgs pw{};
+                pw.H = H; pw.in = H; pw.D = D; pw.dt = l.dt;
+                for (int d = 0; d < D; ++d) pw.w[d] = w_hh[k * D + d];
+                pw.wp = P(workspace, l.whh_tc);
+                pw.bias_p = reinterpret_cast<float*>(P(workspace, l.bias_dummy));
+                LSTM_CUDA(timed(K_PACK, stream, [&] { return launch_pack_ih(pw, stream); }));
+                tr.wpk = reinterpret_cast<const float*>(P(workspace, l.whh_tc));
+            }
             tr.h0 = h0 ? static_cast<const float*>(h0) + (size_t)k * state_elems : nullptr;
             tr.c0 = c0 ? c0 + (size_t)k * state_elems : nullptr;
             tr.hx = reinterpret_cast<float*>(P(workspace, l.hx32));

@@ -193,7 +193,8 @@ struct TcRec32Args {
     int H, B, T, D;
     TcRec32Plan p;
     const float* gx;            // [T][B][D*4H] packed rows 4u+q, biases included
-    const float* wpk;           // [D*4H][H] W_hh packed rows 4u+q, float32
+    const float* wpk;           // [D*4H][H] W_hh packed rows 4u+q, float32, or null: read w
+    const float* w[2];          // W_hh of each direction as given ([4H][H], rows q*H + u), 16-byte aligned
     const float* h0;            // [D][B][H] or null
     const float* c0;            // [D][B][H] or null
     float* hx;                  // exchange [D][T+1][B][2H]: tf32 hi | remainder of h (slot 0 = h0)

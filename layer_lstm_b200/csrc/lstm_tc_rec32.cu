@@ -62,7 +62,8 @@ struct TcRec32Params {
     int nbg, Bg, N, nsl, C, KP;
     int d0;                    // first direction of this launch
     const float* gx;
-    const float* wpk;
+    const float* wpk;          // packed rows 4u+q, or null: W_hh of each direction as given
+    const float* w[2];
     const float* c0;
     float* hx;
     float* hseq;
@@ -162,7 +163,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // tf32 per column; hi at columns kAcol + k, the remainder at kAcol + KP + k.
     if (warp == 0 && lane == 0) tc::prefetch_tmap(&tmX);
     if (warp > kIss && half == 0) {
-        const float* wrow = a.wpk + (size_t)(prow0 + 4 * (r & 31) + (r >> 5)) * H + kbeg;
+        // gate r / 32 of unit 32j + r % 32: packed row 4u + q, or row q*H + u of W_hh as given
+        const float* wrow = a.wpk ? a.wpk + (size_t)(prow0 + 4 * (r & 31) + (r >> 5)) * H + kbeg
+                                  : a.w[d] + ((size_t)(r >> 5) * H + 32 * j + (r & 31)) * H + kbeg;
         for (int c = 0; c < nkc; ++c) {
 #pragma unroll
             for (int h16 = 0; h16 < 2; ++h16) {
@@ -483,7 +486,7 @@ cudaError_t launch_tc_rec32(const TcRec32Args& a, cudaStream_t s, int* nlaunch) 
     TcRec32Params prm{};
     prm.H = a.H; prm.B = a.B; prm.T = a.T; prm.D = a.D;
     prm.nbg = p.nbg; prm.Bg = p.Bg; prm.N = p.N; prm.nsl = p.nsl; prm.C = p.C; prm.KP = p.KP;
-    prm.gx = a.gx; prm.wpk = a.wpk; prm.c0 = a.c0; prm.hx = a.hx;
+    prm.gx = a.gx; prm.wpk = a.wpk; prm.w[0] = a.w[0]; prm.w[1] = a.w[1]; prm.c0 = a.c0; prm.hx = a.hx;
     prm.hseq = a.hseq; prm.out = a.out; prm.out_st = a.out_st; prm.out_sb = a.out_sb;
     prm.h_n = a.h_n; prm.c_n = a.c_n; prm.act = a.act; prm.cst = a.cst;
     prm.ctr = a.ctr; prm.status = a.status; prm.timeout_ns = a.timeout_ns; prm.len = a.len;
