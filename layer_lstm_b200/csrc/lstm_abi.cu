@@ -250,7 +250,7 @@ struct Layout {
     TcRec32Plan tc32;  // tensor-core forward recurrence for float32 (3xTF32), if it fits
     size_t ctr_tc32, hx32;
     TcBwd32Plan tcb32; // tensor-core BPTT recurrence for float32 (3xTF32), if it fits
-    size_t ctr_tcb32, dax32, wT32;
+    size_t ctr_tcb32, dax32;
     size_t status, ctr_f, ctr_b, ctr_tc, ctr_end, wih[32], bias[32], whh_f, whh_b, gx, hT, seq[2], dG, dseq[2], xt,
         dbpart, P, dGT, bop, wcatT, hx, whh_tc, bias_dummy, gemm_ws, total;
     size_t gemm_ws_floats;
@@ -374,8 +374,7 @@ bool make_layout(const lstm_desc* d, Layout& l) {
     // tensor-core BPTT: packed W_hh^T and the bf16 exchange of the gate gradients
     l.wT_tcb = o; o += al(l.tcb.ok ? (size_t)l.D * l.H * l.G * 2 : 0);
     l.dax = o; o += al(l.tcb.ok ? (size_t)l.D * (l.T + 1) * l.B * l.G * 2 : 0);
-    // float32 tensor-core BPTT: packed W_hh^T and the ring of split gate gradients
-    l.wT32 = o; o += al(l.tcb32.ok ? (size_t)l.D * l.H * l.G * 4 : 0);
+    // float32 tensor-core BPTT: the ring of split gate gradients
     l.dax32 = o; o += al(l.tcb32.ok ? (size_t)l.D * l.tcb32.slots * l.B * 2 * l.G * 4 : 0);
     l.P = o; o += al(l.bwd_ok ? (size_t)2 * l.D * l.bwd.nbg * l.bwd.nu * l.bwd.Bg * Hp * 4 : 0);
     l.dGT = o; o += al(TB * l.D * l.G * 4);
@@ -1156,14 +1155,9 @@ lstm_status lstm_backward_varlen(const lstm_desc* desc, const int* lengths, cons
             int nl = 1;
             LSTM_CUDA(timed(K_BWD_REC_TC, stream, [&] { return launch_tc_bwd(tb, stream, &nl); }, &nl));
         } else if (tcb32) {
-            PackWtArgs pw{};
-            pw.H = H; pw.D = D; pw.dt = DType::F32;
-            for (int d = 0; d < D; ++d) pw.w[d] = w_hh[k * D + d];
-            pw.out = P(workspace, l.wT32);
-            LSTM_CUDA(timed(K_PACK, stream, [&] { return launch_pack_wT(pw, stream); }));
             TcBwd32Args tb{};
             tb.H = H; tb.B = B; tb.T = T; tb.D = D; tb.p = l.tcb32;
-            tb.wT = reinterpret_cast<const float*>(pw.out);
+            for (int d = 0; d < D; ++d) tb.w[d] = static_cast<const float*>(w_hh[k * D + d]);   // read as given
             tb.act = b.act; tb.cst = b.cst; tb.c0 = b.c0;
             tb.dy = b.dy; tb.dy_st = b.dy_st; tb.dy_sb = b.dy_sb;
             tb.grad_hn = b.grad_hn; tb.grad_cn = b.grad_cn;

@@ -227,7 +227,7 @@ TcBwd32Plan plan_tc_bwd32(int H, int B, int D, int num_sms, size_t smem_max);
 struct TcBwd32Args {
     int H, B, T, D;
     TcBwd32Plan p;
-    const float* wT;            // [D][H][4H] packed W_hh^T (launch_pack_wT, float32)
+    const float* w[2];          // W_hh of each direction as given, [4H][H] float32
     const float* act;           // [D][T][B][4H] saved gate activations (i, f, g, o per unit)
     const float* cst;           // [D][T][B][H] saved cell states
     const float* c0;            // [D][B][H] or null

@@ -67,7 +67,7 @@ struct TcBwd32Params {
     int H, B, T, D;
     int nbg, Bg, N, nsl, Cl;
     int g0;                    // first (direction, batch group) d * nbg + bg of this launch
-    const float* wT;           // [D][H][4H] W_hh^T, column 4u'+q = W_hh[q*H + u'][u]
+    const float* w[2];         // W_hh of each direction as given, [4H][H]: W_hh^T[u][4u'+q] = w[(q*H + u')*H + u]
     const float* act;
     const float* cst;
     const float* c0;
@@ -167,21 +167,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     // kAcol + kKP + k.
     if (warp == 0 && lane == 0) tc::prefetch_tmap(&tmD);
     if (warp > kIss && half == 0) {
-        const float* wrow = a.wT + ((size_t)d * H + u0 + r) * G + kbeg;
+        // W_hh^T[u][g] for gate g = 4u' + q is W_hh[q*H + u'][u]: a warp's 32
+        // lanes (consecutive u) read 128 contiguous bytes per element
+        const float* wcol = a.w[d] + u0 + r;
         for (int c = 0; c < nkc; ++c) {
 #pragma unroll
             for (int h16 = 0; h16 < 2; ++h16) {
                 uint32_t vh[16], vl[16];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float4 w4 = *reinterpret_cast<const float4*>(wrow + 32 * c + 16 * h16 + 4 * i);
-                    const float w[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-                    for (int x = 0; x < 4; ++x) {
-                        const float hi = tf32_hi(w[x]);
-                        vh[4 * i + x] = __float_as_uint(hi);
-                        vl[4 * i + x] = __float_as_uint(w[x] - hi);
-                    }
+                for (int i = 0; i < 16; ++i) {
+                    const int g = kbeg + 32 * c + 16 * h16 + i;
+                    const float w = wcol[(size_t)((g & 3) * H + (g >> 2)) * H];
+                    const float hi = tf32_hi(w);
+                    vh[i] = __float_as_uint(hi);
+                    vl[i] = __float_as_uint(w - hi);
                 }
                 tc::tmem_st16(trow + kAcol + (uint32_t)(32 * c + 16 * h16), vh);
                 tc::tmem_st16(trow + kAcol + (uint32_t)(kKP + 32 * c + 16 * h16), vl);
@@ -573,7 +572,7 @@ cudaError_t launch_tc_bwd32(const TcBwd32Args& a, cudaStream_t s, int* nlaunch) 
     prm.H = a.H; prm.B = a.B; prm.T = a.T; prm.D = a.D;
     prm.nbg = p.nbg; prm.Bg = p.Bg; prm.N = p.N; prm.nsl = p.nsl; prm.Cl = p.Cl;
     prm.g0 = 0;
-    prm.wT = a.wT;
+    prm.w[0] = a.w[0]; prm.w[1] = a.w[1];
     prm.act = a.act; prm.cst = a.cst; prm.c0 = a.c0;
     prm.dy = a.dy; prm.dy_st = a.dy_st; prm.dy_sb = a.dy_sb;
     prm.grad_hn = a.grad_hn; prm.grad_cn = a.grad_cn;
