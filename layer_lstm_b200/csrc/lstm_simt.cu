@@ -112,19 +112,18 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
 // ==================================================================  packing
 namespace {
 
+// One block per packed row (grid-stride over rows), its threads over the
+// row's contiguous columns: no per-element division.
 template <typename T>
 __global__ void pack_ih_kernel(PackIhArgs a) {
     const int G = 4 * a.H;
-    const long long total = (long long)a.D * G * a.in;
-    T* wp = static_cast<T*>(a.wp);
-    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
-         e += (long long)gridDim.x * blockDim.x) {
-        const int k = (int)(e % a.in);
-        const long long row = e / a.in;
-        const int d = (int)(row / G), p = (int)(row % G);
+    for (int row = blockIdx.x; row < a.D * G; row += gridDim.x) {
+        const int d = row / G, p = row - d * G;
         const int src = (p & 3) * a.H + (p >> 2);
-        wp[e] = static_cast<const T*>(a.w[d])[(long long)src * a.in + k];
-        if (k == 0) {
+        const T* w = static_cast<const T*>(a.w[d]) + (size_t)src * a.in;
+        T* wp = static_cast<T*>(a.wp) + (size_t)row * a.in;
+        for (int k = threadIdx.x; k < a.in; k += blockDim.x) wp[k] = w[k];
+        if (threadIdx.x == 0) {
             float b = 0.f;
             if (a.b_ih[d]) b += to_f(static_cast<const T*>(a.b_ih[d])[src]);
             if (a.b_hh[d]) b += to_f(static_cast<const T*>(a.b_hh[d])[src]);
@@ -162,11 +161,13 @@ inline int grid_for(long long total) {
 }  // namespace
 
 cudaError_t launch_pack_ih(const PackIhArgs& a, cudaStream_t s) {
-    const long long total = (long long)a.D * 4 * a.H * a.in;
+    const int rows = a.D * 4 * a.H;
+    if (rows <= 0) return cudaSuccess;
+    const int grid = std::min(rows, 148 * 16);
     if (a.dt == DType::F32)
-        pack_ih_kernel<float><<<grid_for(total), 256, 0, s>>>(a);
+        pack_ih_kernel<float><<<grid, 256, 0, s>>>(a);
     else
-        pack_ih_kernel<bf16><<<grid_for(total), 256, 0, s>>>(a);
+        pack_ih_kernel<bf16><<<grid, 256, 0, s>>>(a);
     return cudaGetLastError();
 }
 
@@ -191,17 +192,17 @@ __global__ void db_reduce_kernel(DbArgs a) {
     a.db_hh[d][r] = sum;
 }
 
+// One block per (t, b) row (grid-stride over rows), its threads over the
+// row's W contiguous elements: no per-element division.
 template <typename T>
 __global__ void seq_copy_kernel(SeqCopyArgs a) {
-    const long long total = (long long)a.T * a.B * a.W;
     const T* src = static_cast<const T*>(a.src);
     T* dst = static_cast<T*>(a.dst);
-    for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
-         e += (long long)gridDim.x * blockDim.x) {
-        const int w = (int)(e % a.W);
-        const long long tb = e / a.W;
-        const int b = (int)(tb % a.B), t = (int)(tb / a.B);
-        dst[t * a.d_st + b * a.d_sb + w] = src[t * a.s_st + b * a.s_sb + w];
+    for (int tb = blockIdx.x; tb < a.T * a.B; tb += gridDim.x) {
+        const int t = tb / a.B, b = tb - t * a.B;
+        const T* s = src + t * a.s_st + b * a.s_sb;
+        T* o = dst + t * a.d_st + b * a.d_sb;
+        for (int w = threadIdx.x; w < a.W; w += blockDim.x) o[w] = s[w];
     }
 }
 
@@ -281,12 +282,13 @@ cudaError_t launch_db_reduce(const DbArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_seq_copy(const SeqCopyArgs& a, cudaStream_t s) {
-    const long long total = (long long)a.T * a.B * a.W;
-    if (total <= 0) return cudaSuccess;
+    const long long rows = (long long)a.T * a.B;
+    if (rows <= 0 || a.W <= 0) return cudaSuccess;
+    const int grid = (int)std::min<long long>(rows, 148LL * 16);
     if (a.dt == DType::F32)
-        seq_copy_kernel<float><<<grid_for(total), 256, 0, s>>>(a);
+        seq_copy_kernel<float><<<grid, 256, 0, s>>>(a);
     else
-        seq_copy_kernel<bf16><<<grid_for(total), 256, 0, s>>>(a);
+        seq_copy_kernel<bf16><<<grid, 256, 0, s>>>(a);
     return cudaGetLastError();
 }
 

@@ -83,17 +83,17 @@ __device__ __forceinline__ float tf32_hi(float x) { return __uint_as_float(__flo
 __device__ __forceinline__ float sigmoid_f(float z) { return 1.0f / (1.0f + expf(-z)); }
 
 // Exchange slot 0 from h0 (float32 [D][B][H]) or zeros: hi | lo per row.
+// One block per (d, b) row, its threads over the row's units.
 __global__ void rec32_slot0_kernel(const float* h0, float* hx, int D, int T, int B, int H) {
-    const long long n = (long long)D * B * H;
-    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
-        const int u = (int)(i % H);
-        const long long db = i / H;   // d * B + b
-        const int d = (int)(db / B), b = (int)(db % B);
-        const float h = h0 ? h0[i] : 0.f;
-        const float hi = tf32_hi(h);
+    for (int db = blockIdx.x; db < D * B; db += gridDim.x) {
+        const int d = db / B, b = db - d * B;
         float* row = hx + ((size_t)d * (T + 1) * B + b) * 2 * H;
-        row[u] = hi;
-        row[H + u] = h - hi;
+        for (int u = threadIdx.x; u < H; u += blockDim.x) {
+            const float h = h0 ? h0[(size_t)db * H + u] : 0.f;
+            const float hi = tf32_hi(h);
+            row[u] = hi;
+            row[H + u] = h - hi;
+        }
     }
 }
 
@@ -468,9 +468,7 @@ bool make_map_f32_chunks(CUtensorMap* map, const void* base, long long rows, lon
 
 cudaError_t launch_rec32_slot0(const TcRec32Args& a, cudaStream_t s) {
     if (a.T <= 0 || a.B <= 0) return cudaSuccess;
-    const long long n0 = (long long)a.D * a.B * a.H;
-    rec32_slot0_kernel<<<(int)std::min<long long>((n0 + 255) / 256, 4096), 256, 0, s>>>(a.h0, a.hx, a.D, a.T, a.B,
-                                                                                        a.H);
+    rec32_slot0_kernel<<<std::min(a.D * a.B, 148 * 16), 256, 0, s>>>(a.h0, a.hx, a.D, a.T, a.B, a.H);
     return cudaGetLastError();
 }
 
