@@ -153,7 +153,8 @@ lstm_status lstm_forward(const lstm_desc* desc, const void* x, const void* h0, c
  * LSTM_F32 computes in float32: 3xTF32 tensor-core products in the weight
  * phase and, where a tensor-core plan fits (H = 128, 256 or 512, batch groups
  * of at most 64 rows), in the recurrent products W_hh^T da too (operands
- * split as in the forward); gate derivatives, carries and sums in float32.  LSTM_BF16 keeps the cell arithmetic, the dc carry and every sum in
+ * split as in the forward); gate derivatives, carries and sums in float32.
+ * LSTM_BF16 keeps the cell arithmetic, the dc carry and every sum in
  * float32, with bf16 products on the tensor cores: the recurrent products
  * W_hh^T da take the previous step's gate gradients rounded to bf16, and the
  * weight phase takes the gate gradients rounded to bf16 (x, the saved layer
@@ -241,7 +242,11 @@ lstm_status lstm_noalloc_query_status(cudaStream_t stream);
 
 /* Synchronises `stream` and returns the kernel-side status recorded in
  * `workspace` by the last call that used it (LSTM_OK or LSTM_ERR_TIMEOUT), or
- * LSTM_ERR_CUDA if the stream reports an error. */
+ * LSTM_ERR_CUDA if the stream reports an error.  A kernel's inter-block or
+ * barrier wait gives up after 2 s, or after LSTM_B200_WAIT_TIMEOUT_NS
+ * nanoseconds when that environment variable is set (read once per
+ * process); the kernel then records LSTM_ERR_TIMEOUT, drains the copies it
+ * has in flight and returns, leaving the CUDA context usable. */
 lstm_status lstm_query_status(void* workspace, cudaStream_t stream);
 
 /* Static string naming a status code. */
