@@ -23,7 +23,8 @@
 // low 13 mantissa bits cleared and lo = x - hi (exact in fp32).  The stage's
 // float32 values are the hi operand as they stand (a tf32 MMA reads the top
 // 19 bits of each element); warps 2-3 write the lo tiles beside each stage
-// before the MMAs read it.  This is the
+// while the hi*hi MMAs of the stage run, and the two cross products follow
+// once the lo tiles are in place.  This is the
 // error-compensated 3xTF32 scheme of Ootomo & Yokota (2022), "Recovering
 // single precision accuracy from Tensor Cores while surpassing the FP32
 // theoretical peak performance"; the dropped lo*lo term and the truncation
@@ -230,8 +231,7 @@ __global__ void __launch_bounds__(threads_of<KIND>(), 1)
                 const uint32_t acc_t = tmem + (uint32_t)(ab * Cf::MH * BN);
                 for (int kt = 0; kt < c.nk; ++kt, ++it) {
                     const int s = it % S, r = it / S;
-                    uint64_t* ready = kTf32 ? &lofull[s] : &full[s];
-                    if (!tc::mbar_wait(ready, r & 1, abort_flag, e.status, e.timeout_ns)) {
+                    if (!tc::mbar_wait(&full[s], r & 1, abort_flag, e.status, e.timeout_ns)) {
                         ok = false;
                         break;
                     }
@@ -239,26 +239,37 @@ __global__ void __launch_bounds__(threads_of<KIND>(), 1)
                     unsigned char* st = smem + s * Cf::STAGE_BYTES;
                     const uint32_t a_base = tc::smem_u32(st);
                     const uint32_t b_base = a_base + Cf::A_BYTES;
+                    if constexpr (!kTf32) {
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const uint64_t ad = opd(a_base, j, amn);
-                        const uint64_t bd = opd(b_base, j, bmn);
-                        const uint32_t acc = (kt | j) != 0;
-                        if (!kTf32) {
+                        for (int j = 0; j < 4; ++j) {
+                            const uint64_t bd = opd(b_base, j, bmn);
+                            const uint32_t acc = (kt | j) != 0;
                             // rows [128h, 128h + 128) of the tile: 16 KB further in
                             // either layout (128 K-major rows, or two MN blocks)
 #pragma unroll
                             for (int h = 0; h < Cf::MH; ++h)
                                 tc::mma_bf16(acc_t + (uint32_t)(h * BN), opd(a_base + h * 16384, j, amn), bd, idesc,
                                              acc);
-                            (void)ad;
-                        } else {
-                            const uint32_t lo_off = Cf::A_BYTES + Cf::B_BYTES;
-                            const uint64_t adl = opd(a_base + lo_off, j, amn);
-                            const uint64_t bdl = opd(b_base + lo_off, j, bmn);
-                            tc::mma_tf32(acc_t, adl, bd, idesc, acc);   // lo * hi
-                            tc::mma_tf32(acc_t, ad, bdl, idesc, 1);     // hi * lo
-                            tc::mma_tf32(acc_t, ad, bd, idesc, 1);      // hi * hi
+                        }
+                    } else {
+                        // hi * hi reads only what the TMA wrote, so it runs
+                        // while the split warps write the remainders
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            tc::mma_tf32(acc_t, opd(a_base, j, amn), opd(b_base, j, bmn), idesc, (kt | j) != 0);
+                        if (!tc::mbar_wait(&lofull[s], r & 1, abort_flag, e.status, e.timeout_ns)) {
+                            tc::mma_commit(&empty[s]);   // the drain below waits for the products issued
+                            last = it;
+                            ok = false;
+                            break;
+                        }
+                        tc::tc_fence_after();
+                        const uint32_t lo_off = Cf::A_BYTES + Cf::B_BYTES;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const uint64_t ad = opd(a_base, j, amn), bd = opd(b_base, j, bmn);
+                            tc::mma_tf32(acc_t, opd(a_base + lo_off, j, amn), bd, idesc, 1);   // lo * hi
+                            tc::mma_tf32(acc_t, ad, opd(b_base + lo_off, j, bmn), idesc, 1);   // hi * lo
                         }
                     }
                     tc::mma_commit(&empty[s]);
